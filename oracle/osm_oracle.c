@@ -1,0 +1,512 @@
+/*
+ * Reference oracle for the smoothed, outlier-split W4A4 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is a plain, slow, single-purpose CPU
+ * restatement of what the layer computes, written from the method's
+ * description in "W4A4 Quantization for Inference on Wan2.2-I2V-A14B"
+ * (ICME 2026 challenge paper) and from the OCP Microscaling (MX) v1.0
+ * definition of MXFP4. Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load it. It shares no code, header,
+ * table or constant generator with the CUDA library.
+ *
+ * Conventions (each one is a reading of the paper; the list of readings is
+ * kept with the design notes):
+ *   - BF16 values travel as uint16 bit patterns; FP32 arithmetic is IEEE
+ *     single precision, round-to-nearest-even, no contraction
+ *     (compiled with -ffp-contract=off).
+ *   - Accumulation of the dual-branch product is in FP64; every product of
+ *     two dequantised 4-bit values (times their power-of-two scales) or of
+ *     two BF16 values is exact in FP64.
+ *   - J (bulk channels) and O (outlier channels) are both in ascending
+ *     original channel order; bulk blocks of 32 run over the compacted
+ *     bulk index p = 0..Kb-1.
+ *   - Kbp = Kb rounded up to 128, kp = k rounded up to 64; padded
+ *     positions hold code 0 / BF16 zero, and a 32-block with no real
+ *     element gets scale code 0.
+ *
+ * Parity pins: see tests/test_oracle_*.py. Every function below is pinned
+ * except the tanh-form GELU, which is pinned only against libm's tanh
+ * within a stated error bound.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+
+/* ------------------------------------------------------------------ */
+/* Scalar helpers                                                       */
+/* ------------------------------------------------------------------ */
+
+static float u32_as_f32(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t f32_as_u32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* BF16 is the upper half of an IEEE binary32 word. */
+double oracle_bf16_to_f64(uint16_t h) { return (double)u32_as_f32((uint32_t)h << 16); }
+float oracle_bf16_to_f32(uint16_t h) { return u32_as_f32((uint32_t)h << 16); }
+
+/*
+ * Round a binary32 value to the nearest BF16 value, ties to the even
+ * significand (IEEE 754 roundTiesToEven). Written from the definition:
+ * take the two BF16 neighbours of |f| (truncation and the next value up),
+ * pick the nearer, and on a tie the one whose last significand bit is 0.
+ * Overflow follows IEEE: the value just above the largest finite BF16 is
+ * treated as 2^128 when measuring distance.
+ */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u = f32_as_u32(f);
+    uint32_t sign = u & 0x80000000u;
+    uint32_t mag = u & 0x7FFFFFFFu;
+    if (mag > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u); /* NaN stays NaN (quiet) */
+    if (mag == 0x7F800000u) return (uint16_t)(u >> 16);              /* +-inf */
+    uint16_t lo = (uint16_t)(mag >> 16);         /* truncation toward zero */
+    uint16_t hi = (uint16_t)(lo + 1);            /* next magnitude up */
+    double v = (double)u32_as_f32(mag);
+    double vlo = oracle_bf16_to_f64(lo);
+    double vhi = (hi == 0x7F80u) ? ldexp(1.0, 128) : oracle_bf16_to_f64(hi);
+    double dlo = v - vlo, dhi = vhi - v;
+    uint16_t pick;
+    if (dlo < dhi) pick = lo;
+    else if (dhi < dlo) pick = hi;
+    else pick = (lo & 1u) ? hi : lo;
+    return (uint16_t)(pick | (sign >> 16));
+}
+
+/* Round an FP64 value to binary32 (C conversion is round-to-nearest-even). */
+float oracle_f64_to_f32(double v) { return (float)v; }
+
+/* ------------------------------------------------------------------ */
+/* OCP MXFP4: E2M1 elements with one E8M0 scale per block               */
+/* ------------------------------------------------------------------ */
+
+/* The eight non-negative E2M1 magnitudes, indexed by the 3-bit code
+ * (exponent bias 1, one mantissa bit, no inf/NaN). */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_decode(uint8_t code)
+{
+    double m = E2M1_MAG[code & 7u];
+    return (code & 8u) ? -m : m;
+}
+
+/*
+ * Encode one real value v (already divided by the block scale) to E2M1:
+ * nearest representable magnitude, ties to the even code (last mantissa
+ * bit 0), magnitudes above 6 saturate to 6. The sign bit copies the sign
+ * of v, so -0 and small negatives that round to zero give code 0x8.
+ */
+uint8_t oracle_e2m1_encode(double v, int negative)
+{
+    double a = fabs(v);
+    int best = 0;
+    double bestd = fabs(a - E2M1_MAG[0]);
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(a - E2M1_MAG[c]);
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return (uint8_t)(best | (negative ? 8 : 0));
+}
+
+/*
+ * Shared-scale exponent of an MX block (OCP MX v1.0 conversion rule):
+ * X = floor(log2(amax)) - emax, with emax = 2 for E2M1, clamped to the
+ * E8M0 range [-127, 127]. A block whose amax is 0 gets X = -127.
+ * Returns X; the stored E8M0 code is X + 127.
+ */
+int oracle_mx_scale_exponent(double amax)
+{
+    if (!(amax > 0.0)) return -127;
+    int e;
+    (void)frexp(amax, &e);        /* amax = m * 2^e, m in [0.5, 1) */
+    int X = (e - 1) - 2;          /* floor(log2 amax) - emax */
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    return X;
+}
+
+/* Quantise n values (given as BF16 words) with shared exponent X.
+ * Writes one 4-bit code per value into codes[]. */
+static void mx_encode_values(const uint16_t* v16, int n, int X, uint8_t* codes)
+{
+    double inv = ldexp(1.0, -X);
+    for (int i = 0; i < n; ++i) {
+        double v = oracle_bf16_to_f64(v16[i]);
+        int neg = (v16[i] & 0x8000u) != 0;
+        codes[i] = oracle_e2m1_encode(v * inv, neg);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Sizes                                                                */
+/* ------------------------------------------------------------------ */
+
+static int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+int64_t oracle_kbp(int64_t K, int64_t k) { return round_up(K - k, 128); }
+int64_t oracle_kp(int64_t k) { return round_up(k, 64); }
+
+/* ------------------------------------------------------------------ */
+/* Calibration: Eq. (2) and Eq. (4)                                     */
+/* ------------------------------------------------------------------ */
+
+/* act_scale_j = max_t |x_tj| over calibration tokens (Eq. (4) score and the
+ * activation statistic of Eq. (2)). X is [T][K] BF16, row-major. */
+void oracle_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax)
+{
+    for (int64_t j = 0; j < K; ++j) amax[j] = 0.0f;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float a = fabsf(oracle_bf16_to_f32(X[t * K + j]));
+            if (a > amax[j]) amax[j] = a;
+        }
+}
+
+/* weight_scale_j = max_n |W_jn|: the range of input channel j of W [K][N]. */
+void oracle_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax)
+{
+    for (int64_t j = 0; j < K; ++j) {
+        float m = 0.0f;
+        for (int64_t n = 0; n < N; ++n) {
+            float a = fabsf(oracle_bf16_to_f32(W[j * N + n]));
+            if (a > m) m = a;
+        }
+        wmax[j] = m;
+    }
+}
+
+static const int64_t* g_sort_keys_idx;
+static const float* g_sort_amax;
+static int cmp_score_desc(const void* pa, const void* pb)
+{
+    int64_t a = *(const int64_t*)pa, b = *(const int64_t*)pb;
+    float sa = g_sort_amax[a], sb = g_sort_amax[b];
+    if (sa > sb) return -1;
+    if (sa < sb) return 1;
+    return (a < b) ? -1 : (a > b);
+}
+static int cmp_i32(const void* pa, const void* pb)
+{
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a > b) - (a < b);
+}
+
+/*
+ * Eq. (2): s_j = act_scale_j^alpha / weight_scale_j^(1-alpha), evaluated in
+ * FP64 with both statistics floored at 1e-5, then rounded to FP32;
+ * inv_s_j = 1/s_j in FP32. Eq. (4): O = the k channels with the largest
+ * act_scale (ties: lower channel index first), returned ascending.
+ * Returns 0, or 1 if a statistic is not finite.
+ */
+int oracle_calibrate(const float* amax, const float* wmax, int64_t K, float alpha,
+                     int64_t k, float* s, float* inv_s, int32_t* O)
+{
+    for (int64_t j = 0; j < K; ++j)
+        if (!isfinite(amax[j]) || !isfinite(wmax[j])) return 1;
+    double a = (double)alpha;
+    for (int64_t j = 0; j < K; ++j) {
+        double am = (double)amax[j] < 1e-5 ? 1e-5 : (double)amax[j];
+        double wm = (double)wmax[j] < 1e-5 ? 1e-5 : (double)wmax[j];
+        double sj = pow(am, a) / pow(wm, 1.0 - a);
+        s[j] = (float)sj;
+        inv_s[j] = 1.0f / s[j];
+    }
+    if (k > 0) {
+        int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
+        for (int64_t j = 0; j < K; ++j) idx[j] = j;
+        g_sort_amax = amax;
+        qsort(idx, (size_t)K, sizeof(int64_t), cmp_score_desc);
+        for (int64_t i = 0; i < k; ++i) O[i] = (int32_t)idx[i];
+        qsort(O, (size_t)k, sizeof(int32_t), cmp_i32);
+        free(idx);
+    }
+    return 0;
+}
+
+/* J = ascending complement of O in [0, K). Returns Kb. */
+static int64_t build_J(const int32_t* O, int64_t K, int64_t k, int32_t* J)
+{
+    char* is_out = (char*)calloc((size_t)K, 1);
+    for (int64_t i = 0; i < k; ++i) is_out[O[i]] = 1;
+    int64_t p = 0;
+    for (int64_t j = 0; j < K; ++j)
+        if (!is_out[j]) J[p++] = (int32_t)j;
+    free(is_out);
+    return p;
+}
+
+/* ------------------------------------------------------------------ */
+/* Eq. (1): smoothing of activations and folding into weights           */
+/* ------------------------------------------------------------------ */
+
+/* x'_tj = bf16(fp32(x_tj) * inv_s_j): the activations divided by s, by
+ * one FP32 multiply with the FP32 reciprocal, rounded to BF16. */
+void oracle_smooth_act(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, uint16_t* Xs)
+{
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float p = oracle_bf16_to_f32(X[t * K + j]) * inv_s[j];
+            Xs[t * K + j] = oracle_f32_to_bf16(p);
+        }
+}
+
+/* w'_jn = bf16(fp32(w_jn) * s_j): s folded into the master weights. */
+void oracle_fold_weights(const uint16_t* W, int64_t K, int64_t N, const float* s, uint16_t* Ws)
+{
+    for (int64_t j = 0; j < K; ++j)
+        for (int64_t n = 0; n < N; ++n) {
+            float p = oracle_bf16_to_f32(W[j * N + n]) * s[j];
+            Ws[j * N + n] = oracle_f32_to_bf16(p);
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Runtime activation path: smooth, split, MXFP4-encode                 */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For each row t of X [M][K]:
+ *   x' = smoothed row;
+ *   a_hp[t][i] = x'[O_i] (i < k), zero for k <= i < kp;
+ *   bulk row = x'[J_p] for p < Kb, zero for Kb <= p < Kbp;
+ *   for each 32-block b of the bulk row: X_b from the amax of its real
+ *   elements, scale code X_b + 127 (0 if the block has no real element),
+ *   codes E2M1(x'/2^X_b), two per byte, low nibble = even position.
+ * Outputs: codes [M][Kbp/2], scales (logical) [M][Kbp/32], a_hp [M][kp].
+ */
+void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
+                         const float* inv_s, const int32_t* O,
+                         uint8_t* codes, uint8_t* scales, uint16_t* a_hp)
+{
+    int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
+    int64_t nb = Kbp / 32;
+    int32_t* J = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K > 0 ? K : 1));
+    int64_t Kb = build_J(O, K, k, J);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t) {
+        uint16_t* row = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(K > 0 ? K : 1));
+        uint8_t c4[32];
+        for (int64_t j = 0; j < K; ++j) {
+            float p = oracle_bf16_to_f32(X[t * K + j]) * inv_s[j];
+            row[j] = oracle_f32_to_bf16(p);
+        }
+        for (int64_t i = 0; i < kp; ++i) a_hp[t * kp + i] = (i < k) ? row[O[i]] : 0;
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t p0 = 32 * b;
+            int n_real = (int)(p0 >= Kb ? 0 : (Kb - p0 < 32 ? Kb - p0 : 32));
+            uint16_t vals[32];
+            double amax = 0.0;
+            for (int i = 0; i < n_real; ++i) {
+                vals[i] = row[J[p0 + i]];
+                double a = fabs(oracle_bf16_to_f64(vals[i]));
+                if (a > amax) amax = a;
+            }
+            int Xe = oracle_mx_scale_exponent(amax);
+            scales[t * nb + b] = (uint8_t)(n_real ? Xe + 127 : 0);
+            memset(c4, 0, sizeof c4);
+            mx_encode_values(vals, n_real, Xe, c4);
+            for (int i = 0; i < 16; ++i)
+                codes[t * (Kbp / 2) + p0 / 2 + i] = (uint8_t)(c4[2 * i] | (c4[2 * i + 1] << 4));
+        }
+        free(row);
+    }
+    free(J);
+}
+
+/* ------------------------------------------------------------------ */
+/* Offline weight packing with block-wise scales                         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * W [K][N] BF16 row-major (input channel j, output channel n).
+ * w' = folded weights. Outputs are K-major per output channel:
+ *   w_hp [N][kp]: w'[O_i][n], zero padded;
+ *   codes [N][Kbp/2], scales (logical) [N][Kbp/32] over the compacted bulk
+ *   index p, with the block exponent taken from the amax of
+ *     mode 0 (1x32):   the 32 positions of the block of row n;
+ *     mode 1 (32x32):  the 32x32 tile (32 positions x 32 output channels);
+ *     mode 2 (128x1):  the 128-position K-strip of row n;
+ *   and replicated to every 32-block inside the tile or strip. Only real
+ *   elements (p < Kb, n < N) enter an amax; a block with no real element
+ *   gets scale code 0.
+ */
+void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
+                         const float* s, const int32_t* O, int mode,
+                         uint8_t* codes, uint8_t* scales, uint16_t* w_hp)
+{
+    int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
+    int64_t nb = Kbp / 32;
+    int32_t* J = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K > 0 ? K : 1));
+    int64_t Kb = build_J(O, K, k, J);
+    /* folded weights, transposed to [N][K] for convenience */
+    uint16_t* Wt = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(N * (K > 0 ? K : 1)));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K; ++j) {
+            float p = oracle_bf16_to_f32(W[j * N + n]) * s[j];
+            Wt[n * K + j] = oracle_f32_to_bf16(p);
+        }
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t i = 0; i < kp; ++i) w_hp[n * kp + i] = (i < k) ? Wt[n * K + O[i]] : 0;
+
+    /* block amax of row n, block b (real elements only) */
+    double* bam = (double*)calloc((size_t)(N * (nb > 0 ? nb : 1)), sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t b = 0; b < nb; ++b) {
+            double m = 0.0;
+            for (int64_t p = 32 * b; p < 32 * b + 32 && p < Kb; ++p) {
+                double a = fabs(oracle_bf16_to_f64(Wt[n * K + J[p]]));
+                if (a > m) m = a;
+            }
+            bam[n * nb + b] = m;
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        uint8_t c4[32];
+        uint16_t vals[32];
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t p0 = 32 * b;
+            int n_real = (int)(p0 >= Kb ? 0 : (Kb - p0 < 32 ? Kb - p0 : 32));
+            double amax = 0.0;
+            if (mode == 0) {
+                amax = bam[n * nb + b];
+            } else if (mode == 1) {
+                int64_t n0 = n / 32 * 32;
+                for (int64_t nn = n0; nn < n0 + 32 && nn < N; ++nn)
+                    if (bam[nn * nb + b] > amax) amax = bam[nn * nb + b];
+            } else {
+                int64_t b0 = b / 4 * 4;
+                for (int64_t bb = b0; bb < b0 + 4 && bb < nb; ++bb)
+                    if (bam[n * nb + bb] > amax) amax = bam[n * nb + bb];
+            }
+            int Xe = oracle_mx_scale_exponent(amax);
+            scales[n * nb + b] = (uint8_t)(n_real ? Xe + 127 : 0);
+            for (int i = 0; i < n_real; ++i) vals[i] = Wt[n * K + J[p0 + i]];
+            memset(c4, 0, sizeof c4);
+            mx_encode_values(vals, n_real, Xe, c4);
+            for (int i = 0; i < 16; ++i)
+                codes[n * (Kbp / 2) + p0 / 2 + i] = (uint8_t)(c4[2 * i] | (c4[2 * i + 1] << 4));
+        }
+    }
+    free(bam);
+    free(Wt);
+    free(J);
+}
+
+/* ------------------------------------------------------------------ */
+/* Eq. (5) / Eq. (3): the dual-branch product                            */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For each requested activation row r (index rows[r] into the packed
+ * activations) and every output channel n:
+ *   y = sum_b 2^(Xa+Xw) sum_{p in b} e2m1(a) e2m1(w)     (bulk, W4A4)
+ *     + sum_{i<kp} a_hp * w_hp                            (outliers, BF16)
+ *     + bias[n]                                            (if bias != NULL)
+ *   T = the same sum over absolute values of every term (no bias).
+ * Every term is exact in FP64; the sum is accumulated in FP64 in the
+ * order bulk blocks, then outlier slots.
+ * Outputs y, T: [nrows][N].
+ */
+void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
+                           const int64_t* rows, int64_t nrows,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
+                           int64_t N, int64_t Kbp, int64_t kp, const float* bias,
+                           double* y, double* T)
+{
+    int64_t nb = Kbp / 32;
+    /* dequantise all weight rows once: value * 2^Xw, exact in FP64 */
+    double* wd = (double*)malloc(sizeof(double) * (size_t)(N * (Kbp > 0 ? Kbp : 1)));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t p = 0; p < Kbp; ++p) {
+            uint8_t byte = w_codes[n * (Kbp / 2) + p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15u);
+            int Xw = (int)w_scales[n * nb + p / 32] - 127;
+            wd[n * Kbp + p] = oracle_e2m1_decode(c) * ldexp(1.0, Xw);
+        }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows[r];
+        double* ad = (double*)malloc(sizeof(double) * (size_t)(Kbp > 0 ? Kbp : 1));
+        double* hd = (double*)malloc(sizeof(double) * (size_t)(kp > 0 ? kp : 1));
+        for (int64_t p = 0; p < Kbp; ++p) {
+            uint8_t byte = a_codes[t * (Kbp / 2) + p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15u);
+            int Xa = (int)a_scales[t * nb + p / 32] - 127;
+            ad[p] = oracle_e2m1_decode(c) * ldexp(1.0, Xa);
+        }
+        for (int64_t i = 0; i < kp; ++i) hd[i] = oracle_bf16_to_f64(a_hp[t * kp + i]);
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            const double* wr = wd + n * Kbp;
+            for (int64_t p = 0; p < Kbp; ++p) {
+                double term = ad[p] * wr[p];
+                acc += term;
+                mag += fabs(term);
+            }
+            for (int64_t i = 0; i < kp; ++i) {
+                double term = hd[i] * oracle_bf16_to_f64(w_hp[n * kp + i]);
+                acc += term;
+                mag += fabs(term);
+            }
+            if (bias) acc += (double)bias[n];
+            y[r * N + n] = acc;
+            T[r * N + n] = mag;
+        }
+        free(ad);
+        free(hd);
+    }
+    free(wd);
+}
+
+/* ------------------------------------------------------------------ */
+/* GELU (tanh form) in FP32 for the fused FFN epilogue                   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * exp(x) for the GELU's tanh, in FP32 with explicit operations:
+ * Cody-Waite reduction x = n*ln2 + r, |r| <= ln2/2, with ln2 split into a
+ * high part exact in 12 bits and a low remainder; exp(r) by its Taylor
+ * series to degree 7 evaluated by Horner's rule with fused multiply-adds
+ * (fmaf, one rounding each); the result scaled by 2^n with ldexpf.
+ * Arguments are clamped to [-88, 0] because the GELU only needs
+ * exp(-2|u|) in (0, 1].
+ */
+float oracle_gelu_exp_neg(float x)
+{
+    if (x < -88.0f) x = -88.0f;
+    if (x > 0.0f) x = 0.0f;
+    const float LOG2E = 1.44269504088896341f;
+    const float LN2_HI = 0.693145751953125f;       /* 12 significant bits */
+    const float LN2_LO = 1.42860682030941723e-06f; /* ln2 - LN2_HI */
+    float n = rintf(x * LOG2E);
+    float r = fmaf(-n, LN2_HI, x);
+    r = fmaf(-n, LN2_LO, r);
+    /* Taylor coefficients 1/k!, k = 7..0 */
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    return ldexpf(p, (int)n);
+}
+
+/* GELU_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), with
+ * tanh(u) = sign(u) (1 - E)/(1 + E), E = exp(-2|u|), all in FP32. */
+float oracle_gelu_tanh_f32(float x)
+{
+    const float C0 = 0.7978845608028654f;   /* sqrt(2/pi) */
+    const float C1 = 0.044715f;
+    float x3 = x * x * x;
+    float u = C0 * (x + C1 * x3);
+    float E = oracle_gelu_exp_neg(-2.0f * fabsf(u));
+    float th = (1.0f - E) / (1.0f + E);
+    if (u < 0.0f) th = -th;
+    return 0.5f * x * (1.0f + th);
+}
