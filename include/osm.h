@@ -1,0 +1,222 @@
+/*
+ * osm.h -- C ABI of libosm, a B200 (sm_100a) implementation of the
+ * smoothed, outlier-split W4A4 linear layer described in
+ * "W4A4 Quantization for Inference on Wan2.2-I2V-A14B" (ICME 2026
+ * Low-Bit-width Large-Model Quantization Challenge, Sub-Challenge 1).
+ *
+ * The layer computes Y = X W (Eq. (1)) as
+ *     Y = (X/s)_{:,J} W'^(q)_{J,:} + (X/s)_{:,O} W'^(hp)_{O,:}      (Eq. (5))
+ * where s is the SmoothQuant vector of Eq. (2), W' = s (.) W are the
+ * folded weights, O is the static top-k outlier channel set of Eq. (4),
+ * J its complement, (q) is MXFP4 (OCP MX v1.0: E2M1 elements, one E8M0
+ * scale per 32 consecutive bulk channels, round-to-nearest-even) and
+ * (hp) is BF16. The 4-bit format stands in for the paper's HiF4, whose
+ * bit layout the paper does not give.
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless the parameter name ends in
+ *     _host. BF16 tensors are passed as uint16_t bit patterns. All device
+ *     pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device work is enqueued on it and the call returns without
+ *     synchronising, except where stated.
+ *   - The caller allocates every tensor; sizes come from osm_plan_sizes().
+ *     The library allocates device memory only in osm_plan_create() and
+ *     frees it in osm_plan_destroy(). Hot-path calls allocate nothing.
+ *   - Return value: OSM_OK or an OSM_ERR_* code. Nothing is enqueued when
+ *     an argument check fails. osm_last_error() gives a message for the
+ *     calling thread's last failure. No call aborts the process; no device
+ *     code traps.
+ *
+ * Index sets and packed layouts (shared by activations and weights)
+ *   K = input channels, k = |O|, Kb = K - k, Kbp = Kb rounded up to 128,
+ *   kp = k rounded up to 64. O ascending; J = ascending complement of O,
+ *   compacted to bulk positions p = 0..Kb-1. For a matrix with R rows:
+ *   codes  [R][Kbp/2] u8   E2M1 of bulk position p of row r in byte
+ *                          r*Kbp/2 + p/2, low nibble for even p; padding
+ *                          positions p >= Kb hold code 0.
+ *   scales E8M0 of 32-block b = p/32 of row r (exponent + 127), in the
+ *          tcgen05 block-scale layout: 128-row x 4-block atoms of 512
+ *          bytes; atom (r/128, b/4) at byte offset
+ *          ((r/128) * (Kbp/128) + b/4) * 512, and inside the atom
+ *          (r%32)*16 + ((r%128)/32)*4 + b%4. Rows are padded to a multiple
+ *          of 128; a block with no real element (and every padding row)
+ *          holds 0.
+ *   hp     [R][kp] BF16    the outlier channels O_0..O_{k-1}, zero padded.
+ */
+#ifndef OSM_H
+#define OSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define OSM_API __attribute__((visibility("default")))
+#else
+#define OSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes --------------------------------------------------- */
+#define OSM_OK                 0
+#define OSM_ERR_INVALID_ARG    1  /* null / misaligned pointer, bad size or mode          */
+#define OSM_ERR_UNSUPPORTED    2  /* device is not sm_100, or a shape the kernels refuse  */
+#define OSM_ERR_CUDA           3  /* a CUDA runtime call or a launch failed               */
+#define OSM_ERR_TIMEOUT        4  /* a device-side wait gave up (reported via status)     */
+#define OSM_ERR_NONFINITE      5  /* calibration statistics contain inf or NaN           */
+#define OSM_ERR_NOMEM          6  /* plan allocation failed                               */
+
+/* device status bits, returned by osm_plan_status() */
+#define OSM_STATUS_TIMEOUT     1u  /* a pipeline wait in osm_dual_gemm ran out of time */
+
+typedef struct osm_plan osm_plan;
+
+/* Weight block-scale layouts evaluated in the paper's packing paragraph
+ * (Fig. 8): the exponent of a 32-block is taken from the amax of
+ *   OSM_WSCALE_1x32       the block itself (plain MXFP4);
+ *   OSM_WSCALE_TILE32x32  its 32 (bulk channel) x 32 (output channel) tile;
+ *   OSM_WSCALE_STRIP128x1 its 128-channel K-major stripe of one output row;
+ * and replicated to every 32-block inside the tile or stripe. */
+typedef enum {
+    OSM_WSCALE_1x32 = 0,
+    OSM_WSCALE_TILE32x32 = 1,
+    OSM_WSCALE_STRIP128x1 = 2
+} osm_wscale_mode;
+
+/* Epilogues of osm_dual_gemm. */
+typedef enum {
+    OSM_EPI_F32 = 0,          /* Y [M][N] float32                                  */
+    OSM_EPI_BF16 = 1,         /* Y [M][N] BF16 (RNE of the FP32 accumulator)       */
+    OSM_EPI_GELU_REQUANT = 2  /* GELU(tanh) -> x/s_next -> split + MXFP4 for `next`  */
+} osm_epi;
+
+/* ---- calibration (offline) ------------------------------------------
+ * "For each targeted FFN linear map we record per-input-channel activation
+ * maxima, weight column ranges" (implementation/calibration paragraph).
+ */
+
+/* amax[j] = max(amax[j], max_t |X[t][j]|) for X [T][K] BF16 row-major.
+ * amax is device float[K], max-merged in place (zero it before the first
+ * batch), so several calibration batches accumulate. T >= 0, K > 0. */
+OSM_API int osm_act_amax_accumulate(const uint16_t* X, int64_t T, int64_t K, float* amax, void* stream);
+
+/* wmax[j] = max_n |W[j][n]| for W [K][N] BF16 row-major (input channel j,
+ * output channel n); the "weight column range" of Eq. (2). Overwrites wmax
+ * (device float[K]). */
+OSM_API int osm_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, void* stream);
+
+/* Host-side finalisation of Eq. (2) and Eq. (4):
+ *   s_j     = fp32( max(amax_j,1e-5)^alpha / max(wmax_j,1e-5)^(1-alpha) )
+ *             evaluated in double;
+ *   inv_s_j = 1.0f / s_j (IEEE fp32 division);
+ *   O       = the k channels with the largest amax_j (score of Eq. (4);
+ *             ties: lower index first), written ascending.
+ * All arrays are host memory of length K (O_host: k). 0 < alpha < 1,
+ * 0 <= k <= K. Returns OSM_ERR_NONFINITE if a statistic is inf/NaN. */
+OSM_API int osm_calibrate_finalize(const float* amax_host, const float* wmax_host, int64_t K, float alpha,
+                           int64_t k, float* s_host, float* inv_s_host, int32_t* O_host);
+
+/* ---- plans ------------------------------------------------------------ */
+
+/* Build a plan for one linear map with K input and N output channels,
+ * smoothing vector s (host float[K], > 0, finite) and ascending outlier set
+ * O (host int32[k], distinct, in [0, K)). The plan owns device copies of
+ * inv_s = 1.0f/s, the channel routing table and a status word.
+ * Requirements: K % 32 == 0, N % 32 == 0, 0 <= k <= K, K <= 65504.
+ * The plan is bound to the current CUDA device. */
+OSM_API int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const int32_t* O_host,
+                    int wscale_mode, osm_plan** out);
+OSM_API int osm_plan_destroy(osm_plan* plan);
+
+/* Bytes of the packed buffers for `rows` rows (activations: rows = M;
+ * weights: rows = N). scales_bytes includes the padding to 128 rows. */
+OSM_API int osm_plan_sizes(const osm_plan* plan, int64_t rows, size_t* codes_bytes, size_t* scales_bytes,
+                   size_t* hp_bytes);
+
+/* K, N, k, Kb, Kbp, kp of the plan (any pointer may be NULL). */
+OSM_API int osm_plan_dims(const osm_plan* plan, int64_t* K, int64_t* N, int64_t* k, int64_t* Kb,
+                  int64_t* Kbp, int64_t* kp);
+
+/* Reads (and, if clear != 0, resets) the plan's device status word. Waits
+ * for `stream` to finish. status_host receives OSM_STATUS_* bits. */
+OSM_API int osm_plan_status(const osm_plan* plan, void* stream, uint32_t* status_host, int clear);
+
+/* Debug knob for failure-detection tests: the wait limit, in nanoseconds,
+ * of every pipeline wait inside osm_dual_gemm for this plan (default
+ * 2e9). A wait that runs out sets OSM_STATUS_TIMEOUT and the kernel
+ * returns early; the context stays usable. */
+OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
+
+/* ---- offline weight packing --------------------------------------------
+ * "SmoothQuant scales are folded into master weights before HiF4 packing"
+ * and "remaining weights are packed with block-wise scales" (packing and
+ * implementation paragraphs, Fig. 8).
+ * W [K][N] BF16 row-major. w' = bf16(fp32(w_jn) * s_j). Writes
+ *   w_codes  [N][Kbp/2], w_scales (layout above, rows = N), w_hp [N][kp]
+ * with the plan's block-scale mode. */
+OSM_API int osm_pack_weights(const osm_plan* plan, const uint16_t* W, uint8_t* w_codes, uint8_t* w_scales,
+                     uint16_t* w_hp, void* stream);
+
+/* ---- runtime activation path ----------------------------------------------
+ * "activations are divided in-place by s, quantized ..., and routed through
+ * either the W4A4 bulk path or a narrow FP16 outlier path" (implementation
+ * paragraph). X [M][K] BF16 row-major, M >= 1. For each row:
+ *   x' = bf16(fp32(x_j) * inv_s_j);
+ *   a_hp[t][i] = x'[O_i];
+ *   bulk x'[J_p] -> MXFP4 with the exponent floor(log2 amax_b) - 2 of each
+ *   32-block (clamped to [-127,127]; amax 0 -> -127), elements E2M1 RNE,
+ *   saturating at 6; the sign bit is the sign of x'.
+ * Writes a_codes [M][Kbp/2], a_scales (rows padded to 128), a_hp [M][kp]. */
+OSM_API int osm_quantize_act(const osm_plan* plan, const uint16_t* X, int64_t M, uint8_t* a_codes,
+                     uint8_t* a_scales, uint16_t* a_hp, void* stream);
+
+/* ---- the dual-branch GEMM ------------------------------------------------
+ * Eq. (5) with Eq. (3)'s per-group scales taken per 32-block:
+ *   acc[t][n] = sum_b 2^(Xa(t,b)+Xw(n,b)) sum_{p in b} e2m1(a_tp) e2m1(w_np)
+ *             + sum_{i<kp} a_hp[t][i] w_hp[n][i]             (FP32 accumulate)
+ *   y = acc (+ bias[n] if bias != NULL).
+ * Both branches accumulate into one tensor-memory accumulator on tcgen05
+ * (block-scaled MXFP4 MMA, then BF16 MMA) before a single epilogue.
+ * Operands come from osm_quantize_act / osm_pack_weights with the same
+ * plan. M >= 1.
+ *   epi = OSM_EPI_F32:  Y is float [M][N].
+ *   epi = OSM_EPI_BF16: Y is BF16  [M][N].
+ *   epi = OSM_EPI_GELU_REQUANT: not available in this build (returns
+ *         OSM_ERR_UNSUPPORTED); `next`, next_* must be NULL otherwise.
+ * A pipeline wait that exceeds the plan's wait limit sets the plan's
+ * OSM_STATUS_TIMEOUT bit (see osm_plan_status). */
+OSM_API int osm_dual_gemm(const osm_plan* plan, const uint8_t* a_codes, const uint8_t* a_scales,
+                  const uint16_t* a_hp, int64_t M, const uint8_t* w_codes, const uint8_t* w_scales,
+                  const uint16_t* w_hp, const float* bias, int epi, void* Y, const osm_plan* next,
+                  uint8_t* next_codes, uint8_t* next_scales, uint16_t* next_hp, void* stream);
+
+/* ---- end-to-end layer from host memory ------------------------------------
+ * One forward of the layer for a host (preferably pinned) X_host [M][K]
+ * BF16: copies X to the device, runs osm_quantize_act and osm_dual_gemm
+ * against resident packed weights, and copies Y (F32 or BF16, per epi)
+ * back to Y_host. workspace is caller-owned device memory of at least
+ * osm_linear_workspace_size(plan, M, epi) bytes. Enqueued on `stream`; the
+ * caller synchronises before reading Y_host. */
+OSM_API size_t osm_linear_workspace_size(const osm_plan* plan, int64_t M, int epi);
+OSM_API int osm_linear_host(const osm_plan* plan, const uint16_t* X_host, int64_t M, const uint8_t* w_codes,
+                    const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi,
+                    void* Y_host, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- helpers ------------------------------------------------------------ */
+
+/* Host-only: un-swizzle a scales buffer (layout above) of `rows` rows and
+ * `nblocks` = Kbp/32 blocks into a row-major [rows][nblocks] host array. */
+OSM_API int osm_scales_to_logical(const uint8_t* swizzled_host, int64_t rows, int64_t nblocks,
+                          uint8_t* logical_host);
+
+/* Message for the calling thread's most recent failed call ("" if none). */
+OSM_API const char* osm_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OSM_H */

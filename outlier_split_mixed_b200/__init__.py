@@ -1,1 +1,332 @@
-"""B200-native smoothed, outlier-split W4A4 linear layer (placeholder binding)."""
+"""B200 (sm_100a) smoothed, outlier-split W4A4 linear layer.
+
+Python binding of libosm (``include/osm.h``): each function below marshals
+torch tensors / numpy arrays into the C entry point of the same name
+(``osm_<name>``) and raises :class:`OsmError` on a non-zero return code.
+There is no fallback: every computation runs in the CUDA library, and a
+missing library raises at first use.
+
+Method: "W4A4 Quantization for Inference on Wan2.2-I2V-A14B" -- SmoothQuant
+smoothing (Eq. (1), (2)), a static top-k outlier split (Eq. (4), (5)) and a
+dual-branch GEMM whose bulk branch is MXFP4 (E2M1 + E8M0 per 32) and whose
+outlier branch is BF16 (Eq. (3)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libosm.so")
+
+OK = 0
+ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
+STATUS_TIMEOUT = 1
+WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
+EPI_F32, EPI_BF16, EPI_GELU_REQUANT = 0, 1, 2
+
+# Every entry point declared in include/osm.h, with its ctypes signature.
+_P, _I64, _I, _U64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+_SIGNATURES = {
+    "osm_act_amax_accumulate": (_I, [_P, _I64, _I64, _P, _P]),
+    "osm_weight_amax": (_I, [_P, _I64, _I64, _P, _P]),
+    "osm_calibrate_finalize": (_I, [_P, _P, _I64, ctypes.c_float, _I64, _P, _P, _P]),
+    "osm_plan_create": (_I, [_I64, _I64, _I64, _P, _P, _I, ctypes.POINTER(_P)]),
+    "osm_plan_destroy": (_I, [_P]),
+    "osm_plan_sizes": (_I, [_P, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
+    "osm_plan_dims": (_I, [_P] + [ctypes.POINTER(_I64)] * 6),
+    "osm_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _I]),
+    "osm_plan_set_wait_limit": (_I, [_P, _U64]),
+    "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
+    "osm_quantize_act": (_I, [_P, _P, _I64, _P, _P, _P, _P]),
+    "osm_dual_gemm": (_I, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
+    "osm_linear_workspace_size": (_SZ, [_P, _I64, _I]),
+    "osm_linear_host": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "osm_scales_to_logical": (_I, [_P, _I64, _I64, _P]),
+    "osm_last_error": (ctypes.c_char_p, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class OsmError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libosm error {code}: {msg}")
+        self.code = code
+
+
+def lib():
+    """The loaded libosm (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m outlier_split_mixed_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    v = lib().osm_last_error()
+    return v.decode() if v else ""
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise OsmError(rc, last_error())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, name, dtypes=None, numel=None, allow_none=False):
+    """Device pointer of a contiguous CUDA tensor (or None)."""
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if numel is not None and t.numel() * t.element_size() < numel:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _bf16_types():
+    import torch
+    return (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _u8_types():
+    import torch
+    return (torch.uint8,)
+
+
+# ----------------------------------------------------------------- plans
+
+class Plan:
+    """An osm_plan: K, N, k, the smoothing vector s, the outlier set O and
+    the weight block-scale mode, with its device tables."""
+
+    def __init__(self, K: int, N: int, k: int, s: np.ndarray, O: np.ndarray, wscale_mode: int = WSCALE_1x32):
+        s = np.ascontiguousarray(s, dtype=np.float32)
+        O = np.ascontiguousarray(O, dtype=np.int32)
+        if s.shape != (K,) or O.shape != (k,):
+            raise ValueError("s must have shape (K,) and O shape (k,)")
+        h = ctypes.c_void_p()
+        _check(lib().osm_plan_create(K, N, k, _host_ptr(s), _host_ptr(O) if k else None, int(wscale_mode),
+                                     ctypes.byref(h)))
+        self._h = h
+        self.s, self.O, self.wscale_mode = s, O, int(wscale_mode)
+        d = [ctypes.c_int64() for _ in range(6)]
+        _check(lib().osm_plan_dims(self._h, *[ctypes.byref(x) for x in d]))
+        self.K, self.N, self.k, self.Kb, self.Kbp, self.kp = (int(x.value) for x in d)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def sizes(self, rows: int):
+        """(codes_bytes, scales_bytes, hp_bytes) for `rows` rows."""
+        c, s, h = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().osm_plan_sizes(self._h, rows, ctypes.byref(c), ctypes.byref(s), ctypes.byref(h)))
+        return int(c.value), int(s.value), int(h.value)
+
+    def status(self, clear: bool = True, stream=None) -> int:
+        v = ctypes.c_uint32()
+        _check(lib().osm_plan_status(self._h, _stream(stream), ctypes.byref(v), int(clear)))
+        return int(v.value)
+
+    def set_wait_limit(self, ns: int):
+        _check(lib().osm_plan_set_wait_limit(self._h, int(ns)))
+
+    def alloc_packed(self, rows: int, device="cuda"):
+        """Allocate (codes, scales, hp) torch buffers for `rows` rows."""
+        import torch
+        cb, sb, hb = self.sizes(rows)
+        codes = torch.empty(max(cb, 16), dtype=torch.uint8, device=device)[:cb]
+        scales = torch.empty(max(sb, 16), dtype=torch.uint8, device=device)[:sb]
+        hp = torch.empty(max(hb // 2, 8), dtype=torch.bfloat16, device=device)[:hb // 2]
+        return codes, scales, hp
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().osm_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ----------------------------------------------------------------- calibration
+
+def act_amax_accumulate(X, amax, stream=None):
+    """amax = max(amax, max_t |X[t]|) on the device (osm_act_amax_accumulate)."""
+    T, K = X.shape
+    import torch
+    _check(lib().osm_act_amax_accumulate(_ptr(X, "X", _bf16_types()), T, K,
+                                         _ptr(amax, "amax", (torch.float32,), K * 4), _stream(stream)))
+
+
+def weight_amax(W, wmax, stream=None):
+    """wmax[j] = max_n |W[j][n]| (osm_weight_amax)."""
+    K, N = W.shape
+    import torch
+    _check(lib().osm_weight_amax(_ptr(W, "W", _bf16_types()), K, N, _ptr(wmax, "wmax", (torch.float32,), K * 4),
+                                 _stream(stream)))
+
+
+def calibrate_finalize(amax_host: np.ndarray, wmax_host: np.ndarray, alpha: float, k: int):
+    """Eq. (2) and Eq. (4) on host statistics -> (s, inv_s, O) (osm_calibrate_finalize)."""
+    amax_host = np.ascontiguousarray(amax_host, dtype=np.float32)
+    wmax_host = np.ascontiguousarray(wmax_host, dtype=np.float32)
+    K = amax_host.shape[0]
+    s = np.empty(K, np.float32)
+    inv_s = np.empty(K, np.float32)
+    O = np.empty(max(k, 1), np.int32)
+    _check(lib().osm_calibrate_finalize(_host_ptr(amax_host), _host_ptr(wmax_host), K, float(alpha), int(k),
+                                        _host_ptr(s), _host_ptr(inv_s), _host_ptr(O)))
+    return s, inv_s, O[:k].copy()
+
+
+# ----------------------------------------------------------------- layer path
+
+def pack_weights(plan: Plan, W, w_codes, w_scales, w_hp, stream=None):
+    """Fold s into W and pack it (osm_pack_weights). W: [K][N] BF16."""
+    cb, sb, hb = plan.sizes(plan.N)
+    if tuple(W.shape) != (plan.K, plan.N):
+        raise ValueError("W must have shape (K, N)")
+    _check(lib().osm_pack_weights(plan.handle, _ptr(W, "W", _bf16_types()),
+                                  _ptr(w_codes, "w_codes", _u8_types(), cb, allow_none=cb == 0),
+                                  _ptr(w_scales, "w_scales", _u8_types(), sb, allow_none=sb == 0),
+                                  _ptr(w_hp, "w_hp", _bf16_types(), hb, allow_none=hb == 0), _stream(stream)))
+
+
+def quantize_act(plan: Plan, X, a_codes, a_scales, a_hp, stream=None):
+    """Smooth, split and MXFP4-encode activations (osm_quantize_act). X: [M][K] BF16."""
+    M, K = X.shape
+    if K != plan.K:
+        raise ValueError("X must have K columns")
+    cb, sb, hb = plan.sizes(M)
+    _check(lib().osm_quantize_act(plan.handle, _ptr(X, "X", _bf16_types()), M,
+                                  _ptr(a_codes, "a_codes", _u8_types(), cb, allow_none=cb == 0),
+                                  _ptr(a_scales, "a_scales", _u8_types(), sb, allow_none=sb == 0),
+                                  _ptr(a_hp, "a_hp", _bf16_types(), hb, allow_none=hb == 0), _stream(stream)))
+
+
+def dual_gemm(plan: Plan, a_codes, a_scales, a_hp, M: int, w_codes, w_scales, w_hp, Y, bias=None,
+              epi: int = EPI_F32, stream=None):
+    """Eq. (5) on packed operands (osm_dual_gemm). Y: [M][N] float32 or BF16."""
+    import torch
+    cbm, sbm, hbm = plan.sizes(M)
+    cbn, sbn, hbn = plan.sizes(plan.N)
+    ybytes = M * plan.N * (4 if epi == EPI_F32 else 2)
+    ytypes = (torch.float32,) if epi == EPI_F32 else _bf16_types()
+    _check(lib().osm_dual_gemm(plan.handle,
+                               _ptr(a_codes, "a_codes", _u8_types(), cbm, allow_none=cbm == 0),
+                               _ptr(a_scales, "a_scales", _u8_types(), sbm, allow_none=sbm == 0),
+                               _ptr(a_hp, "a_hp", _bf16_types(), hbm, allow_none=hbm == 0), M,
+                               _ptr(w_codes, "w_codes", _u8_types(), cbn, allow_none=cbn == 0),
+                               _ptr(w_scales, "w_scales", _u8_types(), sbn, allow_none=sbn == 0),
+                               _ptr(w_hp, "w_hp", _bf16_types(), hbn, allow_none=hbn == 0),
+                               _ptr(bias, "bias", (torch.float32,), plan.N * 4, allow_none=True), int(epi),
+                               _ptr(Y, "Y", ytypes, ybytes), None, None, None, None, _stream(stream)))
+
+
+def linear_workspace_size(plan: Plan, M: int, epi: int = EPI_F32) -> int:
+    return int(lib().osm_linear_workspace_size(plan.handle, M, int(epi)))
+
+
+def linear_host(plan: Plan, X_host, M: int, w_codes, w_scales, w_hp, Y_host, workspace, bias=None,
+                epi: int = EPI_F32, stream=None):
+    """Host X -> device quantize + dual GEMM -> host Y (osm_linear_host).
+    X_host / Y_host: pinned CPU torch tensors; the caller synchronises."""
+    import torch
+    for t, n in ((X_host, "X_host"), (Y_host, "Y_host")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous host tensor")
+    cbn, sbn, hbn = plan.sizes(plan.N)
+    _check(lib().osm_linear_host(plan.handle, ctypes.c_void_p(X_host.data_ptr()), M,
+                                 _ptr(w_codes, "w_codes", _u8_types(), cbn, allow_none=cbn == 0),
+                                 _ptr(w_scales, "w_scales", _u8_types(), sbn, allow_none=sbn == 0),
+                                 _ptr(w_hp, "w_hp", _bf16_types(), hbn, allow_none=hbn == 0),
+                                 _ptr(bias, "bias", (torch.float32,), plan.N * 4, allow_none=True), int(epi),
+                                 ctypes.c_void_p(Y_host.data_ptr()), _ptr(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def scales_to_logical(swizzled: np.ndarray, rows: int, nblocks: int) -> np.ndarray:
+    """Un-swizzle a scales buffer into [rows][nblocks] (osm_scales_to_logical)."""
+    swizzled = np.ascontiguousarray(swizzled, dtype=np.uint8)
+    out = np.zeros((rows, nblocks), np.uint8)
+    if rows and nblocks:
+        _check(lib().osm_scales_to_logical(_host_ptr(swizzled), rows, nblocks, _host_ptr(out)))
+    return out
+
+
+# ----------------------------------------------------------------- composition
+
+def calibrate(X_batches, W, alpha: float, k: int, stream=None):
+    """Per-channel statistics over calibration batches (device kernels),
+    then Eq. (2)/(4) on the host: returns (s, inv_s, O, amax, wmax)."""
+    import torch
+    K = W.shape[0]
+    amax = torch.zeros(K, dtype=torch.float32, device=W.device)
+    wmax = torch.empty(K, dtype=torch.float32, device=W.device)
+    for X in X_batches:
+        act_amax_accumulate(X, amax, stream)
+    weight_amax(W, wmax, stream)
+    a, w = amax.cpu().numpy(), wmax.cpu().numpy()
+    s, inv_s, O = calibrate_finalize(a, w, alpha, k)
+    return s, inv_s, O, a, w
+
+
+class QuantLinear:
+    """A packed layer: plan + resident packed weights. `forward(X)` runs
+    quantize_act and dual_gemm on the current stream."""
+
+    def __init__(self, plan: Plan, W, bias=None, device="cuda"):
+        self.plan = plan
+        self.w_codes, self.w_scales, self.w_hp = plan.alloc_packed(plan.N, device)
+        pack_weights(plan, W, self.w_codes, self.w_scales, self.w_hp)
+        self.bias = bias
+
+    def forward(self, X, epi: int = EPI_F32, out=None, act_buffers=None, stream=None):
+        import torch
+        M = X.shape[0]
+        a = act_buffers if act_buffers is not None else self.plan.alloc_packed(M, X.device)
+        quantize_act(self.plan, X, *a, stream=stream)
+        if out is None:
+            out = torch.empty((M, self.plan.N), dtype=torch.float32 if epi == EPI_F32 else torch.bfloat16,
+                              device=X.device)
+        dual_gemm(self.plan, *a, M, self.w_codes, self.w_scales, self.w_hp, out, bias=self.bias, epi=epi,
+                  stream=stream)
+        return out

@@ -1,0 +1,54 @@
+// Internal declarations shared by the libosm translation units.
+#pragma once
+
+#include <cstdint>
+#include <cstddef>
+#include <cuda_runtime.h>
+
+#include "osm.h"
+
+struct osm_plan {
+    int device;
+    int64_t K, N, k, Kb, Kbp, kp;
+    int wmode;
+    // device tables, owned by the plan
+    float* d_s;          // [K]  smoothing vector s (Eq. (2))
+    float* d_inv_s;      // [K]  1.0f / s
+    int32_t* d_route;    // [K]  destination of channel j inside a staged row:
+                         //      bulk position p in [0, Kb) or Kbp + i for outlier slot i
+    int32_t* d_J;        // [Kb] bulk position -> channel (ascending)
+    int32_t* d_O;        // [k]  outlier slot -> channel (ascending)
+    uint32_t* d_status;  // OSM_STATUS_* bits written by kernels
+    uint64_t wait_limit_ns;
+};
+
+namespace osm {
+
+// thread-local error message
+void set_error(const char* fmt, ...);
+int fail(int code, const char* fmt, ...);
+int check_cuda(cudaError_t e, const char* what);
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bytes of one scales buffer for `rows` rows of a plan.
+inline int64_t scales_bytes(int64_t rows, int64_t Kbp) {
+    return round_up(rows, 128) * (Kbp / 32);
+}
+
+// launchers (return OSM_OK or an error code; arguments already validated)
+int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st);
+int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cudaStream_t st);
+int launch_pack_weights(const osm_plan* p, const uint16_t* W, uint8_t* codes, uint8_t* scales,
+                        uint16_t* hp, cudaStream_t st);
+int launch_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* codes,
+                        uint8_t* scales, uint16_t* hp, cudaStream_t st);
+int launch_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_scales,
+                     const uint16_t* a_hp, int64_t M, const uint8_t* w_codes,
+                     const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi,
+                     void* Y, cudaStream_t st);
+
+}  // namespace osm
