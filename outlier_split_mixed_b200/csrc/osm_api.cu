@@ -174,9 +174,10 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
         for (int64_t i = 0; i < k; ++i) slot[O_host[i]] = static_cast<int32_t>(i);
         for (int64_t j = 0; j < K; ++j) {
             if (slot[j] >= 0) {
-                route[j] = static_cast<int32_t>(p->Kbp + slot[j]);
+                route[j] = static_cast<int32_t>((p->Kbp / 32) * QA_BLOCK_BYTES + 2 * slot[j]);
             } else {
-                route[j] = static_cast<int32_t>(J.size());
+                const int64_t pos = static_cast<int64_t>(J.size());
+                route[j] = static_cast<int32_t>((pos / 32) * QA_BLOCK_BYTES + (pos % 32) * 2);
                 J.push_back(static_cast<int32_t>(j));
             }
         }

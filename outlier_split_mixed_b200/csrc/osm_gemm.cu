@@ -7,19 +7,33 @@
 //       + sum over outlier K-steps of tcgen05.mma kind::f16 (BF16 x BF16)
 //
 // Both branches accumulate into the same FP32 tensor-memory accumulator
-// before one epilogue. Persistent CTAs (one per SM, 128x256 output tiles),
-// warp-specialised:
-//   warp 0     TMA producer (tiled 128B-swizzled loads of codes / BF16
-//              chunks, 1-D bulk copies of the scale atoms) into a 4-deep
-//              shared-memory ring guarded by mbarriers;
-//   warp 1     tensor-memory allocation and the single MMA-issuing thread
-//              (tcgen05.cp of the scale atoms into tensor memory, then the
-//              MMAs, then tcgen05.commit to release the ring slot);
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, optional bias,
-//              FP32 or BF16 stores.
+// before one epilogue.
+//
+// Work decomposition: persistent CTA pairs (clusters of 2, one CTA per SM);
+// each pair owns a 256 x 256 output tile at a time and issues cta_group::2
+// MMAs (M = 256 split across the two SMs, N = 256 with B split likewise),
+// so each SM streams 128 rows of A and 128 rows of B per K-step for a
+// 128 x 256 share of the output.
+//
+// Roles in each CTA (warp-specialised):
+//   warp 0     TMA producer: 128B-swizzled tiles of its A rows and B rows,
+//              and the scale atoms (its 128 A rows; all 256 B rows), into
+//              a 6-deep shared-memory ring. All copies of both CTAs
+//              complete on the LEADER CTA's ring barrier.
+//   warp 1     tensor-memory allocation for the pair; in the leader CTA the
+//              single MMA-issuing thread: tcgen05.cp of the scale atoms
+//              into tensor memory (both CTAs), the MMAs, and a multicast
+//              tcgen05.commit that frees the ring slot in both CTAs.
+//   warps 2-9  epilogue: each warp drains 32 lanes x 128 columns of its
+//              CTA's accumulator half into registers, hands tensor memory
+//              back (arrivals counted in the leader), then adds the bias and
+//              writes FP32 or BF16 through a double-buffered, 64B-swizzled
+//              shared-memory chunk and a bulk tensor store (full-line global
+//              writes, ragged M/N edges clipped by the tensor map) while the
+//              next tile's MMAs run.
 // Every wait is bounded by %globaltimer; a wait that runs out sets the
-// plan's status word, raises a CTA-wide abort flag, and the CTA drains its
-// in-flight copies and MMAs, frees tensor memory and returns.
+// plan's status word and raises a CTA-wide abort flag; the CTA then lets
+// its in-flight copies and MMAs finish, frees tensor memory and returns.
 // No TMA multicast is used anywhere.
 
 #include <cuda.h>
@@ -37,37 +51,44 @@
 namespace osm {
 namespace {
 
-constexpr int BM = 128;                 // output rows per tile (TMEM lanes)
-constexpr int BN = 256;                 // output columns per tile (TMEM columns)
-constexpr int STAGES = 4;
+constexpr int BM = 128;                 // accumulator rows per CTA (TMEM lanes); pair tile M = 256
+constexpr int BN = 256;                 // output columns per tile; each CTA loads BN/2 rows of B
+constexpr int STAGES = 5;
 constexpr int A_TILE = BM * 128;        // one K-step of A: 128 rows x 128 bytes
-constexpr int B_TILE = BN * 128;        // one K-step of B: 256 rows x 128 bytes
-constexpr int SFA_TILE = 2 * 512;       // two 128x4 scale atoms
-constexpr int SFB_TILE = 2 * 2 * 512;   // two row tiles x two atoms
-constexpr int NUM_THREADS = 192;
+constexpr int B_TILE = (BN / 2) * 128;  // one K-step of this CTA's half of B
+constexpr int SFA_TILE = 2 * 512;       // two 128x4 scale atoms (K = 256)
+constexpr int SFB_TILE = 2 * 2 * 512;   // two 128-row tiles x two atoms (all 256 B rows)
+constexpr int NUM_EPI_WARPS = 8;        // two per TMEM lane quadrant, 128 columns each
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int EPI_CHUNK = 2048;         // 32 rows x 64 bytes: 16 FP32 or 32 BF16 columns
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;       // scale factors live after the accumulator
 constexpr uint32_t SF_STAGE_COLS = 24;  // 8 columns for A, 16 for B per ring slot
-constexpr int GROUP_M = 16;             // raster: 16 M-blocks sweep the N-blocks together
+constexpr int GROUP_M = 8;              // raster: 8 M-tiles sweep the N-tiles together
+constexpr uint16_t PAIR_MASK = 0x3;
 
-// Instruction descriptors (tcgen05 instruction-descriptor format).
+static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+
+// Instruction descriptors (tcgen05 instruction-descriptor format), M = 256
+// over the CTA pair, N = 256.
 // kind::mxf4 block-scaled: A/B E2M1 (1), K-major, N>>3 @17, UE8M0 scales
 // (bit 23), M>>4 @24; scale-factor byte ids at bits 29-30 (A) and 4-5 (B).
 constexpr uint32_t IDESC_MXF4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-                                ((uint32_t)(BM >> 4) << 24);
+                                ((uint32_t)((2 * BM) >> 4) << 24);
 // kind::f16: FP32 accumulate (bit 4), A/B BF16 (1 @7, 1 @10), K-major.
 constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                ((uint32_t)(BM >> 4) << 24);
+                                ((uint32_t)((2 * BM) >> 4) << 24);
 
 struct __align__(1024) Smem {
     uint8_t a[STAGES][A_TILE];
     uint8_t b[STAGES][B_TILE];
     uint8_t sfa[STAGES][SFA_TILE];
     uint8_t sfb[STAGES][SFB_TILE];
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint8_t epi[NUM_EPI_WARPS][2][EPI_CHUNK];
+    uint64_t full[STAGES];   // leader: all copies of both CTAs for the slot have landed
+    uint64_t empty[STAGES];  // both: the MMAs reading the slot have completed
+    uint64_t acc_full;       // both: the tile's accumulator is complete
+    uint64_t acc_empty;      // leader: both CTAs' epilogues have drained the accumulator
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -75,11 +96,12 @@ struct __align__(1024) Smem {
 
 struct GemmParams {
     CUtensorMap tm_a;    // a_codes  [M][Kbp/2] u8, box 128 x 128
-    CUtensorMap tm_b;    // w_codes  [N][Kbp/2] u8, box 128 x 256
+    CUtensorMap tm_b;    // w_codes  [N][Kbp/2] u8, box 128 x 128
     CUtensorMap tm_ah;   // a_hp     [M][kp] bf16, box 64 x 128
-    CUtensorMap tm_bh;   // w_hp     [N][kp] bf16, box 64 x 256
-    const uint8_t* a_scales;
-    const uint8_t* w_scales;
+    CUtensorMap tm_bh;   // w_hp     [N][kp] bf16, box 64 x 128
+    CUtensorMap tm_sa;   // a_scales as [bytes/16][16] u8, box 16 x 32 (one 512-byte atom)
+    CUtensorMap tm_sb;   // w_scales likewise
+    CUtensorMap tm_y;    // Y [M][N] f32 (box 16 x 32) or bf16 (box 32 x 32), 64B swizzle
     const float* bias;
     void* Y;
     uint32_t* status;
@@ -117,43 +139,64 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
     return ptx::smem_desc(saddr, 0, 128, ptx::LAYOUT_NONE);
 }
 
-__device__ __forceinline__ void store_chunk(const GemmParams& p, int64_t row, int64_t col0,
-                                            const uint32_t (&r)[32]) {
-    float v[32];
+// Write one 32-row x 64-byte chunk (16 FP32 or 32 BF16 columns per row) of
+// the warp's accumulator slice into a 64B-swizzled staging buffer: row r
+// (= lane) keeps its four 16-byte pieces at positions c ^ ((r >> 1) & 3),
+// the layout the tensor map's 64B swizzle expects, which also keeps each
+// group of eight lanes on distinct banks.
+template <int C, bool BF16>
+__device__ __forceinline__ void stage_chunk(uint32_t buf, int lane, const uint32_t (&r)[128]) {
+    const uint32_t row = buf + lane * 64;
+    const int sw = (lane >> 1) & 3;
+    if (!BF16) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-    if (p.bias) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + col0 + i));
-            v[i] += b.x;
-            v[i + 1] += b.y;
-            v[i + 2] += b.z;
-            v[i + 3] += b.w;
+        for (int c = 0; c < 4; ++c) {
+            const int i = 16 * C + 4 * c;
+            ptx::st_shared_v4(row + ((c ^ sw) << 4), r[i], r[i + 1], r[i + 2], r[i + 3]);
         }
-    }
-    if (p.epi == OSM_EPI_F32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + row * p.N + col0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     } else {
-        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = 32 * C + 8 * c + 2 * j;
+                const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                w[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            ptx::st_shared_v4(row + ((c ^ sw) << 4), w[0], w[1], w[2], w[3]);
         }
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.Y) + row * p.N + col0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
     }
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) dual_gemm_kernel(const __grid_constant__ GemmParams p) {
+// Stage chunk C and hand it to the tensor store; `seq` counts this warp's
+// chunks so the two staging buffers alternate.
+template <int C, bool BF16>
+__device__ __forceinline__ void emit_chunk(const GemmParams& p, Smem& S, int ew, int lane, const uint32_t (&r)[128],
+                                           int32_t x, int32_t y, uint32_t& seq) {
+    const uint32_t buf = ptx::smem_u32(S.epi[ew][seq & 1]);
+    if (lane == 0) ptx::bulk_wait_group_read<1>();  // the store that last read this buffer is done with it
+    __syncwarp();
+    stage_chunk<C, BF16>(buf, lane, r);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        ptx::tma_store_2d(&p.tm_y, x, y, buf);
+        ptx::bulk_commit_group();
+    }
+    ++seq;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    dual_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
+    const bool leader = rank == 0;
+    const int pair = static_cast<int>(ptx::cluster_id_x());
+    const int npairs = static_cast<int>(ptx::num_clusters_x());
     const int tiles = p.num_m * p.num_n;
     const int ksteps = p.n_fp4 + p.n_hp;
     const volatile int* abort = &S.abort_flag;
@@ -168,84 +211,100 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) dual_gemm_kernel(const __grid_
             ptx::mbar_init(ptx::smem_u32(&S.empty[s]), 1);
         }
         ptx::mbar_init(ptx::smem_u32(&S.acc_full), 1);
-        ptx::mbar_init(ptx::smem_u32(&S.acc_empty), 4);
+        ptx::mbar_init(ptx::smem_u32(&S.acc_empty), 2 * NUM_EPI_WARPS);
         ptx::mbar_init(ptx::smem_u32(&S.drain), 1);
         S.abort_flag = 0;
         never = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        if (p.n_fp4) { ptx::prefetch_tmap(&p.tm_a); ptx::prefetch_tmap(&p.tm_b); }
+        if (p.n_fp4) {
+            ptx::prefetch_tmap(&p.tm_a);
+            ptx::prefetch_tmap(&p.tm_b);
+            ptx::prefetch_tmap(&p.tm_sa);
+            ptx::prefetch_tmap(&p.tm_sb);
+        }
         if (p.n_hp) { ptx::prefetch_tmap(&p.tm_ah); ptx::prefetch_tmap(&p.tm_bh); }
+        ptx::prefetch_tmap(&p.tm_y);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_u32(&S.tmem_base), TMEM_COLS);
-        ptx::tmem_relinquish();
+        ptx::tmem_alloc_pair(ptx::smem_u32(&S.tmem_base), TMEM_COLS);
+        ptx::tmem_relinquish_pair();
     }
+    __syncwarp();
     ptx::tc_fence_before();
-    __syncthreads();
+    ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
     ptx::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------------ TMA producer (both CTAs)
         if (ptx::elect_one()) {
             int stage = 0;
             uint32_t phase = 0;
-            int issued[STAGES];
-            uint32_t issued_phase[STAGES];
-            for (int s = 0; s < STAGES; ++s) issued[s] = 0, issued_phase[s] = 0;
+            int last_stage = -1;
+            uint32_t last_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < tiles && ok; tile += npairs) {
                 int m_blk, n_blk;
                 tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
-                const int m0 = m_blk * BM, n0 = n_blk * BN;
-                const int nbt = min(2, p.n_row_tiles - 2 * n_blk);  // valid 128-row scale tiles of W
+                const int arow = m_blk * 2 * BM + static_cast<int>(rank) * BM;        // this CTA's A rows
+                const int brow = n_blk * BN + static_cast<int>(rank) * (BN / 2);      // this CTA's B rows
+                const int nbt = min(2, p.n_row_tiles - 2 * n_blk);                   // valid B scale row tiles
+                const int sfa_tile = 2 * m_blk + static_cast<int>(rank);              // A scale row tile
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    const uint32_t eb = ptx::smem_u32(&S.empty[stage]);
-                    if (!ptx::mbar_wait_bounded(eb, phase ^ 1u, p.wait_limit_ns, abort)) {
+                    if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.empty[stage]), phase ^ 1u, p.wait_limit_ns,
+                                                abort)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = ptx::smem_u32(&S.full[stage]);
+                    const uint32_t fb = ptx::mapa(ptx::smem_u32(&S.full[stage]), 0);  // leader's barrier
                     if (ks < p.n_fp4) {
                         const int natoms = min(2, p.katoms - 2 * ks);
-                        const uint32_t sf_bytes = natoms * 512u;
-                        ptx::mbar_arrive_expect_tx(fb, A_TILE + B_TILE + sf_bytes * (1 + nbt));
-                        ptx::tma_load_2d(ptx::smem_u32(S.a[stage]), &p.tm_a, ks * 128, m0, fb);
-                        ptx::tma_load_2d(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, n0, fb);
-                        ptx::bulk_load(ptx::smem_u32(S.sfa[stage]),
-                                       p.a_scales + ((int64_t)m_blk * p.katoms + 2 * ks) * 512, sf_bytes, fb);
-                        for (int h = 0; h < nbt; ++h)
-                            ptx::bulk_load(ptx::smem_u32(S.sfb[stage]) + h * 1024,
-                                           p.w_scales + ((int64_t)(2 * n_blk + h) * p.katoms + 2 * ks) * 512,
-                                           sf_bytes, fb);
+                        if (leader)
+                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]),
+                                                       2u * (A_TILE + B_TILE + natoms * 512u * (1u + nbt)));
+                        ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_a, ks * 128, arow, fb);
+                        ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, brow, fb);
+                        for (int a = 0; a < natoms; ++a) {
+                            ptx::tma_load_2d_pair(ptx::smem_u32(S.sfa[stage]) + 512 * a, &p.tm_sa, 0,
+                                                  (sfa_tile * p.katoms + 2 * ks + a) * 32, fb);
+                            for (int h = 0; h < nbt; ++h)
+                                ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + 1024 * h + 512 * a, &p.tm_sb, 0,
+                                                      ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 32, fb);
+                        }
                     } else {
                         const int kh = ks - p.n_fp4;
-                        ptx::mbar_arrive_expect_tx(fb, A_TILE + B_TILE);
-                        ptx::tma_load_2d(ptx::smem_u32(S.a[stage]), &p.tm_ah, kh * 64, m0, fb);
-                        ptx::tma_load_2d(ptx::smem_u32(S.b[stage]), &p.tm_bh, kh * 64, n0, fb);
+                        if (leader)
+                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]), 2u * (A_TILE + B_TILE));
+                        ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_ah, kh * 64, arow, fb);
+                        ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_bh, kh * 64, brow, fb);
                     }
-                    issued[stage] = 1;
-                    issued_phase[stage] = phase;
+                    last_stage = stage;
+                    last_phase = phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
             if (!ok) raise_abort(S, p.status);
-            // every copy this thread issued has landed before the CTA can exit
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s])
-                    ptx::mbar_wait_bounded(ptx::smem_u32(&S.full[s]), issued_phase[s], drain_ns, &never);
+            // Let every copy this thread issued land before the pair exits: the
+            // last slot it filled is released (empty) only after the MMAs that
+            // read it completed, which implies all earlier copies completed too.
+            if (last_stage >= 0) {
+                if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.empty[last_stage]), last_phase, drain_ns,
+                                                    &never))
+                    ptx::spin_ns(1000000);  // an aborted pipeline: give any in-flight copy ample time to land
+            }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
-        if (ptx::elect_one()) {
+        // ------------------------------------------------------ MMA issuer (leader CTA)
+        if (leader && ptx::elect_one()) {
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             const uint32_t acc = tmem;  // lane 0, column 0
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-                if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.acc_empty), acc_phase ^ 1u, p.wait_limit_ns, abort)) {
+            for (int tile = pair; tile < tiles && ok; tile += npairs) {
+                if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.acc_empty), acc_phase ^ 1u, p.wait_limit_ns,
+                                                    abort)) {
                     ok = false;
                     break;
                 }
@@ -266,42 +325,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) dual_gemm_kernel(const __grid_
                         const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
                         const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
                         for (int a = 0; a < natoms; ++a) {
-                            ptx::tc_cp_32x128_x4(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
-                            ptx::tc_cp_32x128_x4(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
-                            ptx::tc_cp_32x128_x4(sfb_col + 8 * a + 4, desc_sf(sfb_s + 1024 + 512 * a));
+                            ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
+                            ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
+                            ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + 1024 + 512 * a));
                         }
                         for (int kk = 0; kk < 2 * natoms; ++kk) {
                             const uint32_t sf_id = (uint32_t)(kk & 1) * 2u;  // bytes 0-1 or 2-3 of the atom
                             const uint32_t idesc = IDESC_MXF4 | (sf_id << 29) | (sf_id << 4);
-                            ptx::mma_mxf4(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32), idesc,
-                                          sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
+                            ptx::mma_mxf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32), idesc,
+                                               sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
                             accumulate = 1;
                         }
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            ptx::mma_bf16(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
-                                          IDESC_BF16, accumulate);
+                            ptx::mma_bf16_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                                               IDESC_BF16, accumulate);
                             accumulate = 1;
                         }
                     }
-                    ptx::tc_commit(ptx::smem_u32(&S.empty[stage]));
+                    ptx::tc_commit_pair_mc(ptx::smem_u32(&S.empty[stage]), PAIR_MASK);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                ptx::tc_commit(ptx::smem_u32(&S.acc_full));
+                ptx::tc_commit_pair_mc(ptx::smem_u32(&S.acc_full), PAIR_MASK);
                 acc_phase ^= 1u;
             }
             if (!ok) raise_abort(S, p.status);
             // all issued tensor-core work has finished before tensor memory is freed
-            ptx::tc_commit(ptx::smem_u32(&S.drain));
+            ptx::tc_commit_pair_mc(ptx::smem_u32(&S.drain), 0x1);
             ptx::mbar_wait_bounded(ptx::smem_u32(&S.drain), 0, drain_ns, &never);
         }
     } else {
-        // ------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
-        uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        // ------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;           // TMEM lanes 32q..32q+31 are reachable from this warp
+        const int half = (warp - 2) >> 2;  // columns [128*half, 128*half + 128) of the tile
+        const int ew = warp - 2;          // staging buffers of this warp
+        const uint32_t acc_empty_leader = ptx::mapa(ptx::smem_u32(&S.acc_empty), 0);
+        uint32_t acc_phase = 0, seq = 0;
+        for (int tile = pair; tile < tiles; tile += npairs) {
             int m_blk, n_blk;
             tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
             int ok = 1;
@@ -313,29 +375,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) dual_gemm_kernel(const __grid_
                 break;
             }
             ptx::tc_fence_after();
-            const int64_t row = (int64_t)m_blk * BM + q * 32 + lane;
-            const int64_t n0 = (int64_t)n_blk * BN;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                ptx::tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c * 32, r);
-                ptx::tmem_ld_wait();
-                const int64_t col0 = n0 + c * 32;
-                if (row < p.M && col0 < p.N) store_chunk(p, row, col0, r);
-            }
+            uint32_t r[128];
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + half * 128;
+            ptx::tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            ptx::tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            ptx::tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+            ptx::tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+            ptx::tmem_ld_wait();
+            // the accumulator is in registers: hand tensor memory back to the leader's MMA issuer
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&S.acc_empty));
+            if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
             acc_phase ^= 1u;
+            if (p.bias) {
+                const int64_t col0 = (int64_t)n_blk * BN + half * 128;
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    r[i] = __float_as_uint(__uint_as_float(r[i]) + (col0 + i < p.N ? __ldg(p.bias + col0 + i) : 0.0f));
+            }
+            const int32_t y0 = m_blk * 2 * BM + static_cast<int>(rank) * BM + q * 32;
+            const int32_t x0 = n_blk * BN + half * 128;
+            if (p.epi == OSM_EPI_F32) {
+                emit_chunk<0, false>(p, S, ew, lane, r, x0, y0, seq);
+                emit_chunk<1, false>(p, S, ew, lane, r, x0 + 16, y0, seq);
+                emit_chunk<2, false>(p, S, ew, lane, r, x0 + 32, y0, seq);
+                emit_chunk<3, false>(p, S, ew, lane, r, x0 + 48, y0, seq);
+                emit_chunk<4, false>(p, S, ew, lane, r, x0 + 64, y0, seq);
+                emit_chunk<5, false>(p, S, ew, lane, r, x0 + 80, y0, seq);
+                emit_chunk<6, false>(p, S, ew, lane, r, x0 + 96, y0, seq);
+                emit_chunk<7, false>(p, S, ew, lane, r, x0 + 112, y0, seq);
+            } else {
+                emit_chunk<0, true>(p, S, ew, lane, r, x0, y0, seq);
+                emit_chunk<1, true>(p, S, ew, lane, r, x0 + 32, y0, seq);
+                emit_chunk<2, true>(p, S, ew, lane, r, x0 + 64, y0, seq);
+                emit_chunk<3, true>(p, S, ew, lane, r, x0 + 96, y0, seq);
+            }
         }
+        if (lane == 0) ptx::bulk_wait_group_all();  // every tensor store of this warp has completed
     }
 
+    __syncwarp();  // lanes that skipped a single-thread role wait here for their elected lane
     ptx::tc_fence_before();
-    __syncthreads();
+    ptx::cluster_sync();  // both CTAs done: no MMA, copy or tensor-memory read in flight
     if (warp == 1) {
         __syncwarp();
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, TMEM_COLS);
+        ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -355,19 +440,24 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 int make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
-             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, const char* what) {
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz,
+             const char* what) {
     auto enc = get_encode_fn();
     if (!enc) return fail(OSM_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {row_stride_bytes};
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(OSM_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
     return OSM_OK;
 }
+
+struct LaunchInfo {
+    int max_pairs = 0;
+    bool ready = false;
+};
 
 }  // namespace
 
@@ -380,24 +470,40 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
     int rc;
+    const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B, NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
     if (pl->Kbp > 0) {
-        if ((rc = make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, pl->Kbp / 2, M, pl->Kbp / 2, 128, BM,
+        if ((rc = make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, pl->Kbp / 2, M, pl->Kbp / 2, 128, BM, SW,
                            "a_codes")))
             return rc;
         if ((rc = make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, pl->Kbp / 2, pl->N, pl->Kbp / 2, 128,
-                           BN, "w_codes")))
+                           BN / 2, SW, "w_codes")))
+            return rc;
+        const uint64_t sa_rows = static_cast<uint64_t>(scales_bytes(M, pl->Kbp)) / 16;
+        const uint64_t sb_rows = static_cast<uint64_t>(scales_bytes(pl->N, pl->Kbp)) / 16;
+        if ((rc = make_map(&p.tm_sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 16, sa_rows, 16, 16, 32, NOSW,
+                           "a_scales")))
+            return rc;
+        if ((rc = make_map(&p.tm_sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 16, sb_rows, 16, 16, 32, NOSW,
+                           "w_scales")))
             return rc;
     }
     if (pl->kp > 0) {
-        if ((rc = make_map(&p.tm_ah, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_hp, pl->kp, M, pl->kp * 2, 64, BM,
+        if ((rc = make_map(&p.tm_ah, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_hp, pl->kp, M, pl->kp * 2, 64, BM, SW,
                            "a_hp")))
             return rc;
-        if ((rc = make_map(&p.tm_bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_hp, pl->kp, pl->N, pl->kp * 2, 64, BN,
-                           "w_hp")))
+        if ((rc = make_map(&p.tm_bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_hp, pl->kp, pl->N, pl->kp * 2, 64, BN / 2,
+                           SW, "w_hp")))
             return rc;
     }
-    p.a_scales = a_scales;
-    p.w_scales = w_scales;
+    if (epi == OSM_EPI_F32) {
+        if ((rc = make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, pl->N, M, pl->N * 4, 16, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B, "Y")))
+            return rc;
+    } else {
+        if ((rc = make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, pl->N, M, pl->N * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B, "Y")))
+            return rc;
+    }
     p.bias = bias;
     p.Y = Y;
     p.status = pl->d_status;
@@ -407,24 +513,49 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     p.katoms = static_cast<int>(pl->Kbp / 128);
     p.n_fp4 = (p.katoms + 1) / 2;
     p.n_hp = static_cast<int>(pl->kp / 64);
-    p.num_m = static_cast<int>(ceil_div(M, BM));
+    p.num_m = static_cast<int>(ceil_div(M, 2 * BM));
     p.num_n = static_cast<int>(ceil_div(pl->N, BN));
     p.n_row_tiles = static_cast<int>(ceil_div(pl->N, 128));
     p.epi = epi;
 
-    int dev = 0, sms = 0;
+    // co-resident clusters of two CTAs, queried once per device
+    static LaunchInfo info[64];
+    static std::mutex mu;
+    int dev = 0;
     if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
-    if ((rc = check_cuda(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count")))
-        return rc;
+    if (dev < 0 || dev >= 64) return fail(OSM_ERR_UNSUPPORTED, "device index %d", dev);
     const size_t smem = sizeof(Smem) + 1024;
-    if ((rc = check_cuda(cudaFuncSetAttribute(dual_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(smem)),
-                         "dual_gemm smem attribute")))
-        return rc;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!info[dev].ready) {
+            if ((rc = check_cuda(cudaFuncSetAttribute(dual_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(smem)),
+                                 "dual_gemm smem attribute")))
+                return rc;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2, 1, 1);
+            cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if ((rc = check_cuda(cudaOccupancyMaxActiveClusters(&clusters, dual_gemm_kernel, &cfg),
+                                 "dual_gemm cluster occupancy")))
+                return rc;
+            if (clusters < 1) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: no CTA pair fits on this device");
+            info[dev].max_pairs = clusters;
+            info[dev].ready = true;
+        }
+    }
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
     if (tiles > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: too many tiles");
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    dual_gemm_kernel<<<grid, NUM_THREADS, smem, st>>>(p);
+    const int pairs = static_cast<int>(tiles < info[dev].max_pairs ? tiles : info[dev].max_pairs);
+    dual_gemm_kernel<<<2 * pairs, NUM_THREADS, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "dual_gemm launch");
 }
 

@@ -14,8 +14,9 @@ struct osm_plan {
     // device tables, owned by the plan
     float* d_s;          // [K]  smoothing vector s (Eq. (2))
     float* d_inv_s;      // [K]  1.0f / s
-    int32_t* d_route;    // [K]  destination of channel j inside a staged row:
-                         //      bulk position p in [0, Kb) or Kbp + i for outlier slot i
+    int32_t* d_route;    // [K]  byte offset of channel j inside a row staged by quantize_act:
+                         //      bulk position p -> (p/32)*QA_BLOCK_BYTES + (p%32)*2,
+                         //      outlier slot i  -> (Kbp/32)*QA_BLOCK_BYTES + 2*i
     int32_t* d_J;        // [Kb] bulk position -> channel (ascending)
     int32_t* d_O;        // [k]  outlier slot -> channel (ascending)
     uint32_t* d_status;  // OSM_STATUS_* bits written by kernels
@@ -23,6 +24,10 @@ struct osm_plan {
 };
 
 namespace osm {
+
+// Bytes of one 32-value bulk block in a row staged by quantize_act
+// (64 bytes of BF16 plus 16 bytes of padding against bank conflicts).
+constexpr int QA_BLOCK_BYTES = 80;
 
 // thread-local error message
 void set_error(const char* fmt, ...);

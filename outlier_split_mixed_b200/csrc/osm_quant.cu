@@ -45,35 +45,6 @@ __device__ __forceinline__ float exp2_neg(int X) {
                     : __uint_as_float(0x00400000u >> (X - 127));
 }
 
-// Eight non-negative magnitudes -> eight E2M1 codes (round to nearest even,
-// saturating at 6), element i in nibble i.
-__device__ __forceinline__ uint32_t e2m1x8(const float (&a)[8]) {
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(out)
-        : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
-    return out;
-}
-
-// Encode 8 BF16 values (bits in h[0..7]) with shared exponent X. The sign
-// bit of each code is the sign bit of the BF16 input.
-__device__ __forceinline__ uint32_t encode8(const uint32_t (&h)[8], int X) {
-    const float inv = exp2_neg(X);
-    float a[8];
-    uint32_t signs = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        a[i] = bf16_bits_to_f32(h[i] & 0x7FFFu) * inv;  // exact: power-of-two scaling
-        signs |= ((h[i] >> 15) & 1u) << (4 * i + 3);
-    }
-    return e2m1x8(a) | signs;
-}
-
 // Byte offset of E8M0 scale (row r, 32-block b) in the tcgen05 block-scale
 // layout: 512-byte atoms of 128 rows x 4 blocks.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t b, int64_t katoms) {
@@ -86,6 +57,47 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+__device__ __forceinline__ uint32_t ldg_nc_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Two FP32 values -> E2M1x2 (round to nearest even, saturating at +-6):
+// element `lo` in the low nibble. The sign of the code is the sign of the
+// input, including for inputs that round to zero.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint16_t out;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+        "cvt.u16.u8 %0, b;\n\t}"
+        : "=h"(out)
+        : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Eight BF16 values (4 packed words) scaled by `inv` (a power of two, so
+// exact) -> eight E2M1 codes, element i in nibble i.
+__device__ __forceinline__ uint32_t encode8_words(uint4 q, float inv) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16) * inv;
+        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
+        out |= e2m1x2(lo, hi) << (8 * i);
+    }
+    return out;
 }
 
 // ------------------------------------------------------------ calibration
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(256) pack_bulk_kernel(PackParams p) {
     const int64_t katoms = p.Kbp / 128;
     if (strip >= katoms) return;  // uniform per warp
     const bool nvalid = n < p.N;
-    uint32_t h[128];
+    uint32_t h[64];  // 128 folded BF16 weights, two per word
     float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 128; ++i) {
@@ -174,7 +186,7 @@ __global__ void __launch_bounds__(256) pack_bulk_kernel(PackParams p) {
             const float w = bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + n]);
             bits = f32_to_bf16_bits(w * __ldg(p.s + j));
         }
-        h[i] = bits;
+        if (i & 1) h[i >> 1] |= bits << 16; else h[i >> 1] = bits;
         am[i >> 5] = fmaxf(am[i >> 5], bf16_bits_to_f32(bits & 0x7FFFu));
     }
     if (p.mode == OSM_WSCALE_STRIP128x1) {
@@ -194,15 +206,12 @@ __global__ void __launch_bounds__(256) pack_bulk_kernel(PackParams p) {
         const uint32_t code = (nvalid && pos0 < p.Kb) ? static_cast<uint32_t>(X + 127) : 0u;
         sc |= code << (8 * b);
         if (nvalid) {
+            const float inv = exp2_neg(X);
             uint4 out;
-            uint32_t* o4 = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint32_t hh[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) hh[e] = h[b * 32 + g * 8 + e];
-                o4[g] = encode8(hh, X);
-            }
+            out.x = encode8_words(make_uint4(h[16 * b + 0], h[16 * b + 1], h[16 * b + 2], h[16 * b + 3]), inv);
+            out.y = encode8_words(make_uint4(h[16 * b + 4], h[16 * b + 5], h[16 * b + 6], h[16 * b + 7]), inv);
+            out.z = encode8_words(make_uint4(h[16 * b + 8], h[16 * b + 9], h[16 * b + 10], h[16 * b + 11]), inv);
+            out.w = encode8_words(make_uint4(h[16 * b + 12], h[16 * b + 13], h[16 * b + 14], h[16 * b + 15]), inv);
             *reinterpret_cast<uint4*>(p.codes + n * (p.Kbp / 2) + strip * 64 + b * 16) = out;
         }
     }
@@ -230,8 +239,8 @@ __global__ void __launch_bounds__(256) pack_hp_kernel(PackParams p) {
 struct QuantParams {
     const uint16_t* X;       // [M][K]
     const float* inv_s;      // [K]
-    const int32_t* route;    // [K]
-    int64_t M, K, k, Kb, Kbp, kp;
+    const int32_t* route;    // [K] byte offset of channel j inside a staged row
+    int M, K, k, Kb, Kbp, kp;
     uint8_t* codes;          // [M][Kbp/2]
     uint8_t* scales;         // layout, rows padded to 128
     uint16_t* hp;            // [M][kp]
@@ -239,110 +248,122 @@ struct QuantParams {
 
 constexpr int QA_THREADS = 256;
 
-// Each CTA handles R consecutive rows.
-//  phase 1: coalesced 16-byte loads of the rows; x' = bf16(x * inv_s) is
-//           scattered into a shared-memory row in [bulk J | outliers O]
-//           order (the routing table is the channel -> slot map);
-//  phase 2: four threads per 32-block of the compacted bulk row: 16-byte
-//           shared loads, amax by two xor-shuffles, E8M0 scale, E2M1 codes
-//           (one coalesced 32-bit store per thread);
-//  phase 3: the outlier slots go out as 16-byte stores.
+__host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * QA_BLOCK_BYTES + kp * 2 + 15) & ~15; }
+
+// Each CTA handles R consecutive rows, staged in shared memory in
+// [bulk blocks | outlier slots] order; a bulk block of 32 BF16 values takes
+// 80 bytes (64 + 16 padding) so that phase 2's 128-bit reads by consecutive
+// threads hit distinct banks.
+//  phase 1: each lane loads 2 channels (32-bit) of each of the R rows -- a
+//           warp reads 128 contiguous bytes per row -- computes
+//           x' = bf16(x * inv_s) and stores both values at their routed
+//           offsets (bulk position or outlier slot); consecutive lanes write
+//           into one 128-byte window, so the stores are conflict-free;
+//  phase 2: one thread per (row, 32-block): four 128-bit shared loads,
+//           amax by packed u16 max, E8M0 exponent, sixteen E2M1x2
+//           conversions, one 128-bit code store and one scale byte;
+//  phase 3: the outlier slots go out as 128-bit stores.
 template <int R>
 __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p) {
-    extern __shared__ __align__(16) uint16_t srow[];
-    const int64_t W = p.Kbp + p.kp;             // staged row length (elements)
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
+    extern __shared__ __align__(16) uint8_t sbuf[];
+    constexpr int UNROLL = 16 / R;
+    const int nb = p.Kbp >> 5;
+    const int stride = qa_row_stride(nb, p.kp);
+    const int row0 = blockIdx.x * R;
     const int tid = threadIdx.x;
 
-    // zero the padding slots [Kb, Kbp) and [Kbp + k, Kbp + kp)
-    const int64_t npad_b = p.Kbp - p.Kb, npad_h = p.kp - p.k;
-    for (int64_t i = tid; i < R * (npad_b + npad_h); i += QA_THREADS) {
-        const int64_t r = i / (npad_b + npad_h), c = i % (npad_b + npad_h);
-        const int64_t col = c < npad_b ? p.Kb + c : p.Kbp + p.k + (c - npad_b);
-        srow[r * W + col] = 0;
+    // zero the padding slots: bulk positions [Kb, Kbp) and outlier slots [k, kp)
+    {
+        const int npb = p.Kbp - p.Kb, npad = npb + (p.kp - p.k);
+        for (int i = tid; i < R * npad; i += QA_THREADS) {
+            const int r = i / npad, c = i - r * npad;
+            const int pos = p.Kb + c;
+            const int off = c < npb ? (pos >> 5) * QA_BLOCK_BYTES + (pos & 31) * 2
+                                    : nb * QA_BLOCK_BYTES + (p.k + c - npb) * 2;
+            *reinterpret_cast<uint16_t*>(sbuf + r * stride + off) = 0;
+        }
     }
 
     // phase 1
-    const int64_t nvec = p.K / 8;
-    for (int64_t v = tid; v < nvec; v += QA_THREADS) {
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.inv_s + v * 8));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.inv_s + v * 8 + 4));
-        const int4 d0 = __ldg(reinterpret_cast<const int4*>(p.route + v * 8));
-        const int4 d1 = __ldg(reinterpret_cast<const int4*>(p.route + v * 8 + 4));
-        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const int dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-        uint4 xv[R];
+    const int npairs = p.K >> 1;
+    const uint32_t* X32 = reinterpret_cast<const uint32_t*>(p.X);
+    const float2* is2 = reinterpret_cast<const float2*>(p.inv_s);
+    const int2* rt2 = reinterpret_cast<const int2*>(p.route);
+    for (int c0 = tid; c0 < npairs; c0 += QA_THREADS * UNROLL) {
+        uint32_t w[UNROLL][R];
+        float2 sv[UNROLL];
+        int2 dv[UNROLL];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t t = row0 + r;
-            xv[r] = (t < p.M) ? ldg_nc_v4(p.X + t * p.K + v * 8) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < UNROLL; ++u) {
+            const int c = c0 + u * QA_THREADS;
+            if (c < npairs) {
+                sv[u] = __ldg(is2 + c);
+                dv[u] = __ldg(rt2 + c);
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    w[u][r] = (row0 + r < p.M) ? ldg_nc_u32(X32 + static_cast<size_t>(row0 + r) * npairs + c) : 0u;
+            }
         }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const uint32_t w[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
+        for (int u = 0; u < UNROLL; ++u) {
+            const int c = c0 + u * QA_THREADS;
+            if (c < npairs) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t hb = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-                const float xs = bf16_bits_to_f32(hb) * sv[i];
-                srow[r * W + dv[i]] = static_cast<uint16_t>(f32_to_bf16_bits(xs));
+                for (int r = 0; r < R; ++r) {
+                    const float lo = __uint_as_float(w[u][r] << 16) * sv[u].x;
+                    const float hi = __uint_as_float(w[u][r] & 0xFFFF0000u) * sv[u].y;
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+                    const uint32_t pk = *reinterpret_cast<const uint32_t*>(&h);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].x) = static_cast<uint16_t>(pk);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].y) = static_cast<uint16_t>(pk >> 16);
+                }
             }
         }
     }
     __syncthreads();
 
     // phase 2
-    const int64_t G = p.Kbp / 8;   // 8-element groups per row
-    const int64_t katoms = p.Kbp / 128;
-    const int lane = tid & 31;
-    for (int64_t gb = (tid & ~31); gb < R * G; gb += QA_THREADS) {
-        const int64_t g = gb + lane;
-        const bool valid = g < R * G;
-        const int64_t r = valid ? g / G : 0, q = valid ? g % G : 0;
-        uint32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (valid) {
-            const uint4 u = *reinterpret_cast<const uint4*>(srow + r * W + q * 8);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                h[2 * i] = w[i] & 0xFFFFu;
-                h[2 * i + 1] = w[i] >> 16;
-            }
-        }
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = max(m, h[i] & 0x7FFFu);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const int X = mx_exponent(bf16_bits_to_f32(m));
-        const uint32_t word = encode8(h, X);
-        const int64_t t = row0 + r;
-        if (valid && t < p.M) {
-            *reinterpret_cast<uint32_t*>(p.codes + t * (p.Kbp / 2) + q * 4) = word;
-            if ((q & 3) == 0) {
-                const int64_t b = q >> 2;
-                p.scales[sf_offset(t, b, katoms)] =
-                    static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
-            }
-        }
+    const int katoms = p.Kbp >> 7;
+    for (int wi = tid; wi < R * nb; wi += QA_THREADS) {
+        const int r = wi / nb, b = wi - r * nb;
+        const int t = row0 + r;
+        if (t >= p.M) continue;
+        const uint8_t* src = sbuf + r * stride + b * QA_BLOCK_BYTES;
+        const uint4 q0 = lds128(src), q1 = lds128(src + 16), q2 = lds128(src + 32), q3 = lds128(src + 48);
+        uint32_t m = vmax_u16x2(vmax_u16x2(q0.x & 0x7FFF7FFFu, q0.y & 0x7FFF7FFFu),
+                                vmax_u16x2(q0.z & 0x7FFF7FFFu, q0.w & 0x7FFF7FFFu));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q1.x & 0x7FFF7FFFu, q1.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q1.z & 0x7FFF7FFFu, q1.w & 0x7FFF7FFFu)));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q2.x & 0x7FFF7FFFu, q2.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q2.z & 0x7FFF7FFFu, q2.w & 0x7FFF7FFFu)));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q3.x & 0x7FFF7FFFu, q3.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q3.z & 0x7FFF7FFFu, q3.w & 0x7FFF7FFFu)));
+        const uint32_t amax = max(m & 0xFFFFu, m >> 16);
+        const int X = mx_exponent(bf16_bits_to_f32(amax));
+        const float inv = exp2_neg(X);
+        const uint4 out = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv), encode8_words(q2, inv),
+                                     encode8_words(q3, inv));
+        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16) = out;
+        p.scales[sf_offset(t, b, katoms)] = static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
     }
 
     // phase 3: outlier slots
-    const int64_t hv = p.kp / 8;
-    for (int64_t i = tid; i < R * hv; i += QA_THREADS) {
-        const int64_t r = i / hv, c = i % hv;
-        const int64_t t = row0 + r;
+    const int hv = p.kp >> 3;
+    for (int i = tid; i < R * hv; i += QA_THREADS) {
+        const int r = i / hv, c = i - r * hv;
+        const int t = row0 + r;
         if (t < p.M)
-            *reinterpret_cast<uint4*>(p.hp + t * p.kp + c * 8) =
-                *reinterpret_cast<const uint4*>(srow + r * W + p.Kbp + c * 8);
+            *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(t) * p.kp + c * 8) =
+                lds128(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
     }
 
     // scale bytes of the padding rows [M, round_up(M,128)) are zero
     if (row0 <= p.M - 1 && p.M - 1 < row0 + R && (p.M & 127) != 0) {
-        const int64_t tile = (p.M - 1) >> 7;
-        const int64_t rem = p.M & 127;
-        const int64_t nwords = (128 - rem) * katoms;
-        for (int64_t i = tid; i < nwords; i += QA_THREADS) {
-            const int64_t rr = rem + i % (128 - rem), a = i / (128 - rem);
+        const int tile = (p.M - 1) >> 7;
+        const int rem = p.M & 127;
+        const int nwords = (128 - rem) * katoms;
+        for (int i = tid; i < nwords; i += QA_THREADS) {
+            const int a = i / (128 - rem), rr = rem + (i - a * (128 - rem));
             *reinterpret_cast<uint32_t*>(p.scales + sf_offset(tile * 128 + rr, a * 4, katoms)) = 0u;
         }
     }
@@ -394,16 +415,18 @@ static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
         if (rc) return rc;
     }
     const int64_t grid = ceil_div(p.M, R);
-    if (grid > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: M too large");
     kern<<<static_cast<unsigned>(grid), QA_THREADS, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
 int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st) {
-    QuantParams p{X, pl->d_inv_s, pl->d_route, M, pl->K, pl->k, pl->Kb, pl->Kbp, pl->kp, codes, scales, hp};
-    const size_t row_bytes = static_cast<size_t>(pl->Kbp + pl->kp) * 2;
-    const size_t budget = 64 * 1024;
+    if (M > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: M too large");
+    QuantParams p{X, pl->d_inv_s, pl->d_route, static_cast<int>(M), static_cast<int>(pl->K),
+                  static_cast<int>(pl->k), static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp),
+                  static_cast<int>(pl->kp), codes, scales, hp};
+    const size_t row_bytes = static_cast<size_t>(qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp)));
+    const size_t budget = 72 * 1024;
     if (row_bytes * 8 <= budget) return launch_qa<8>(p, row_bytes * 8, st);
     if (row_bytes * 4 <= budget) return launch_qa<4>(p, row_bytes * 4, st);
     if (row_bytes * 2 <= budget) return launch_qa<2>(p, row_bytes * 2, st);
