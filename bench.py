@@ -167,6 +167,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     import torch.distributed as dist
 
     import outlier_split_mixed_b200 as osm
+    from outlier_split_mixed_b200 import dist as odist
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -185,9 +186,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     wmax = torch.empty(K, dtype=torch.float32, device=dev)
     osm.act_amax_accumulate(Xd, amax)
     osm.weight_amax(Wd, wmax)
-    if world > 1:
-        dist.all_reduce(amax, op=dist.ReduceOp.MAX)
-    s, inv_s, O = osm.calibrate_finalize(amax.cpu().numpy(), wmax.cpu().numpy(), cfg.alpha, cfg.k)
+    s, inv_s, O = odist.calibrate_from_local_stats(amax, wmax, cfg.alpha, cfg.k)
     plan = osm.Plan(K, N, cfg.k, s, O, cfg.wmode)
     wc, wsc, wh = plan.alloc_packed(N, dev)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
