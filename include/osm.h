@@ -125,7 +125,7 @@ OSM_API int osm_calibrate_finalize(const float* amax_host, const float* wmax_hos
  * smoothing vector s (host float[K], > 0, finite) and ascending outlier set
  * O (host int32[k], distinct, in [0, K)). The plan owns device copies of
  * inv_s = 1.0f/s, the channel routing table and a status word.
- * Requirements: K % 32 == 0, N % 32 == 0, 0 <= k <= K, K <= 65504.
+ * Requirements: K % 32 == 0, N % 32 == 0, 0 <= k <= K, K <= 65536.
  * The plan is bound to the current CUDA device. */
 OSM_API int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const int32_t* O_host,
                     int wscale_mode, osm_plan** out);
@@ -204,6 +204,30 @@ OSM_API size_t osm_linear_workspace_size(const osm_plan* plan, int64_t M, int ep
 OSM_API int osm_linear_host(const osm_plan* plan, const uint16_t* X_host, int64_t M, const uint8_t* w_codes,
                     const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi,
                     void* Y_host, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- allocation-free device forward --------------------------------------
+ * The paper has no counterpart to this entry point; it serves callers that
+ * build their plans and pack their weights at load time but may not
+ * allocate device memory while the layer runs (code captured into a CUDA
+ * graph, or a runtime whose device memory belongs to its own pool).
+ *
+ * Same result as osm_quantize_act followed by osm_dual_gemm, on device
+ * X [M][K] BF16 and device Y [M][N] (F32 or BF16, per epi), with no
+ * activation buffers from the caller: the packed activations live in a
+ * static device array of OSM_NOALLOC_SCRATCH_BYTES inside the library
+ * (every GPU that loads the library holds one until the process exits).
+ * It calls no allocator. A call whose packed activations (codes + scales +
+ * outlier slots, each rounded up to 256 bytes; see osm_plan_sizes) exceed
+ * the array returns OSM_ERR_UNSUPPORTED before launching anything.
+ * The first call on a device looks up the array's device address; make
+ * that first call before any stream capture. All calls share the array:
+ * calls whose work overlaps on the GPU (different streams, or different
+ * host threads, without ordering between them) race on it. A timeout sets
+ * the plan's status word as osm_dual_gemm does. */
+#define OSM_NOALLOC_SCRATCH_BYTES (16u << 20)
+OSM_API int osm_linear_noalloc(const osm_plan* plan, const uint16_t* X, int64_t M, const uint8_t* w_codes,
+                               const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi, void* Y,
+                               void* stream);
 
 /* ---- helpers ------------------------------------------------------------ */
 

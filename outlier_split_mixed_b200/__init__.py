@@ -46,6 +46,7 @@ _SIGNATURES = {
     "osm_linear_workspace_size": (_SZ, [_P, _I64, _I]),
     "osm_linear_host": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "osm_scales_to_logical": (_I, [_P, _I64, _I64, _P]),
+    "osm_linear_noalloc": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P]),
     "osm_last_error": (ctypes.c_char_p, []),
 }
 
@@ -281,6 +282,30 @@ def linear_host(plan: Plan, X_host, M: int, w_codes, w_scales, w_hp, Y_host, wor
                                  _ptr(bias, "bias", (torch.float32,), plan.N * 4, allow_none=True), int(epi),
                                  ctypes.c_void_p(Y_host.data_ptr()), _ptr(workspace, "workspace"),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def linear_noalloc(plan: Plan, X, w_codes, w_scales, w_hp, Y, bias=None, epi: int = EPI_F32, stream=None):
+    """quantize_act + dual_gemm with the packed activations in the library's
+    static scratch (osm_linear_noalloc): nothing is allocated, for callers
+    that may not allocate device memory at run time (CUDA-graph capture,
+    pool-owned device memory). Calls that overlap on the GPU race on the
+    shared scratch; the first call on a device should precede any capture."""
+    import torch
+    M, K = X.shape
+    if K != plan.K:
+        raise ValueError("X must have K columns")
+    cbn, sbn, hbn = plan.sizes(plan.N)
+    ybytes = M * plan.N * (4 if epi == EPI_F32 else 2)
+    ytypes = (torch.float32,) if epi == EPI_F32 else _bf16_types()
+    _check(lib().osm_linear_noalloc(plan.handle, _ptr(X, "X", _bf16_types()), M,
+                                    _ptr(w_codes, "w_codes", _u8_types(), cbn, allow_none=cbn == 0),
+                                    _ptr(w_scales, "w_scales", _u8_types(), sbn, allow_none=sbn == 0),
+                                    _ptr(w_hp, "w_hp", _bf16_types(), hbn, allow_none=hbn == 0),
+                                    _ptr(bias, "bias", (torch.float32,), plan.N * 4, allow_none=True), int(epi),
+                                    _ptr(Y, "Y", ytypes, ybytes), _stream(stream)))
 
 
 def scales_to_logical(swizzled: np.ndarray, rows: int, nblocks: int) -> np.ndarray:
