@@ -25,12 +25,12 @@
 //              into tensor memory (both CTAs), the MMAs, and a multicast
 //              tcgen05.commit that frees the ring slot in both CTAs.
 //   warps 2-9  epilogue: each warp drains 32 lanes x 128 columns of its
-//              CTA's accumulator half into registers, hands tensor memory
-//              back (arrivals counted in the leader), then adds the bias and
-//              writes FP32 or BF16 through a double-buffered, 64B-swizzled
-//              shared-memory chunk and a bulk tensor store (full-line global
-//              writes, ragged M/N edges clipped by the tensor map) while the
-//              next tile's MMAs run.
+//              CTA's accumulator half into registers (16x256b loads: four
+//              lanes per row), hands tensor memory back (arrivals counted in
+//              the leader), then adds the bias and stores FP32 or BF16
+//              straight from registers in full 32-byte sectors while the
+//              next tile's MMAs run. Keeping shared memory for the operand
+//              ring (6 stages) matters more than store coalescing here.
 // Every wait is bounded by %globaltimer; a wait that runs out sets the
 // plan's status word and raises a CTA-wide abort flag; the CTA then lets
 // its in-flight copies and MMAs finish, frees tensor memory and returns.
@@ -53,14 +53,13 @@ namespace {
 
 constexpr int BM = 128;                 // accumulator rows per CTA (TMEM lanes); pair tile M = 256
 constexpr int BN = 256;                 // output columns per tile; each CTA loads BN/2 rows of B
-constexpr int STAGES = 5;
+constexpr int STAGES = 6;
 constexpr int A_TILE = BM * 128;        // one K-step of A: 128 rows x 128 bytes
 constexpr int B_TILE = (BN / 2) * 128;  // one K-step of this CTA's half of B
 constexpr int SFA_TILE = 2 * 512;       // two 128x4 scale atoms (K = 256)
 constexpr int SFB_TILE = 2 * 2 * 512;   // two 128-row tiles x two atoms (all 256 B rows)
 constexpr int NUM_EPI_WARPS = 8;        // two per TMEM lane quadrant, 128 columns each
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-constexpr int EPI_CHUNK = 2048;         // 32 rows x 64 bytes: 16 FP32 or 32 BF16 columns
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;       // scale factors live after the accumulator
 constexpr uint32_t SF_STAGE_COLS = 24;  // 8 columns for A, 16 for B per ring slot
@@ -84,7 +83,6 @@ struct __align__(1024) Smem {
     uint8_t b[STAGES][B_TILE];
     uint8_t sfa[STAGES][SFA_TILE];
     uint8_t sfb[STAGES][SFB_TILE];
-    uint8_t epi[NUM_EPI_WARPS][2][EPI_CHUNK];
     uint64_t full[STAGES];   // leader: all copies of both CTAs for the slot have landed
     uint64_t empty[STAGES];  // both: the MMAs reading the slot have completed
     uint64_t acc_full;       // both: the tile's accumulator is complete
@@ -99,9 +97,8 @@ struct GemmParams {
     CUtensorMap tm_b;    // w_codes  [N][Kbp/2] u8, box 128 x 128
     CUtensorMap tm_ah;   // a_hp     [M][kp] bf16, box 64 x 128
     CUtensorMap tm_bh;   // w_hp     [N][kp] bf16, box 64 x 128
-    CUtensorMap tm_sa;   // a_scales as [bytes/16][16] u8, box 16 x 32 (one 512-byte atom)
+    CUtensorMap tm_sa;   // a_scales as [bytes/128][128] u8, box 128 x 4 (one 512-byte atom)
     CUtensorMap tm_sb;   // w_scales likewise
-    CUtensorMap tm_y;    // Y [M][N] f32 (box 16 x 32) or bf16 (box 32 x 32), 64B swizzle
     const float* bias;
     void* Y;
     uint32_t* status;
@@ -139,54 +136,54 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
     return ptx::smem_desc(saddr, 0, 128, ptx::LAYOUT_NONE);
 }
 
-// Write one 32-row x 64-byte chunk (16 FP32 or 32 BF16 columns per row) of
-// the warp's accumulator slice into a 64B-swizzled staging buffer: row r
-// (= lane) keeps its four 16-byte pieces at positions c ^ ((r >> 1) & 3),
-// the layout the tensor map's 64B swizzle expects, which also keeps each
-// group of eight lanes on distinct banks.
-template <int C, bool BF16>
-__device__ __forceinline__ void stage_chunk(uint32_t buf, int lane, const uint32_t (&r)[128]) {
-    const uint32_t row = buf + lane * 64;
-    const int sw = (lane >> 1) & 3;
-    if (!BF16) {
+// Load one 16-lane slab of the accumulator: 16 TMEM lanes x 128 columns.
+// Thread t receives lanes t/4 and t/4 + 8 and, for each 8-column block j,
+// columns 8j + 2(t%4) and 8j + 2(t%4) + 1 (registers 4j .. 4j+3), so the
+// four lanes of a quad hold one row's 32 contiguous bytes.
+__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+// Add the bias and store one 16-row x 128-column slab from registers: each
+// store instruction of the warp writes eight full 32-byte sectors (one per
+// row), FP32 as 8-byte pairs or BF16 as 4-byte pairs. Rows >= M and
+// columns >= N (N % 32 == 0, so whole 8-column blocks) are skipped.
+__device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, int64_t col0, int lane, const uint32_t* r) {
+    const int64_t ra = row0 + (lane >> 2), rb = ra + 8;
+    const int cq = 2 * (lane & 3);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int i = 16 * C + 4 * c;
-            ptx::st_shared_v4(row + ((c ^ sw) << 4), r[i], r[i + 1], r[i + 2], r[i + 3]);
+    for (int j = 0; j < 16; ++j) {
+        const int64_t col = col0 + 8 * j + cq;
+        if (col >= p.N) break;
+        float a0 = __uint_as_float(r[4 * j]), a1 = __uint_as_float(r[4 * j + 1]);
+        float b0 = __uint_as_float(r[4 * j + 2]), b1 = __uint_as_float(r[4 * j + 3]);
+        if (p.bias) {
+            const float2 bb = __ldg(reinterpret_cast<const float2*>(p.bias + col));
+            a0 += bb.x; a1 += bb.y; b0 += bb.x; b1 += bb.y;
         }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = 32 * C + 8 * c + 2 * j;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-                w[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            ptx::st_shared_v4(row + ((c ^ sw) << 4), w[0], w[1], w[2], w[3]);
+        if (p.epi == OSM_EPI_F32) {
+            if (ra < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + ra * p.N + col) = make_float2(a0, a1);
+            if (rb < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + rb * p.N + col) = make_float2(b0, b1);
+        } else {
+            const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1), hb = __floats2bfloat162_rn(b0, b1);
+            if (ra < p.M) *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(p.Y) + ra * p.N + col) = ha;
+            if (rb < p.M) *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(p.Y) + rb * p.N + col) = hb;
         }
     }
 }
-
-// Stage chunk C and hand it to the tensor store; `seq` counts this warp's
-// chunks so the two staging buffers alternate.
-template <int C, bool BF16>
-__device__ __forceinline__ void emit_chunk(const GemmParams& p, Smem& S, int ew, int lane, const uint32_t (&r)[128],
-                                           int32_t x, int32_t y, uint32_t& seq) {
-    const uint32_t buf = ptx::smem_u32(S.epi[ew][seq & 1]);
-    if (lane == 0) ptx::bulk_wait_group_read<1>();  // the store that last read this buffer is done with it
-    __syncwarp();
-    stage_chunk<C, BF16>(buf, lane, r);
-    ptx::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-        ptx::tma_store_2d(&p.tm_y, x, y, buf);
-        ptx::bulk_commit_group();
-    }
-    ++seq;
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     dual_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -225,7 +222,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             ptx::prefetch_tmap(&p.tm_sb);
         }
         if (p.n_hp) { ptx::prefetch_tmap(&p.tm_ah); ptx::prefetch_tmap(&p.tm_bh); }
-        ptx::prefetch_tmap(&p.tm_y);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(ptx::smem_u32(&S.tmem_base), TMEM_COLS);
@@ -268,10 +264,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, brow, fb);
                         for (int a = 0; a < natoms; ++a) {
                             ptx::tma_load_2d_pair(ptx::smem_u32(S.sfa[stage]) + 512 * a, &p.tm_sa, 0,
-                                                  (sfa_tile * p.katoms + 2 * ks + a) * 32, fb);
+                                                  (sfa_tile * p.katoms + 2 * ks + a) * 4, fb);
                             for (int h = 0; h < nbt; ++h)
                                 ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + 1024 * h + 512 * a, &p.tm_sb, 0,
-                                                      ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 32, fb);
+                                                      ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 4, fb);
                         }
                     } else {
                         const int kh = ks - p.n_fp4;
@@ -360,9 +356,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;           // TMEM lanes 32q..32q+31 are reachable from this warp
         const int half = (warp - 2) >> 2;  // columns [128*half, 128*half + 128) of the tile
-        const int ew = warp - 2;          // staging buffers of this warp
         const uint32_t acc_empty_leader = ptx::mapa(ptx::smem_u32(&S.acc_empty), 0);
-        uint32_t acc_phase = 0, seq = 0;
+        uint32_t acc_phase = 0;
         for (int tile = pair; tile < tiles; tile += npairs) {
             int m_blk, n_blk;
             tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
@@ -377,41 +372,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_fence_after();
             uint32_t r[128];
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + half * 128;
-            ptx::tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            ptx::tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-            ptx::tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-            ptx::tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+            tmem_ld_16x256b_x16(taddr, r);
+            tmem_ld_16x256b_x16(taddr + (16u << 16), r + 64);
             ptx::tmem_ld_wait();
-            // the accumulator is in registers: hand tensor memory back to the leader's MMA issuer
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
             acc_phase ^= 1u;
-            if (p.bias) {
-                const int64_t col0 = (int64_t)n_blk * BN + half * 128;
-#pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    r[i] = __float_as_uint(__uint_as_float(r[i]) + (col0 + i < p.N ? __ldg(p.bias + col0 + i) : 0.0f));
-            }
-            const int32_t y0 = m_blk * 2 * BM + static_cast<int>(rank) * BM + q * 32;
-            const int32_t x0 = n_blk * BN + half * 128;
-            if (p.epi == OSM_EPI_F32) {
-                emit_chunk<0, false>(p, S, ew, lane, r, x0, y0, seq);
-                emit_chunk<1, false>(p, S, ew, lane, r, x0 + 16, y0, seq);
-                emit_chunk<2, false>(p, S, ew, lane, r, x0 + 32, y0, seq);
-                emit_chunk<3, false>(p, S, ew, lane, r, x0 + 48, y0, seq);
-                emit_chunk<4, false>(p, S, ew, lane, r, x0 + 64, y0, seq);
-                emit_chunk<5, false>(p, S, ew, lane, r, x0 + 80, y0, seq);
-                emit_chunk<6, false>(p, S, ew, lane, r, x0 + 96, y0, seq);
-                emit_chunk<7, false>(p, S, ew, lane, r, x0 + 112, y0, seq);
-            } else {
-                emit_chunk<0, true>(p, S, ew, lane, r, x0, y0, seq);
-                emit_chunk<1, true>(p, S, ew, lane, r, x0 + 32, y0, seq);
-                emit_chunk<2, true>(p, S, ew, lane, r, x0 + 64, y0, seq);
-                emit_chunk<3, true>(p, S, ew, lane, r, x0 + 96, y0, seq);
+            const int64_t y0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + q * 32;
+            const int64_t x0 = (int64_t)n_blk * BN + half * 128;
+            if (x0 < p.N) {
+                store_slab(p, y0, x0, lane, r);
+                store_slab(p, y0 + 16, x0, lane, r + 64);
             }
         }
-        if (lane == 0) ptx::bulk_wait_group_all();  // every tensor store of this warp has completed
     }
 
     __syncwarp();  // lanes that skipped a single-thread role wait here for their elected lane
@@ -478,12 +452,14 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
         if ((rc = make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, pl->Kbp / 2, pl->N, pl->Kbp / 2, 128,
                            BN / 2, SW, "w_codes")))
             return rc;
-        const uint64_t sa_rows = static_cast<uint64_t>(scales_bytes(M, pl->Kbp)) / 16;
-        const uint64_t sb_rows = static_cast<uint64_t>(scales_bytes(pl->N, pl->Kbp)) / 16;
-        if ((rc = make_map(&p.tm_sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 16, sa_rows, 16, 16, 32, NOSW,
+        // scale atoms are contiguous 512-byte runs: view them as 128-byte rows so
+        // that one atom is four wide TMA requests rather than 32 narrow ones
+        const uint64_t sa_rows = static_cast<uint64_t>(scales_bytes(M, pl->Kbp)) / 128;
+        const uint64_t sb_rows = static_cast<uint64_t>(scales_bytes(pl->N, pl->Kbp)) / 128;
+        if ((rc = make_map(&p.tm_sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 128, sa_rows, 128, 128, 4, NOSW,
                            "a_scales")))
             return rc;
-        if ((rc = make_map(&p.tm_sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 16, sb_rows, 16, 16, 32, NOSW,
+        if ((rc = make_map(&p.tm_sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 128, sb_rows, 128, 128, 4, NOSW,
                            "w_scales")))
             return rc;
     }
@@ -493,15 +469,6 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
             return rc;
         if ((rc = make_map(&p.tm_bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_hp, pl->kp, pl->N, pl->kp * 2, 64, BN / 2,
                            SW, "w_hp")))
-            return rc;
-    }
-    if (epi == OSM_EPI_F32) {
-        if ((rc = make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, pl->N, M, pl->N * 4, 16, 32,
-                           CU_TENSOR_MAP_SWIZZLE_64B, "Y")))
-            return rc;
-    } else {
-        if ((rc = make_map(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, pl->N, M, pl->N * 2, 32, 32,
-                           CU_TENSOR_MAP_SWIZZLE_64B, "Y")))
             return rc;
     }
     p.bias = bias;
