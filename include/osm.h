@@ -86,11 +86,18 @@ typedef enum {
     OSM_WSCALE_STRIP128x1 = 2
 } osm_wscale_mode;
 
-/* Epilogues of osm_dual_gemm. */
+/* Epilogues of osm_dual_gemm. GELU below is the tanh form in FP32,
+ * 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated exactly as
+ * this library specifies it, with only IEEE round-to-nearest-even adds,
+ * multiplies and fused multiply-adds: 0.5 (1 + tanh(u)) = sigma(2u) is
+ * 1/(1 + E) for x >= 0 and E/(1 + E) for x < 0, E = exp(-2|u|) (Cody-Waite
+ * reduction, degree-7 Taylor polynomial, 0 below exp(-86)), the reciprocal
+ * by a linear seed and three Newton steps. */
 typedef enum {
-    OSM_EPI_F32 = 0,          /* Y [M][N] float32                                  */
-    OSM_EPI_BF16 = 1,         /* Y [M][N] BF16 (RNE of the FP32 accumulator)       */
-    OSM_EPI_GELU_REQUANT = 2  /* GELU(tanh) -> x/s_next -> split + MXFP4 for `next`  */
+    OSM_EPI_F32 = 0,          /* Y [M][N] float32                                     */
+    OSM_EPI_BF16 = 1,         /* Y [M][N] BF16 (RNE of the FP32 accumulator)          */
+    OSM_EPI_GELU_REQUANT = 2, /* FFN hidden layer handed to `next` already quantised  */
+    OSM_EPI_GELU_BF16 = 3     /* Y [M][N] BF16 = bf16(GELU(acc (+ bias)))             */
 } osm_epi;
 
 /* ---- calibration (offline) ------------------------------------------
@@ -150,6 +157,12 @@ OSM_API int osm_plan_status(const osm_plan* plan, void* stream, uint32_t* status
  * returns early; the context stays usable. */
 OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
 
+/* Channel order in which a previous layer must produce this plan's input
+ * for OSM_EPI_GELU_REQUANT: order_host[c] = J[c] for c < Kb (bulk channels
+ * ascending), O[c - Kb] for Kb <= c < K (outlier channels ascending).
+ * order_host: host int32[K]. */
+OSM_API int osm_plan_channel_order(const osm_plan* plan, int32_t* order_host);
+
 /* ---- offline weight packing --------------------------------------------
  * "SmoothQuant scales are folded into master weights before HiF4 packing"
  * and "remaining weights are packed with block-wise scales" (packing and
@@ -159,6 +172,17 @@ OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
  * with the plan's block-scale mode. */
 OSM_API int osm_pack_weights(const osm_plan* plan, const uint16_t* W, uint8_t* w_codes, uint8_t* w_scales,
                      uint16_t* w_hp, void* stream);
+
+/* As osm_pack_weights, for the first projection of an FFN whose output
+ * feeds `next` through OSM_EPI_GELU_REQUANT: packed row c (output channel)
+ * is column osm_plan_channel_order(next)[c] of W, so the layer's output
+ * columns come out in next's [J | O] order and every 32 consecutive bulk
+ * columns form one MXFP4 block of next's input (paper: GELU and smoothing
+ * act per channel, so the permutation changes no value). Requires
+ * plan->N == next->K. With OSM_WSCALE_TILE32x32 the 32-row tiles are taken
+ * in the permuted order. */
+OSM_API int osm_pack_weights_for_next(const osm_plan* plan, const osm_plan* next, const uint16_t* W,
+                                      uint8_t* w_codes, uint8_t* w_scales, uint16_t* w_hp, void* stream);
 
 /* ---- runtime activation path ----------------------------------------------
  * "activations are divided in-place by s, quantized ..., and routed through
@@ -182,10 +206,19 @@ OSM_API int osm_quantize_act(const osm_plan* plan, const uint16_t* X, int64_t M,
  * (block-scaled MXFP4 MMA, then BF16 MMA) before a single epilogue.
  * Operands come from osm_quantize_act / osm_pack_weights with the same
  * plan. M >= 1.
- *   epi = OSM_EPI_F32:  Y is float [M][N].
- *   epi = OSM_EPI_BF16: Y is BF16  [M][N].
- *   epi = OSM_EPI_GELU_REQUANT: not available in this build (returns
- *         OSM_ERR_UNSUPPORTED); `next`, next_* must be NULL otherwise.
+ *   epi = OSM_EPI_F32:       Y is float [M][N].
+ *   epi = OSM_EPI_BF16:      Y is BF16  [M][N].
+ *   epi = OSM_EPI_GELU_BF16: Y is BF16  [M][N] = bf16(GELU(acc + bias)).
+ *   epi = OSM_EPI_GELU_REQUANT (the FFN up-projection fused with the next
+ *         layer's activation path; implementation paragraph: activations
+ *         are divided by s, quantised and routed): Y and bias must be NULL;
+ *         the weights must come from osm_pack_weights_for_next(plan, next);
+ *         for each row, h = bf16(GELU(acc)) is written straight into the
+ *         next layer's packed activations, exactly as osm_quantize_act(next)
+ *         would write them for the BF16 matrix H = h in next's natural
+ *         channel order: next_codes [M][Kbp'/2], next_scales (rows padded to
+ *         128, padding rows 0), next_hp [M][kp'] (primes: next's sizes).
+ *   `next` and next_* must be NULL for the other epilogues.
  * A pipeline wait that exceeds the plan's wait limit sets the plan's
  * OSM_STATUS_TIMEOUT bit (see osm_plan_status). */
 OSM_API int osm_dual_gemm(const osm_plan* plan, const uint8_t* a_codes, const uint8_t* a_scales,

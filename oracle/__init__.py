@@ -81,6 +81,9 @@ def _load():
             lib.oracle_gelu_tanh_f32.argtypes = [ctypes.c_float]
             lib.oracle_gelu_exp_neg.restype = ctypes.c_float
             lib.oracle_gelu_exp_neg.argtypes = [ctypes.c_float]
+            lib.oracle_gelu_recip.restype = ctypes.c_float
+            lib.oracle_gelu_recip.argtypes = [ctypes.c_float]
+            lib.oracle_gelu_bf16_rows.argtypes = [P, I64, P]
             _lib = lib
     return _lib
 
@@ -136,6 +139,10 @@ def gelu_tanh_f32(x: float) -> float:
 
 def gelu_exp_neg(x: float) -> float:
     return float(_load().oracle_gelu_exp_neg(float(np.float32(x))))
+
+
+def gelu_recip(d: float) -> float:
+    return float(_load().oracle_gelu_recip(float(np.float32(d))))
 
 
 # ---- arrays --------------------------------------------------------------
@@ -229,6 +236,14 @@ def pack_weights(W: np.ndarray, s: np.ndarray, O: np.ndarray, mode: int):
     Op = O if k else np.zeros(1, np.int32)
     _load().oracle_pack_weights(_p(W), K, N, k, _p(s), _p(Op), int(mode), _p(codes), _p(scales), _p(w_hp))
     return codes, scales, w_hp
+
+
+def gelu_bf16(y: np.ndarray) -> np.ndarray:
+    """h = bf16(GELU_tanh(fp32(y))) element-wise for FP64 accumulators y."""
+    y = _c(y, np.float64)
+    out = np.empty(y.shape, np.uint16)
+    _load().oracle_gelu_bf16_rows(_p(y), y.size, _p(out))
+    return out
 
 
 def dual_gemm_rows(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, bias=None):

@@ -467,46 +467,82 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
 /* ------------------------------------------------------------------ */
 
 /*
- * exp(x) for the GELU's tanh, in FP32 with explicit operations:
- * Cody-Waite reduction x = n*ln2 + r, |r| <= ln2/2, with ln2 split into a
- * high part exact in 12 bits and a low remainder; exp(r) by its Taylor
- * series to degree 7 evaluated by Horner's rule with fused multiply-adds
- * (fmaf, one rounding each); the result scaled by 2^n with ldexpf.
- * Arguments are clamped to [-88, 0] because the GELU only needs
- * exp(-2|u|) in (0, 1].
+ * exp(a) for a <= 0 in FP32, taken as exactly 0 below -86 (where exp(a) <
+ * 2^-124); on [-86, 0] with explicit operations: Cody-Waite
+ * reduction a = n*ln2 + r (|r| <= ln2/2) with ln2 split into a 12-bit high
+ * part and a low remainder; exp(r) by its Taylor series to degree 7 in
+ * Horner form with fused multiply-adds (fmaf, one rounding each); the
+ * result scaled by 2^n. n is a*log2(e) rounded to the nearest integer (ties
+ * to even) in one fused step: t = fmaf(a, LOG2E, 1.5*2^23) lies in
+ * [2^23, 2^24), where the FP32 spacing is 1, and n = t - 1.5*2^23 exactly.
+ * On that range 2^n (and the result) stay normal, so the scaling is exact.
+ * Constants are the binary32 values of log2(e), ln2 split, and 1/k!.
  */
-float oracle_gelu_exp_neg(float x)
+float oracle_gelu_exp_neg(float a)
 {
-    if (x < -88.0f) x = -88.0f;
-    if (x > 0.0f) x = 0.0f;
-    const float LOG2E = 1.44269504088896341f;
-    const float LN2_HI = 0.693145751953125f;       /* 12 significant bits */
-    const float LN2_LO = 1.42860682030941723e-06f; /* ln2 - LN2_HI */
-    float n = rintf(x * LOG2E);
-    float r = fmaf(-n, LN2_HI, x);
+    if (a < -86.0f) return 0.0f;
+    if (a > 0.0f) a = 0.0f;
+    const float LOG2E = 0x1.715476p+0f;
+    const float LN2_HI = 0x1.62e4p-1f;      /* 12 significant bits */
+    const float LN2_LO = 0x1.7f7d1cp-20f;   /* ln2 - LN2_HI */
+    const float SHIFT = 0x1.8p+23f;         /* 1.5 * 2^23 */
+    float t = fmaf(a, LOG2E, SHIFT);
+    float n = t - SHIFT;
+    float r = fmaf(-n, LN2_HI, a);
     r = fmaf(-n, LN2_LO, r);
-    /* Taylor coefficients 1/k!, k = 7..0 */
-    float p = 1.0f / 5040.0f;
-    p = fmaf(p, r, 1.0f / 720.0f);
-    p = fmaf(p, r, 1.0f / 120.0f);
-    p = fmaf(p, r, 1.0f / 24.0f);
-    p = fmaf(p, r, 1.0f / 6.0f);
+    float p = 0x1.a01a02p-13f;              /* 1/7! */
+    p = fmaf(p, r, 0x1.6c16c2p-10f);        /* 1/6! */
+    p = fmaf(p, r, 0x1.111112p-7f);         /* 1/5! */
+    p = fmaf(p, r, 0x1.555556p-5f);         /* 1/4! */
+    p = fmaf(p, r, 0x1.555556p-3f);         /* 1/3! */
     p = fmaf(p, r, 0.5f);
     p = fmaf(p, r, 1.0f);
     p = fmaf(p, r, 1.0f);
     return ldexpf(p, (int)n);
 }
 
-/* GELU_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), with
- * tanh(u) = sign(u) (1 - E)/(1 + E), E = exp(-2|u|), all in FP32. */
+/*
+ * 1/d for d in [1, 2] by Newton's iteration for the reciprocal: the linear
+ * seed y0 = 24/17 - (8/17) d (relative error at most 1/17 on [1, 2]), then
+ * three steps y <- y + y (1 - d y), each as e = fmaf(-d, y, 1),
+ * y = fmaf(y, e, y). The error squares at each step: 1/17 -> 2^-8.2 ->
+ * 2^-16.3 -> below FP32 rounding.
+ */
+float oracle_gelu_recip(float d)
+{
+    float y = fmaf(-0x1.e1e1e2p-2f, d, 0x1.69696ap+0f);   /* 24/17 - (8/17) d */
+    for (int i = 0; i < 3; ++i) {
+        float e = fmaf(-d, y, 1.0f);
+        y = fmaf(y, e, y);
+    }
+    return y;
+}
+
+/*
+ * GELU in its tanh form, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi)(x + 0.044715
+ * x^3), for finite x, evaluated through the identity 0.5 (1 + tanh(u)) =
+ * sigma(2u) = 1 / (1 + exp(-2u)): with E = exp(-2|u|),
+ *   sigma(2u) = 1 / (1 + E)  for u >= 0,   E / (1 + E)  for u < 0,
+ * and u has the sign of x. Every operation in FP32 in the order written:
+ * x2 = x*x; k = fmaf(C1, x2, 1); u = (C0*x)*k; E = exp(-2|u|) as above;
+ * y = recip(1 + E); result (x * (x < 0 ? E : 1)) * y.
+ */
 float oracle_gelu_tanh_f32(float x)
 {
-    const float C0 = 0.7978845608028654f;   /* sqrt(2/pi) */
-    const float C1 = 0.044715f;
-    float x3 = x * x * x;
-    float u = C0 * (x + C1 * x3);
+    const float C0 = 0x1.988454p-1f;   /* sqrt(2/pi) */
+    const float C1 = 0x1.6e4e26p-5f;   /* 0.044715 */
+    float x2 = x * x;
+    float k = fmaf(C1, x2, 1.0f);
+    float u = (C0 * x) * k;
     float E = oracle_gelu_exp_neg(-2.0f * fabsf(u));
-    float th = (1.0f - E) / (1.0f + E);
-    if (u < 0.0f) th = -th;
-    return 0.5f * x * (1.0f + th);
+    float y = oracle_gelu_recip(1.0f + E);
+    float s = x < 0.0f ? E : 1.0f;
+    return (x * s) * y;
+}
+
+/* FFN hidden activations from FP64 accumulators: h = bf16(GELU(fp32(y))),
+ * y [n] FP64 -> h [n] BF16 words. */
+void oracle_gelu_bf16_rows(const double* y, int64_t n, uint16_t* h)
+{
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_f32_to_bf16(oracle_gelu_tanh_f32((float)y[i]));
 }

@@ -26,7 +26,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
 STATUS_TIMEOUT = 1
 WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
-EPI_F32, EPI_BF16, EPI_GELU_REQUANT = 0, 1, 2
+EPI_F32, EPI_BF16, EPI_GELU_REQUANT, EPI_GELU_BF16 = 0, 1, 2, 3
 
 # Every entry point declared in include/osm.h, with its ctypes signature.
 _P, _I64, _I, _U64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
@@ -41,6 +41,8 @@ _SIGNATURES = {
     "osm_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _I]),
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
     "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
+    "osm_pack_weights_for_next": (_I, [_P, _P, _P, _P, _P, _P, _P]),
+    "osm_plan_channel_order": (_I, [_P, _P]),
     "osm_quantize_act": (_I, [_P, _P, _I64, _P, _P, _P, _P]),
     "osm_dual_gemm": (_I, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     "osm_linear_workspace_size": (_SZ, [_P, _I64, _I]),
@@ -163,6 +165,12 @@ class Plan:
         _check(lib().osm_plan_status(self._h, _stream(stream), ctypes.byref(v), int(clear)))
         return int(v.value)
 
+    def channel_order(self) -> np.ndarray:
+        """[J ascending | O ascending] (osm_plan_channel_order)."""
+        out = np.empty(self.K, np.int32)
+        _check(lib().osm_plan_channel_order(self._h, _host_ptr(out)))
+        return out
+
     def set_wait_limit(self, ns: int):
         _check(lib().osm_plan_set_wait_limit(self._h, int(ns)))
 
@@ -231,6 +239,18 @@ def pack_weights(plan: Plan, W, w_codes, w_scales, w_hp, stream=None):
                                   _ptr(w_hp, "w_hp", _bf16_types(), hb, allow_none=hb == 0), _stream(stream)))
 
 
+def pack_weights_for_next(plan: Plan, next_plan: Plan, W, w_codes, w_scales, w_hp, stream=None):
+    """Pack W with its output columns in next_plan's channel order
+    (osm_pack_weights_for_next), for OSM_EPI_GELU_REQUANT."""
+    cb, sb, hb = plan.sizes(plan.N)
+    if tuple(W.shape) != (plan.K, plan.N):
+        raise ValueError("W must have shape (K, N)")
+    _check(lib().osm_pack_weights_for_next(plan.handle, next_plan.handle, _ptr(W, "W", _bf16_types()),
+                                           _ptr(w_codes, "w_codes", _u8_types(), cb, allow_none=cb == 0),
+                                           _ptr(w_scales, "w_scales", _u8_types(), sb, allow_none=sb == 0),
+                                           _ptr(w_hp, "w_hp", _bf16_types(), hb, allow_none=hb == 0), _stream(stream)))
+
+
 def quantize_act(plan: Plan, X, a_codes, a_scales, a_hp, stream=None):
     """Smooth, split and MXFP4-encode activations (osm_quantize_act). X: [M][K] BF16."""
     M, K = X.shape
@@ -244,11 +264,30 @@ def quantize_act(plan: Plan, X, a_codes, a_scales, a_hp, stream=None):
 
 
 def dual_gemm(plan: Plan, a_codes, a_scales, a_hp, M: int, w_codes, w_scales, w_hp, Y, bias=None,
-              epi: int = EPI_F32, stream=None):
-    """Eq. (5) on packed operands (osm_dual_gemm). Y: [M][N] float32 or BF16."""
+              epi: int = EPI_F32, stream=None, next_plan: Plan | None = None, next_buffers=None):
+    """Eq. (5) on packed operands (osm_dual_gemm). Y: [M][N] float32 or BF16.
+    With epi=EPI_GELU_REQUANT, Y and bias are None and next_buffers are the
+    (codes, scales, hp) of next_plan for M rows."""
     import torch
     cbm, sbm, hbm = plan.sizes(M)
     cbn, sbn, hbn = plan.sizes(plan.N)
+    if epi == EPI_GELU_REQUANT:
+        if next_plan is None or next_buffers is None or Y is not None or bias is not None:
+            raise ValueError("GELU_REQUANT needs next_plan and next_buffers, and no Y or bias")
+        ncb, nsb, nhb = next_plan.sizes(M)
+        nc, ns, nh = next_buffers
+        _check(lib().osm_dual_gemm(plan.handle,
+                                   _ptr(a_codes, "a_codes", _u8_types(), cbm, allow_none=cbm == 0),
+                                   _ptr(a_scales, "a_scales", _u8_types(), sbm, allow_none=sbm == 0),
+                                   _ptr(a_hp, "a_hp", _bf16_types(), hbm, allow_none=hbm == 0), M,
+                                   _ptr(w_codes, "w_codes", _u8_types(), cbn, allow_none=cbn == 0),
+                                   _ptr(w_scales, "w_scales", _u8_types(), sbn, allow_none=sbn == 0),
+                                   _ptr(w_hp, "w_hp", _bf16_types(), hbn, allow_none=hbn == 0),
+                                   None, int(epi), None, next_plan.handle,
+                                   _ptr(nc, "next_codes", _u8_types(), ncb, allow_none=ncb == 0),
+                                   _ptr(ns, "next_scales", _u8_types(), nsb, allow_none=nsb == 0),
+                                   _ptr(nh, "next_hp", _bf16_types(), nhb, allow_none=nhb == 0), _stream(stream)))
+        return
     ybytes = M * plan.N * (4 if epi == EPI_F32 else 2)
     ytypes = (torch.float32,) if epi == EPI_F32 else _bf16_types()
     _check(lib().osm_dual_gemm(plan.handle,

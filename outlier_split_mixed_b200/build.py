@@ -16,7 +16,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libosm.so")
 
 SOURCES = ["osm_api.cu", "osm_quant.cu", "osm_gemm.cu", "osm_noalloc.cu"]
-HEADERS = ["osm_internal.h", "osm_ptx.cuh"]
+HEADERS = ["osm_internal.h", "osm_ptx.cuh", "osm_mx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",

@@ -167,7 +167,7 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
 
     std::vector<float> inv_s(static_cast<size_t>(K));
     for (int64_t j = 0; j < K; ++j) inv_s[j] = 1.0f / s_host[j];
-    std::vector<int32_t> route(static_cast<size_t>(K)), J;
+    std::vector<int32_t> route(static_cast<size_t>(K)), J, order;
     J.reserve(static_cast<size_t>(K - k));
     {
         std::vector<int32_t> slot(static_cast<size_t>(K), -1);
@@ -182,6 +182,10 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
             }
         }
     }
+    order = J;
+    order.insert(order.end(), O_host, O_host + k);
+    std::vector<float> inv_s_ord(static_cast<size_t>(K));
+    for (int64_t c = 0; c < K; ++c) inv_s_ord[c] = inv_s[order[c]];
     auto cleanup = [&](int code) {
         osm_plan_destroy(p);
         return code;
@@ -193,6 +197,8 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
     if (e == cudaSuccess && K - k > 0) e = cudaMalloc(&p->d_J, sizeof(int32_t) * (K - k));
     if (e == cudaSuccess && k > 0) e = cudaMalloc(&p->d_O, sizeof(int32_t) * k);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_status, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * K);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_inv_s_ord, sizeof(float) * K);
     if (e != cudaSuccess) return cleanup(fail(OSM_ERR_NOMEM, "plan_create: %s", cudaGetErrorString(e)));
     e = cudaMemcpy(p->d_s, s_host, sizeof(float) * K, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_inv_s, inv_s.data(), sizeof(float) * K, cudaMemcpyHostToDevice);
@@ -201,6 +207,9 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
         e = cudaMemcpy(p->d_J, J.data(), sizeof(int32_t) * (K - k), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && k > 0) e = cudaMemcpy(p->d_O, O_host, sizeof(int32_t) * k, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemcpy(p->d_order, order.data(), sizeof(int32_t) * K, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(p->d_inv_s_ord, inv_s_ord.data(), sizeof(float) * K, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cleanup(fail(OSM_ERR_CUDA, "plan_create: %s", cudaGetErrorString(e)));
     *out = p;
     return OSM_OK;
@@ -214,6 +223,8 @@ int osm_plan_destroy(osm_plan* p) {
     cudaFree(p->d_J);
     cudaFree(p->d_O);
     cudaFree(p->d_status);
+    cudaFree(p->d_order);
+    cudaFree(p->d_inv_s_ord);
     delete p;
     return OSM_OK;
 }
@@ -269,7 +280,30 @@ int osm_pack_weights(const osm_plan* p, const uint16_t* W, uint8_t* w_codes, uin
                 "pack_weights: w_codes / w_scales null or misaligned");
     OSM_REQUIRE(p->kp == 0 || (w_hp && aligned16(w_hp)), "pack_weights: w_hp null or misaligned");
     OSM_TRY(check_device());
-    return launch_pack_weights(p, W, w_codes, w_scales, w_hp, static_cast<cudaStream_t>(stream));
+    return launch_pack_weights(p, W, nullptr, w_codes, w_scales, w_hp, static_cast<cudaStream_t>(stream));
+}
+
+int osm_pack_weights_for_next(const osm_plan* p, const osm_plan* next, const uint16_t* W, uint8_t* w_codes,
+                              uint8_t* w_scales, uint16_t* w_hp, void* stream) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(p));
+    OSM_TRY(check_plan(next));
+    OSM_REQUIRE(next->K == p->N, "pack_weights_for_next: next->K (%lld) must equal plan->N (%lld)",
+                (long long)next->K, (long long)p->N);
+    OSM_REQUIRE(W && aligned16(W), "pack_weights_for_next: W must be a 16-byte aligned device pointer");
+    OSM_REQUIRE(p->Kbp == 0 || (w_codes && aligned16(w_codes) && w_scales && aligned16(w_scales)),
+                "pack_weights_for_next: w_codes / w_scales null or misaligned");
+    OSM_REQUIRE(p->kp == 0 || (w_hp && aligned16(w_hp)), "pack_weights_for_next: w_hp null or misaligned");
+    OSM_TRY(check_device());
+    return launch_pack_weights(p, W, next->d_order, w_codes, w_scales, w_hp, static_cast<cudaStream_t>(stream));
+}
+
+int osm_plan_channel_order(const osm_plan* p, int32_t* order_host) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(p));
+    OSM_REQUIRE(order_host, "plan_channel_order: order_host is NULL");
+    return check_cuda(cudaMemcpy(order_host, p->d_order, sizeof(int32_t) * p->K, cudaMemcpyDeviceToHost),
+                      "plan_channel_order: read");
 }
 
 int osm_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* a_codes, uint8_t* a_scales,
@@ -291,20 +325,30 @@ int osm_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_sc
     g_err[0] = 0;
     OSM_TRY(check_plan(p));
     OSM_REQUIRE(M >= 1 && M <= (int64_t(1) << 31) - 1, "dual_gemm: need 1 <= M < 2^31");
-    if (epi == OSM_EPI_GELU_REQUANT)
-        return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: the fused GELU/requantize epilogue is not built");
-    OSM_REQUIRE(epi == OSM_EPI_F32 || epi == OSM_EPI_BF16, "dual_gemm: unknown epilogue %d", epi);
-    OSM_REQUIRE(!next && !next_codes && !next_scales && !next_hp, "dual_gemm: next-layer buffers need GELU_REQUANT");
-    OSM_REQUIRE(Y && aligned16(Y), "dual_gemm: Y must be a 16-byte aligned device pointer");
-    OSM_REQUIRE(!bias || aligned16(bias), "dual_gemm: bias must be 16-byte aligned");
+    OSM_REQUIRE(epi == OSM_EPI_F32 || epi == OSM_EPI_BF16 || epi == OSM_EPI_GELU_BF16 || epi == OSM_EPI_GELU_REQUANT,
+                "dual_gemm: unknown epilogue %d", epi);
+    if (epi == OSM_EPI_GELU_REQUANT) {
+        OSM_TRY(check_plan(next));
+        OSM_REQUIRE(next->K == p->N, "dual_gemm: next->K (%lld) must equal plan->N (%lld)", (long long)next->K,
+                    (long long)p->N);
+        OSM_REQUIRE(!Y && !bias, "dual_gemm: GELU_REQUANT writes next_* only; Y and bias must be NULL");
+        OSM_REQUIRE(next->Kbp == 0 || (next_codes && aligned16(next_codes) && next_scales && aligned16(next_scales)),
+                    "dual_gemm: next_codes / next_scales null or misaligned");
+        OSM_REQUIRE(next->kp == 0 || (next_hp && aligned16(next_hp)), "dual_gemm: next_hp null or misaligned");
+    } else {
+        OSM_REQUIRE(!next && !next_codes && !next_scales && !next_hp,
+                    "dual_gemm: next-layer buffers need OSM_EPI_GELU_REQUANT");
+        OSM_REQUIRE(Y && aligned16(Y), "dual_gemm: Y must be a 16-byte aligned device pointer");
+        OSM_REQUIRE(!bias || aligned16(bias), "dual_gemm: bias must be 16-byte aligned");
+    }
     OSM_REQUIRE(p->Kbp == 0 || (a_codes && aligned16(a_codes) && a_scales && aligned16(a_scales) && w_codes &&
                                 aligned16(w_codes) && w_scales && aligned16(w_scales)),
                 "dual_gemm: bulk operands null or misaligned");
     OSM_REQUIRE(p->kp == 0 || (a_hp && aligned16(a_hp) && w_hp && aligned16(w_hp)),
                 "dual_gemm: outlier operands null or misaligned");
     OSM_TRY(check_device());
-    return launch_dual_gemm(p, a_codes, a_scales, a_hp, M, w_codes, w_scales, w_hp, bias, epi, Y,
-                            static_cast<cudaStream_t>(stream));
+    return launch_dual_gemm(p, a_codes, a_scales, a_hp, M, w_codes, w_scales, w_hp, bias, epi, Y, next, next_codes,
+                            next_scales, next_hp, static_cast<cudaStream_t>(stream));
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

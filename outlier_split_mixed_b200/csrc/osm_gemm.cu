@@ -46,6 +46,7 @@
 #include <mutex>
 
 #include "osm_internal.h"
+#include "osm_mx.cuh"
 #include "osm_ptx.cuh"
 
 namespace osm {
@@ -59,7 +60,26 @@ constexpr int B_TILE = (BN / 2) * 128;  // one K-step of this CTA's half of B
 constexpr int SFA_TILE = 2 * 512;       // two 128x4 scale atoms (K = 256)
 constexpr int SFB_TILE = 2 * 2 * 512;   // two 128-row tiles x two atoms (all 256 B rows)
 constexpr int NUM_EPI_WARPS = 8;        // two per TMEM lane quadrant, 128 columns each
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int CTRL_WG = 2;              // warpgroup of the producer (warp 8) and MMA issuer (warp 9)
+constexpr int PRODUCER_WARP = 4 * CTRL_WG;
+constexpr int MMA_WARP = PRODUCER_WARP + 1;
+constexpr int NUM_THREADS = 32 * NUM_EPI_WARPS + 128;  // epilogue = warpgroups 0 and 1
+// Register split. The kernel is launched with LAUNCH_REGS per thread (the
+// most 384 threads may hold: a warp's registers come from one SM
+// sub-partition of 16384, and each sub-partition holds three warps).
+// Warpgroup 2 (producer, MMA issuer, two idle warps) then gives registers
+// back and the epilogue warpgroups take them: a lane's 128 accumulators,
+// 64 packed x' words and the loop state must fit in EPI_REGS.
+constexpr int LAUNCH_REGS = 168;
+constexpr int CTRL_REGS = 56;
+constexpr int EPI_REGS = 224;
+static_assert(NUM_THREADS == 384, "three warpgroups");
+static_assert((LAUNCH_REGS - CTRL_REGS) * 128 >= (EPI_REGS - LAUNCH_REGS) * 256, "register split exceeds the launch");
+static_assert(CTRL_REGS + 2 * EPI_REGS <= 512, "register split exceeds a sub-partition");
+static_assert(LAUNCH_REGS * 3 <= 512 && CTRL_REGS % 8 == 0 && EPI_REGS % 8 == 0, "register counts");
+// Each epilogue kind is its own kernel instantiation with its own register
+// allocation; only the FFN requantisation needs more than LAUNCH_REGS.
+__host__ __device__ constexpr bool uses_register_split(int epi) { return epi == OSM_EPI_GELU_REQUANT; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;       // scale factors live after the accumulator
 constexpr uint32_t SF_STAGE_COLS = 24;  // 8 columns for A, 16 for B per ring slot
@@ -110,6 +130,13 @@ struct GemmParams {
     int num_m, num_n;
     int n_row_tiles; // ceil(N / 128): scale-atom rows of W
     int epi;
+    // OSM_EPI_GELU_REQUANT: the next layer's packed activations
+    uint8_t* next_codes;      // [M][nKbp/2]
+    uint8_t* next_scales;     // layout, rows padded to 128
+    uint16_t* next_hp;        // [M][nkp]
+    const float* inv_s_ord;   // next's inv_s in its [J | O] channel order (= this layer's column order)
+    int nKb, nKbp, nk, nkp;   // next's bulk / outlier widths
+    int64_t m_pad;            // M rounded up to 128 (rows of next_scales)
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
@@ -161,6 +188,7 @@ __device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r)
 // store instruction of the warp writes eight full 32-byte sectors (one per
 // row), FP32 as 8-byte pairs or BF16 as 4-byte pairs. Rows >= M and
 // columns >= N (N % 32 == 0, so whole 8-column blocks) are skipped.
+template <int EPI>
 __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, int64_t col0, int lane, const uint32_t* r) {
     const int64_t ra = row0 + (lane >> 2), rb = ra + 8;
     const int cq = 2 * (lane & 3);
@@ -174,7 +202,11 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
             const float2 bb = __ldg(reinterpret_cast<const float2*>(p.bias + col));
             a0 += bb.x; a1 += bb.y; b0 += bb.x; b1 += bb.y;
         }
-        if (p.epi == OSM_EPI_F32) {
+        if constexpr (EPI == OSM_EPI_GELU_BF16) {
+            a0 = mx::gelu_tanh(a0); a1 = mx::gelu_tanh(a1);
+            b0 = mx::gelu_tanh(b0); b1 = mx::gelu_tanh(b1);
+        }
+        if constexpr (EPI == OSM_EPI_F32) {
             if (ra < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + ra * p.N + col) = make_float2(a0, a1);
             if (rb < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + rb * p.N + col) = make_float2(b0, b1);
         } else {
@@ -184,6 +216,301 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
         }
     }
 }
+// Wait for this warp's tensor-memory loads, then tell the leader CTA's
+// MMA warp that the accumulator may be overwritten (16 arrivals: 8 warps in
+// each CTA of the pair).
+__device__ __forceinline__ void release_accumulator(uint32_t acc_empty_leader, int lane) {
+    ptx::tmem_ld_wait();
+    ptx::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
+}
+// OSM_EPI_GELU_REQUANT, step 1: the lane's 128 accumulators (one row,
+// columns c_base .. c_base+127) become x' = bf16(bf16(GELU(acc)) * inv_s) of
+// the next layer, packed as BF16 pairs (element 2i in the low half of word
+// i). Column c of this layer is channel order[c] of the next layer, whose
+// reciprocal smoothing factor is inv_s_ord[c]. Columns >= N are not read.
+__device__ __forceinline__ void requant_convert(const GemmParams& p, int64_t c_base, const uint32_t (&r)[128],
+                                                uint32_t (&hw)[64]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        if (c_base + 4 * i >= p.N) break;
+        const float4 sv = __ldg(reinterpret_cast<const float4*>(p.inv_s_ord + c_base) + i);
+        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+        uint32_t xs[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t hb = mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])));
+            xs[j] = mx::f32_to_bf16_bits(__fmul_rn(mx::bf16_bits_to_f32(hb), s4[j]));
+        }
+        hw[2 * i] = xs[0] | (xs[1] << 16);
+        hw[2 * i + 1] = xs[2] | (xs[3] << 16);
+    }
+}
+// Step 2, one 32-column group G (columns c0 = c_base + 32G ..): column
+// c < nKb is bulk position c, column c >= nKb is outlier slot c - nKb. The
+// bulk part is MXFP4-encoded as one block (codes 16 bytes, one scale byte;
+// in a partial last block the positions >= nKb are padding, code 0) and
+// the outlier part goes to next_hp. The group holding the last bulk position
+// also writes the next layer's padding blocks (code 0, scale 0), the group
+// holding the last column the outlier padding slots, and lanes of padding
+// rows (M <= row < M rounded up to 128) write scale 0.
+template <int G>
+__device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, int64_t c_base, const uint32_t (&hwall)[64]) {
+    const int64_t c0 = c_base + 32 * G;
+    if (c0 >= p.N) return;
+    const uint32_t* hw = hwall + 16 * G;
+    const int katoms = p.nKbp >> 7;
+    const bool holds_last_bulk = p.nKb > 0 && c0 <= p.nKb - 1 && p.nKb - 1 < c0 + 32;
+    if (row >= p.M) {
+        if (row < p.m_pad) {
+            if (c0 < p.nKb) p.next_scales[mx::sf_offset(row, c0 >> 5, katoms)] = 0;
+            if (holds_last_bulk)
+                for (int b = (p.nKb + 31) >> 5; b < (p.nKbp >> 5); ++b) p.next_scales[mx::sf_offset(row, b, katoms)] = 0;
+        }
+        return;
+    }
+    if (c0 < p.nKb) {
+        const int nreal = static_cast<int>(p.nKb - c0 < 32 ? p.nKb - c0 : 32);
+        uint32_t bw[16];
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = (2 * i < nreal) ? (hw[i] & 0xFFFFu) : 0u;
+            const uint32_t hi = (2 * i + 1 < nreal) ? (hw[i] & 0xFFFF0000u) : 0u;
+            bw[i] = lo | hi;
+            const uint32_t a = bw[i] & 0x7FFF7FFFu;
+            m = max(m, max(a & 0xFFFFu, a >> 16));
+        }
+        const int X = mx::exponent(mx::bf16_bits_to_f32(m));
+        const float inv = mx::exp2_neg(X);
+        const uint4 out = make_uint4(mx::encode8_words(bw[0], bw[1], bw[2], bw[3], inv),
+                                     mx::encode8_words(bw[4], bw[5], bw[6], bw[7], inv),
+                                     mx::encode8_words(bw[8], bw[9], bw[10], bw[11], inv),
+                                     mx::encode8_words(bw[12], bw[13], bw[14], bw[15], inv));
+        *reinterpret_cast<uint4*>(p.next_codes + row * (p.nKbp >> 1) + (c0 >> 1)) = out;
+        p.next_scales[mx::sf_offset(row, c0 >> 5, katoms)] = static_cast<uint8_t>(X + 127);
+        if (holds_last_bulk) {
+            for (int b = (p.nKb + 31) >> 5; b < (p.nKbp >> 5); ++b) {
+                *reinterpret_cast<uint4*>(p.next_codes + row * (p.nKbp >> 1) + b * 16) = make_uint4(0, 0, 0, 0);
+                p.next_scales[mx::sf_offset(row, b, katoms)] = 0;
+            }
+        }
+    }
+    if (c0 + 32 > p.nKb) {
+        // outlier part: columns max(c0, nKb) .. c0+31 -> slots c - nKb
+        uint16_t* hp = p.next_hp + row * p.nkp;
+        if (c0 >= p.nKb && ((c0 - p.nKb) & 7) == 0) {
+            uint4* dst = reinterpret_cast<uint4*>(hp + (c0 - p.nKb));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hw[4 * i], hw[4 * i + 1], hw[4 * i + 2], hw[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (c0 + e >= p.nKb)
+                    hp[c0 + e - p.nKb] = static_cast<uint16_t>((e & 1) ? (hw[e >> 1] >> 16) : (hw[e >> 1] & 0xFFFFu));
+        }
+        if (p.nkp > p.nk && c0 <= p.N - 1 && p.N - 1 < c0 + 32)
+            for (int i = p.nk; i < p.nkp; ++i) hp[i] = 0;
+    }
+}
+
+// TMA producer, one elected thread in each CTA of the pair.
+__device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint32_t rank, bool leader, int pair,
+                                              int npairs, int tiles, int ksteps, const volatile int* abort,
+                                              const volatile int* never, uint64_t drain_ns) {
+    if (ptx::elect_one()) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int last_stage = -1;
+        uint32_t last_phase = 0;
+        bool ok = true;
+        for (int tile = pair; tile < tiles && ok; tile += npairs) {
+            int m_blk, n_blk;
+            tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
+            const int arow = m_blk * 2 * BM + static_cast<int>(rank) * BM;        // this CTA's A rows
+            const int brow = n_blk * BN + static_cast<int>(rank) * (BN / 2);      // this CTA's B rows
+            const int nbt = min(2, p.n_row_tiles - 2 * n_blk);                   // valid B scale row tiles
+            const int sfa_tile = 2 * m_blk + static_cast<int>(rank);              // A scale row tile
+            for (int ks = 0; ks < ksteps; ++ks) {
+                if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.empty[stage]), phase ^ 1u, p.wait_limit_ns,
+                                            abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = ptx::mapa(ptx::smem_u32(&S.full[stage]), 0);  // leader's barrier
+                if (ks < p.n_fp4) {
+                    const int natoms = min(2, p.katoms - 2 * ks);
+                    if (leader)
+                        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]),
+                                                   2u * (A_TILE + B_TILE + natoms * 512u * (1u + nbt)));
+                    ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_a, ks * 128, arow, fb);
+                    ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, brow, fb);
+                    for (int a = 0; a < natoms; ++a) {
+                        ptx::tma_load_2d_pair(ptx::smem_u32(S.sfa[stage]) + 512 * a, &p.tm_sa, 0,
+                                              (sfa_tile * p.katoms + 2 * ks + a) * 4, fb);
+                        for (int h = 0; h < nbt; ++h)
+                            ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + 1024 * h + 512 * a, &p.tm_sb, 0,
+                                                  ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 4, fb);
+                    }
+                } else {
+                    const int kh = ks - p.n_fp4;
+                    if (leader)
+                        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]), 2u * (A_TILE + B_TILE));
+                    ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_ah, kh * 64, arow, fb);
+                    ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_bh, kh * 64, brow, fb);
+                }
+                last_stage = stage;
+                last_phase = phase;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (!ok) raise_abort(S, p.status);
+        // Let every copy this thread issued land before the pair exits: the
+        // last slot it filled is released (empty) only after the MMAs that
+        // read it completed, which implies all earlier copies completed too.
+        if (last_stage >= 0) {
+            if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.empty[last_stage]), last_phase, drain_ns,
+                                                never))
+                ptx::spin_ns(1000000);  // an aborted pipeline: give any in-flight copy ample time to land
+        }
+    }
+}
+
+// MMA issuer, one elected thread of the leader CTA.
+__device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool leader, int pair, int npairs, int tiles,
+                                         int ksteps, const volatile int* abort, const volatile int* never,
+                                         uint64_t drain_ns, uint32_t tmem) {
+    if (leader && ptx::elect_one()) {
+        int stage = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true;
+        const uint32_t acc = tmem;  // lane 0, column 0
+        for (int tile = pair; tile < tiles && ok; tile += npairs) {
+            if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.acc_empty), acc_phase ^ 1u, p.wait_limit_ns,
+                                                abort)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            uint32_t accumulate = 0;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.full[stage]), phase, p.wait_limit_ns, abort)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t a_base = ptx::smem_u32(S.a[stage]);
+                const uint32_t b_base = ptx::smem_u32(S.b[stage]);
+                if (ks < p.n_fp4) {
+                    const int natoms = min(2, p.katoms - 2 * ks);
+                    const uint32_t sfa_col = tmem + SF_COL0 + stage * SF_STAGE_COLS;
+                    const uint32_t sfb_col = sfa_col + 8;
+                    const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
+                    const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
+                    for (int a = 0; a < natoms; ++a) {
+                        ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
+                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
+                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + 1024 + 512 * a));
+                    }
+                    for (int kk = 0; kk < 2 * natoms; ++kk) {
+                        const uint32_t sf_id = (uint32_t)(kk & 1) * 2u;  // bytes 0-1 or 2-3 of the atom
+                        const uint32_t idesc = IDESC_MXF4 | (sf_id << 29) | (sf_id << 4);
+                        ptx::mma_mxf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32), idesc,
+                                           sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
+                        accumulate = 1;
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        ptx::mma_bf16_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                                           IDESC_BF16, accumulate);
+                        accumulate = 1;
+                    }
+                }
+                ptx::tc_commit_pair_mc(ptx::smem_u32(&S.empty[stage]), PAIR_MASK);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            ptx::tc_commit_pair_mc(ptx::smem_u32(&S.acc_full), PAIR_MASK);
+            acc_phase ^= 1u;
+        }
+        if (!ok) raise_abort(S, p.status);
+        // all issued tensor-core work has finished before tensor memory is freed
+        ptx::tc_commit_pair_mc(ptx::smem_u32(&S.drain), 0x1);
+        ptx::mbar_wait_bounded(ptx::smem_u32(&S.drain), 0, drain_ns, never);
+    }
+}
+
+// Epilogue, warps 0..7 of both CTAs: drain the accumulator, release
+// it to the MMA issuer, then convert and store.
+template <int EPI>
+__device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int warp, int lane, uint32_t rank,
+                                              int pair, int npairs, int tiles, const volatile int* abort,
+                                              uint32_t tmem) {
+    const int q = warp & 3;                   // TMEM lanes 32q..32q+31 are reachable from this warp
+    const int half = warp >> 2;  // columns [128*half, 128*half + 128) of the tile
+    const uint32_t acc_empty_leader = ptx::mapa(ptx::smem_u32(&S.acc_empty), 0);
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < tiles; tile += npairs) {
+        int m_blk, n_blk;
+        tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
+        int ok = 1;
+        if (lane == 0)
+            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&S.acc_full), acc_phase, p.wait_limit_ns, abort) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            if (lane == 0) raise_abort(S, p.status);
+            break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + half * 128;
+        const int64_t y0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + q * 32;
+        const int64_t x0 = (int64_t)n_blk * BN + half * 128;
+        if constexpr (EPI == OSM_EPI_GELU_REQUANT) {
+            // lane = row, 32 consecutive columns per load: whole MX blocks per lane
+            uint32_t r[128];
+            ptx::tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            ptx::tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            ptx::tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+            ptx::tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+            release_accumulator(acc_empty_leader, lane);
+            uint32_t hw[64];
+            requant_convert(p, x0, r, hw);
+            requant_group<0>(p, y0 + lane, x0, hw);
+            requant_group<1>(p, y0 + lane, x0, hw);
+            requant_group<2>(p, y0 + lane, x0, hw);
+            requant_group<3>(p, y0 + lane, x0, hw);
+        } else {
+            // four lanes per row: full 32-byte sectors per store
+            uint32_t r[128];
+            tmem_ld_16x256b_x16(taddr, r);
+            tmem_ld_16x256b_x16(taddr + (16u << 16), r + 64);
+            release_accumulator(acc_empty_leader, lane);
+            if (x0 < p.N) {
+                store_slab<EPI>(p, y0, x0, lane, r);
+                store_slab<EPI>(p, y0 + 16, x0, lane, r + 64);
+            }
+        }
+        acc_phase ^= 1u;
+    }
+}
+
+// Both CTAs done (no MMA, copy or tensor-memory read in flight), then warp 1
+// frees the pair's tensor memory. Lanes that skipped a single-thread role
+// wait for their elected lane first.
+__device__ __forceinline__ void teardown(int warp, uint32_t tmem) {
+    __syncwarp();
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     dual_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -214,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         never = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == PRODUCER_WARP && lane == 0) {
         if (p.n_fp4) {
             ptx::prefetch_tmap(&p.tm_a);
             ptx::prefetch_tmap(&p.tm_b);
@@ -232,169 +559,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
     ptx::tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer (both CTAs)
-        if (ptx::elect_one()) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int last_stage = -1;
-            uint32_t last_phase = 0;
-            bool ok = true;
-            for (int tile = pair; tile < tiles && ok; tile += npairs) {
-                int m_blk, n_blk;
-                tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
-                const int arow = m_blk * 2 * BM + static_cast<int>(rank) * BM;        // this CTA's A rows
-                const int brow = n_blk * BN + static_cast<int>(rank) * (BN / 2);      // this CTA's B rows
-                const int nbt = min(2, p.n_row_tiles - 2 * n_blk);                   // valid B scale row tiles
-                const int sfa_tile = 2 * m_blk + static_cast<int>(rank);              // A scale row tile
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.empty[stage]), phase ^ 1u, p.wait_limit_ns,
-                                                abort)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = ptx::mapa(ptx::smem_u32(&S.full[stage]), 0);  // leader's barrier
-                    if (ks < p.n_fp4) {
-                        const int natoms = min(2, p.katoms - 2 * ks);
-                        if (leader)
-                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]),
-                                                       2u * (A_TILE + B_TILE + natoms * 512u * (1u + nbt)));
-                        ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_a, ks * 128, arow, fb);
-                        ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, brow, fb);
-                        for (int a = 0; a < natoms; ++a) {
-                            ptx::tma_load_2d_pair(ptx::smem_u32(S.sfa[stage]) + 512 * a, &p.tm_sa, 0,
-                                                  (sfa_tile * p.katoms + 2 * ks + a) * 4, fb);
-                            for (int h = 0; h < nbt; ++h)
-                                ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + 1024 * h + 512 * a, &p.tm_sb, 0,
-                                                      ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 4, fb);
-                        }
-                    } else {
-                        const int kh = ks - p.n_fp4;
-                        if (leader)
-                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]), 2u * (A_TILE + B_TILE));
-                        ptx::tma_load_2d_pair(ptx::smem_u32(S.a[stage]), &p.tm_ah, kh * 64, arow, fb);
-                        ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_bh, kh * 64, brow, fb);
-                    }
-                    last_stage = stage;
-                    last_phase = phase;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                }
-            }
-            if (!ok) raise_abort(S, p.status);
-            // Let every copy this thread issued land before the pair exits: the
-            // last slot it filled is released (empty) only after the MMAs that
-            // read it completed, which implies all earlier copies completed too.
-            if (last_stage >= 0) {
-                if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.empty[last_stage]), last_phase, drain_ns,
-                                                    &never))
-                    ptx::spin_ns(1000000);  // an aborted pipeline: give any in-flight copy ample time to land
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer (leader CTA)
-        if (leader && ptx::elect_one()) {
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            bool ok = true;
-            const uint32_t acc = tmem;  // lane 0, column 0
-            for (int tile = pair; tile < tiles && ok; tile += npairs) {
-                if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.acc_empty), acc_phase ^ 1u, p.wait_limit_ns,
-                                                    abort)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                uint32_t accumulate = 0;
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.full[stage]), phase, p.wait_limit_ns, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    const uint32_t a_base = ptx::smem_u32(S.a[stage]);
-                    const uint32_t b_base = ptx::smem_u32(S.b[stage]);
-                    if (ks < p.n_fp4) {
-                        const int natoms = min(2, p.katoms - 2 * ks);
-                        const uint32_t sfa_col = tmem + SF_COL0 + stage * SF_STAGE_COLS;
-                        const uint32_t sfb_col = sfa_col + 8;
-                        const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
-                        const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
-                        for (int a = 0; a < natoms; ++a) {
-                            ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
-                            ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
-                            ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + 1024 + 512 * a));
-                        }
-                        for (int kk = 0; kk < 2 * natoms; ++kk) {
-                            const uint32_t sf_id = (uint32_t)(kk & 1) * 2u;  // bytes 0-1 or 2-3 of the atom
-                            const uint32_t idesc = IDESC_MXF4 | (sf_id << 29) | (sf_id << 4);
-                            ptx::mma_mxf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32), idesc,
-                                               sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
-                            accumulate = 1;
-                        }
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            ptx::mma_bf16_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
-                                               IDESC_BF16, accumulate);
-                            accumulate = 1;
-                        }
-                    }
-                    ptx::tc_commit_pair_mc(ptx::smem_u32(&S.empty[stage]), PAIR_MASK);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                }
-                if (!ok) break;
-                ptx::tc_commit_pair_mc(ptx::smem_u32(&S.acc_full), PAIR_MASK);
-                acc_phase ^= 1u;
-            }
-            if (!ok) raise_abort(S, p.status);
-            // all issued tensor-core work has finished before tensor memory is freed
-            ptx::tc_commit_pair_mc(ptx::smem_u32(&S.drain), 0x1);
-            ptx::mbar_wait_bounded(ptx::smem_u32(&S.drain), 0, drain_ns, &never);
-        }
+    // Warpgroup-uniform register split (for the epilogues that need it). Each
+    // side ends with its own copy of the teardown, so that no code is shared
+    // between the two budgets.
+    if (warp >= PRODUCER_WARP) {
+        if constexpr (uses_register_split(EPI)) ptx::setmaxnreg_dec<CTRL_REGS>();
+        if (warp == PRODUCER_WARP) producer_role(p, S, rank, leader, pair, npairs, tiles, ksteps, abort, &never, drain_ns);
+        else if (warp == MMA_WARP) mma_role(p, S, leader, pair, npairs, tiles, ksteps, abort, &never, drain_ns, tmem);
+        teardown(warp, tmem);
     } else {
-        // ------------------------------------------------------ epilogue (both CTAs)
-        const int q = warp & 3;           // TMEM lanes 32q..32q+31 are reachable from this warp
-        const int half = (warp - 2) >> 2;  // columns [128*half, 128*half + 128) of the tile
-        const uint32_t acc_empty_leader = ptx::mapa(ptx::smem_u32(&S.acc_empty), 0);
-        uint32_t acc_phase = 0;
-        for (int tile = pair; tile < tiles; tile += npairs) {
-            int m_blk, n_blk;
-            tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
-            int ok = 1;
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(ptx::smem_u32(&S.acc_full), acc_phase, p.wait_limit_ns, abort) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
-                if (lane == 0) raise_abort(S, p.status);
-                break;
-            }
-            ptx::tc_fence_after();
-            uint32_t r[128];
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + half * 128;
-            tmem_ld_16x256b_x16(taddr, r);
-            tmem_ld_16x256b_x16(taddr + (16u << 16), r + 64);
-            ptx::tmem_ld_wait();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
-            acc_phase ^= 1u;
-            const int64_t y0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + q * 32;
-            const int64_t x0 = (int64_t)n_blk * BN + half * 128;
-            if (x0 < p.N) {
-                store_slab(p, y0, x0, lane, r);
-                store_slab(p, y0 + 16, x0, lane, r + 64);
-            }
-        }
-    }
-
-    __syncwarp();  // lanes that skipped a single-thread role wait here for their elected lane
-    ptx::tc_fence_before();
-    ptx::cluster_sync();  // both CTAs done: no MMA, copy or tensor-memory read in flight
-    if (warp == 1) {
-        __syncwarp();
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+        if constexpr (uses_register_split(EPI)) ptx::setmaxnreg_inc<EPI_REGS>();
+        epilogue_role<EPI>(p, S, warp, lane, rank, pair, npairs, tiles, abort, tmem);
+        teardown(warp, tmem);
     }
 }
 
@@ -439,7 +615,8 @@ size_t dual_gemm_smem_bytes() { return sizeof(Smem) + 1024; }
 
 int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
                      int64_t M, const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
-                     const float* bias, int epi, void* Y, cudaStream_t st) {
+                     const float* bias, int epi, void* Y, const osm_plan* next, uint8_t* next_codes,
+                     uint8_t* next_scales, uint16_t* next_hp, cudaStream_t st) {
     static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -484,18 +661,46 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     p.num_n = static_cast<int>(ceil_div(pl->N, BN));
     p.n_row_tiles = static_cast<int>(ceil_div(pl->N, 128));
     p.epi = epi;
+    if (epi == OSM_EPI_GELU_REQUANT) {
+        p.next_codes = next_codes;
+        p.next_scales = next_scales;
+        p.next_hp = next_hp;
+        p.inv_s_ord = next->d_inv_s_ord;
+        p.nKb = static_cast<int>(next->Kb);
+        p.nKbp = static_cast<int>(next->Kbp);
+        p.nk = static_cast<int>(next->k);
+        p.nkp = static_cast<int>(next->kp);
+        p.m_pad = round_up(M, 128);
+    }
 
-    // co-resident clusters of two CTAs, queried once per device
-    static LaunchInfo info[64];
+    void (*kernel)(GemmParams) = nullptr;
+    switch (epi) {
+        case OSM_EPI_F32: kernel = dual_gemm_kernel<OSM_EPI_F32>; break;
+        case OSM_EPI_BF16: kernel = dual_gemm_kernel<OSM_EPI_BF16>; break;
+        case OSM_EPI_GELU_REQUANT: kernel = dual_gemm_kernel<OSM_EPI_GELU_REQUANT>; break;
+        case OSM_EPI_GELU_BF16: kernel = dual_gemm_kernel<OSM_EPI_GELU_BF16>; break;
+        default: return fail(OSM_ERR_INVALID_ARG, "dual_gemm: epilogue %d", epi);
+    }
+
+    // co-resident clusters of two CTAs, queried once per device and epilogue
+    static LaunchInfo info[64][4];
     static std::mutex mu;
     int dev = 0;
     if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
     if (dev < 0 || dev >= 64) return fail(OSM_ERR_UNSUPPORTED, "device index %d", dev);
     const size_t smem = sizeof(Smem) + 1024;
+    LaunchInfo& li = info[dev][epi];
     {
         std::lock_guard<std::mutex> lk(mu);
-        if (!info[dev].ready) {
-            if ((rc = check_cuda(cudaFuncSetAttribute(dual_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (!li.ready) {
+            // The register split assumes the launch gives every thread exactly
+            // LAUNCH_REGS: with fewer, the epilogue's increase could never be met.
+            cudaFuncAttributes fa;
+            if ((rc = check_cuda(cudaFuncGetAttributes(&fa, kernel), "dual_gemm attributes"))) return rc;
+            if (uses_register_split(epi) && fa.numRegs != LAUNCH_REGS)
+                return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: built with %d registers per thread, the split needs %d",
+                            fa.numRegs, LAUNCH_REGS);
+            if ((rc = check_cuda(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                       static_cast<int>(smem)),
                                  "dual_gemm smem attribute")))
                 return rc;
@@ -511,18 +716,18 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int clusters = 0;
-            if ((rc = check_cuda(cudaOccupancyMaxActiveClusters(&clusters, dual_gemm_kernel, &cfg),
+            if ((rc = check_cuda(cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg),
                                  "dual_gemm cluster occupancy")))
                 return rc;
             if (clusters < 1) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: no CTA pair fits on this device");
-            info[dev].max_pairs = clusters;
-            info[dev].ready = true;
+            li.max_pairs = clusters;
+            li.ready = true;
         }
     }
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
     if (tiles > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: too many tiles");
-    const int pairs = static_cast<int>(tiles < info[dev].max_pairs ? tiles : info[dev].max_pairs);
-    dual_gemm_kernel<<<2 * pairs, NUM_THREADS, smem, st>>>(p);
+    const int pairs = static_cast<int>(tiles < li.max_pairs ? tiles : li.max_pairs);
+    kernel<<<2 * pairs, NUM_THREADS, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "dual_gemm launch");
 }
 

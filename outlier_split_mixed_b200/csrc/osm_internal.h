@@ -19,6 +19,8 @@ struct osm_plan {
                          //      outlier slot i  -> (Kbp/32)*QA_BLOCK_BYTES + 2*i
     int32_t* d_J;        // [Kb] bulk position -> channel (ascending)
     int32_t* d_O;        // [k]  outlier slot -> channel (ascending)
+    int32_t* d_order;    // [K]  channel order [J ascending | O ascending] (bulk positions, then slots)
+    float* d_inv_s_ord;  // [K]  inv_s in that order: inv_s[d_order[c]]
     uint32_t* d_status;  // OSM_STATUS_* bits written by kernels
     uint64_t wait_limit_ns;
 };
@@ -47,13 +49,14 @@ inline int64_t scales_bytes(int64_t rows, int64_t Kbp) {
 // launchers (return OSM_OK or an error code; arguments already validated)
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st);
 int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cudaStream_t st);
-int launch_pack_weights(const osm_plan* p, const uint16_t* W, uint8_t* codes, uint8_t* scales,
-                        uint16_t* hp, cudaStream_t st);
+int launch_pack_weights(const osm_plan* p, const uint16_t* W, const int32_t* col_order, uint8_t* codes,
+                        uint8_t* scales, uint16_t* hp, cudaStream_t st);
 int launch_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st);
 int launch_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_scales,
                      const uint16_t* a_hp, int64_t M, const uint8_t* w_codes,
                      const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi,
-                     void* Y, cudaStream_t st);
+                     void* Y, const osm_plan* next, uint8_t* next_codes, uint8_t* next_scales,
+                     uint16_t* next_hp, cudaStream_t st);
 
 }  // namespace osm

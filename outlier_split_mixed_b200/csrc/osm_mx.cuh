@@ -1,0 +1,134 @@
+// Device helpers shared by the kernels that produce MXFP4 operands
+// (quantize_act, pack_weights and the fused FFN epilogue of dual_gemm):
+// BF16 rounding, the OCP MX shared exponent, E2M1 conversion, and the FP32
+// tanh-form GELU used between the two FFN projections.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+namespace osm {
+namespace mx {
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// FP32 -> BF16 bits, round to nearest even (cvt.rn.bf16.f32).
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+// MX shared exponent X = floor(log2 amax) - 2, clamped to [-127, 127],
+// amax == 0 -> -127. amax is a finite, non-negative float; floor(log2) is
+// read from the exponent field (subnormals from the leading mantissa bit).
+__device__ __forceinline__ int exponent(float amax) {
+    const uint32_t u = __float_as_uint(amax);
+    if (u == 0u) return -127;
+    const int e = static_cast<int>((u >> 23) & 0xFFu);
+    const int fl = e ? e - 127 : (31 - __clz(u & 0x7FFFFFu)) - 149;
+    int X = fl - 2;
+    X = X < -127 ? -127 : X;
+    X = X > 127 ? 127 : X;
+    return X;
+}
+
+// 2^-X as an exact float for X in [-127, 127].
+__device__ __forceinline__ float exp2_neg(int X) {
+    return X <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - X) << 23)
+                    : __uint_as_float(0x00400000u >> (X - 127));
+}
+
+// Two FP32 values -> E2M1x2 (round to nearest even, saturating at +-6),
+// element `lo` in the low nibble; the sign of a code is the sign of its
+// input, also for inputs that round to zero.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint16_t out;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+        "cvt.u16.u8 %0, b;\n\t}"
+        : "=h"(out)
+        : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Eight BF16 values (4 packed words, element 0 in the low half of word 0)
+// scaled by `inv` (a power of two, so exact) -> eight E2M1 codes, element i
+// in nibble i.
+__device__ __forceinline__ uint32_t encode8_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float inv) {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16) * inv;
+        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
+        out |= e2m1x2(lo, hi) << (8 * i);
+    }
+    return out;
+}
+
+// exp(a) for a <= 0 in FP32, exactly 0 below -86 (exp(a) < 2^-124 there).
+// On [-86, 0]: Cody-Waite reduction a = n ln2 + r with ln2 split into a
+// 12-bit high part and a low remainder, the degree-7 Taylor polynomial of
+// exp(r) in Horner form with fused multiply-adds, and an exact scaling by
+// 2^n. n = round(a log2 e) comes from one fused multiply-add onto 1.5*2^23
+// (FP32 spacing 1 there), so its integer value is read off the low bits of
+// the sum and no conversion instruction is needed. Every operation is an
+// explicitly rounded intrinsic so that no contraction or reassociation
+// changes the result.
+__device__ __forceinline__ float gelu_exp_neg(float a) {
+    const float ac = fminf(fmaxf(a, -86.0f), 0.0f);
+    const float t = __fmaf_rn(ac, 0x1.715476p+0f, 0x1.8p+23f);
+    const float n = __fsub_rn(t, 0x1.8p+23f);
+    float r = __fmaf_rn(-n, 0x1.62e4p-1f, ac);
+    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);
+    float p = 0x1.a01a02p-13f;
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    // t = 1.5*2^23 + n with n in [-124, 0]: its bit pattern is that of 1.5*2^23 plus n
+    const uint32_t e = (__float_as_uint(t) - 0x4B400000u + 127u) << 23;
+    const float v = __fmul_rn(p, __uint_as_float(e));
+    return a < -86.0f ? 0.0f : v;
+}
+
+// 1/d for d in [1, 2]: linear seed 24/17 - (8/17) d, then three Newton
+// steps y <- y + y (1 - d y) as two fused multiply-adds each.
+__device__ __forceinline__ float gelu_recip(float d) {
+    float y = __fmaf_rn(-0x1.e1e1e2p-2f, d, 0x1.69696ap+0f);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const float e = __fmaf_rn(-d, y, 1.0f);
+        y = __fmaf_rn(y, e, y);
+    }
+    return y;
+}
+
+// GELU_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), for
+// finite x, through 0.5 (1 + tanh(u)) = sigma(2u): with E = exp(-2|u|),
+// sigma(2u) = 1/(1+E) for u >= 0 and E/(1+E) for u < 0 (u has the sign of
+// x). Operations in this order: x2 = x x; k = fma(C1, x2, 1); u = (C0 x) k;
+// E; y = recip(1 + E); (x (x < 0 ? E : 1)) y. No division, no branch.
+__device__ __forceinline__ float gelu_tanh(float x) {
+    const float C0 = 0x1.988454p-1f;  // sqrt(2/pi)
+    const float C1 = 0x1.6e4e26p-5f;  // 0.044715
+    const float x2 = __fmul_rn(x, x);
+    const float k = __fmaf_rn(C1, x2, 1.0f);
+    const float u = __fmul_rn(__fmul_rn(C0, x), k);
+    const float E = gelu_exp_neg(__fmul_rn(-2.0f, fabsf(u)));
+    const float y = gelu_recip(__fadd_rn(1.0f, E));
+    const float s = x < 0.0f ? E : 1.0f;
+    return __fmul_rn(__fmul_rn(x, s), y);
+}
+
+// Byte offset of E8M0 scale (row r, 32-block b) in the tcgen05 block-scale
+// layout: 512-byte atoms of 128 rows x 4 blocks.
+__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t b, int64_t katoms) {
+    return ((r >> 7) * katoms + (b >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
+}  // namespace mx
+}  // namespace osm

@@ -18,6 +18,14 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// Per-warpgroup register budget (setmaxnreg): every warp of the warpgroup
+// executes the same instruction; an increase waits until registers released
+// by other warpgroups of the CTA cover it.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
     asm volatile(

@@ -12,44 +12,19 @@
 #include <cstdint>
 
 #include "osm_internal.h"
+#include "osm_mx.cuh"
 
 namespace osm {
 namespace {
 
 // ------------------------------------------------------------ helpers
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+using mx::bf16_bits_to_f32;
+using mx::exp2_neg;
+using mx::f32_to_bf16_bits;
+using mx::sf_offset;
 
-// FP32 -> BF16 bits, round to nearest even (cvt.rn.bf16.f32).
-__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
-}
-
-// MX shared exponent X = floor(log2 amax) - 2, clamped to [-127, 127],
-// amax == 0 -> -127. amax is a finite, non-negative float; floor(log2) is
-// read from the exponent field (subnormals from the leading mantissa bit).
-__device__ __forceinline__ int mx_exponent(float amax) {
-    const uint32_t u = __float_as_uint(amax);
-    if (u == 0u) return -127;
-    const int e = static_cast<int>((u >> 23) & 0xFFu);
-    const int fl = e ? e - 127 : (31 - __clz(u & 0x7FFFFFu)) - 149;
-    int X = fl - 2;
-    X = X < -127 ? -127 : X;
-    X = X > 127 ? 127 : X;
-    return X;
-}
-
-// 2^-X as an exact float for X in [-127, 127].
-__device__ __forceinline__ float exp2_neg(int X) {
-    return X <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - X) << 23)
-                    : __uint_as_float(0x00400000u >> (X - 127));
-}
-
-// Byte offset of E8M0 scale (row r, 32-block b) in the tcgen05 block-scale
-// layout: 512-byte atoms of 128 rows x 4 blocks.
-__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t b, int64_t katoms) {
-    return ((r >> 7) * katoms + (b >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
-}
+__device__ __forceinline__ int mx_exponent(float amax) { return mx::exponent(amax); }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;
@@ -73,32 +48,7 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Two FP32 values -> E2M1x2 (round to nearest even, saturating at +-6):
-// element `lo` in the low nibble. The sign of the code is the sign of the
-// input, including for inputs that round to zero.
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-    uint16_t out;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
-        "cvt.u16.u8 %0, b;\n\t}"
-        : "=h"(out)
-        : "f"(lo), "f"(hi));
-    return out;
-}
-
-// Eight BF16 values (4 packed words) scaled by `inv` (a power of two, so
-// exact) -> eight E2M1 codes, element i in nibble i.
-__device__ __forceinline__ uint32_t encode8_words(uint4 q, float inv) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t out = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16) * inv;
-        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
-        out |= e2m1x2(lo, hi) << (8 * i);
-    }
-    return out;
-}
+__device__ __forceinline__ uint32_t encode8_words(uint4 q, float inv) { return mx::encode8_words(q.x, q.y, q.z, q.w, inv); }
 
 // ------------------------------------------------------------ calibration
 
@@ -156,6 +106,7 @@ __global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t* __rest
 
 struct PackParams {
     const uint16_t* W;  // [K][N]
+    const int32_t* col_order;  // packed row n takes W column col_order[n] (NULL: n)
     const float* s;     // [K]
     const int32_t* J;   // [Kb]
     const int32_t* O;   // [k]
@@ -183,7 +134,8 @@ __global__ void __launch_bounds__(256) pack_bulk_kernel(PackParams p) {
         uint32_t bits = 0;
         if (nvalid && pos < p.Kb) {
             const int32_t j = __ldg(p.J + pos);
-            const float w = bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + n]);
+            const int64_t src = p.col_order ? __ldg(p.col_order + n) : n;
+            const float w = bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + src]);
             bits = f32_to_bf16_bits(w * __ldg(p.s + j));
         }
         if (i & 1) h[i >> 1] |= bits << 16; else h[i >> 1] = bits;
@@ -229,7 +181,8 @@ __global__ void __launch_bounds__(256) pack_hp_kernel(PackParams p) {
     uint32_t bits = 0;
     if (i < p.k) {
         const int32_t j = p.O[i];
-        bits = f32_to_bf16_bits(bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + n]) * p.s[j]);
+        const int64_t src = p.col_order ? p.col_order[n] : n;
+        bits = f32_to_bf16_bits(bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + src]) * p.s[j]);
     }
     p.hp[n * p.kp + i] = static_cast<uint16_t>(bits);
 }
@@ -386,9 +339,9 @@ int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cud
     return check_cuda(cudaGetLastError(), "weight_amax launch");
 }
 
-int launch_pack_weights(const osm_plan* pl, const uint16_t* W, uint8_t* codes, uint8_t* scales,
-                        uint16_t* hp, cudaStream_t st) {
-    PackParams p{W, pl->d_s, pl->d_J, pl->d_O, pl->K, pl->N, pl->k, pl->Kb, pl->Kbp, pl->kp,
+int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* col_order, uint8_t* codes,
+                        uint8_t* scales, uint16_t* hp, cudaStream_t st) {
+    PackParams p{W, col_order, pl->d_s, pl->d_J, pl->d_O, pl->K, pl->N, pl->k, pl->Kb, pl->Kbp, pl->kp,
                  pl->wmode, codes, scales, hp};
     if (pl->Kbp > 0) {
         dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 32),

@@ -1,0 +1,150 @@
+"""The FFN epilogues of dual_gemm: OSM_EPI_GELU_BF16 and the fused
+OSM_EPI_GELU_REQUANT, which hands the hidden activations of an FFN
+up-projection to the down-projection already smoothed, split and
+MXFP4-encoded (implementation paragraph of "W4A4 Quantization for
+Inference on Wan2.2-I2V-A14B": activations divided by s, quantised,
+routed)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import outlier_split_mixed_b200 as osm  # noqa: E402
+from outlier_split_mixed_b200 import synth  # noqa: E402
+from gpu_helpers import assert_bitexact, to_dev_bf16, to_np_u16, unswizzle  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    osm.lib()
+
+
+def _grid_values(rng, shape, scale_exp):
+    # magnitudes 4 or 6 (E2M1 values, so every 32-block has exponent 0 before
+    # the power-of-two scale) with random signs: every product and every
+    # partial sum of the layer is then exact in FP32
+    mags = rng.choice(np.array([4.0, 6.0], np.float32), size=shape)
+    signs = rng.choice(np.array([-1.0, 1.0], np.float32), size=shape)
+    return synth.to_bf16_bits(mags * signs * np.float32(2.0 ** scale_exp))
+
+
+def _order(K, O):
+    return np.concatenate([np.setdiff1d(np.arange(K), O), O]).astype(np.int32)
+
+
+def test_fused_requant_is_bitexact_with_exact_accumulators():
+    rng = np.random.default_rng(2024)
+    M, K, N, k = 300, 512, 768, 32            # up-projection: K -> N = next K
+    Nn, kn = 256, 64                          # next (down) layer: N -> Nn with kn outliers
+    X = _grid_values(rng, (M, K), 0)
+    W = _grid_values(rng, (K, N), -10)
+    O_up = np.sort(rng.choice(K, k, replace=False)).astype(np.int32)
+    s_up = np.ones(K, np.float32)
+    s_next = np.exp(rng.uniform(-0.7, 0.7, N)).astype(np.float32)
+    O_next = np.sort(rng.choice(N, kn, replace=False)).astype(np.int32)
+    inv_next = (np.float32(1.0) / s_next).astype(np.float32)
+    order = _order(N, O_next)
+
+    # ---- CUDA path
+    up = osm.Plan(K, N, k, s_up, O_up, osm.WSCALE_STRIP128x1)
+    nxt = osm.Plan(N, Nn, kn, s_next, O_next, osm.WSCALE_1x32)
+    assert np.array_equal(nxt.channel_order(), order)
+    Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
+    ac, asc, ah = up.alloc_packed(M)
+    osm.quantize_act(up, Xd, ac, asc, ah)
+    wc, wsc, wh = up.alloc_packed(N)
+    osm.pack_weights_for_next(up, nxt, Wd, wc, wsc, wh)
+    nc, ns, nh = nxt.alloc_packed(M)
+    osm.dual_gemm(up, ac, asc, ah, M, wc, wsc, wh, None, epi=osm.EPI_GELU_REQUANT, next_plan=nxt,
+                  next_buffers=(nc, ns, nh))
+    # GELU_BF16 on the natural packing
+    wc2, wsc2, wh2 = up.alloc_packed(N)
+    osm.pack_weights(up, Wd, wc2, wsc2, wh2)
+    H = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(up, ac, asc, ah, M, wc2, wsc2, wh2, H, epi=osm.EPI_GELU_BF16)
+    torch.cuda.synchronize()
+    assert up.status() == 0
+
+    # ---- oracle: natural order
+    ac_o, asc_o, ah_o = oracle.quantize_act(X, s_up, O_up)
+    wc_o, wsc_o, wh_o = oracle.pack_weights(W, s_up, O_up, osm.WSCALE_STRIP128x1)
+    y, _ = oracle.dual_gemm_rows(ac_o, asc_o, ah_o, np.arange(M), wc_o, wsc_o, wh_o)
+    assert np.array_equal(y, y.astype(np.float32).astype(np.float64)), "construction: accumulators exact in FP32"
+    H_o = oracle.gelu_bf16(y)
+    assert_bitexact("GELU_BF16 output", to_np_u16(H), H_o)
+    nc_o, ns_o, nh_o = oracle.quantize_act(H_o, inv_next, O_next)
+    assert_bitexact("next codes", nc.cpu().numpy().reshape(M, nxt.Kbp // 2), nc_o)
+    sc = unswizzle(ns.cpu().numpy(), M, nxt.Kbp // 32)
+    assert_bitexact("next scales", sc[:M], ns_o)
+    assert np.all(sc[M:] == 0)
+    assert_bitexact("next outlier slots", to_np_u16(nh).reshape(M, nxt.kp), nh_o)
+
+
+@pytest.mark.parametrize("shape", [(512, 1024, 1536, 32, 48), (130, 512, 1024, 0, 64), (256, 512, 768, 64, 0)],
+                         ids=["partial_bulk_block", "up_k0", "next_k0"])
+def test_fused_requant_equals_gelu_bf16_then_quantize(shape):
+    # Realistic data: the fused epilogue must equal the unfused pipeline
+    # (GELU_BF16 epilogue, then quantize_act of the next layer) bit for bit,
+    # since both see the same FP32 accumulators.
+    M, K, N, k, kn = shape
+    X = synth.acts_heavy_tailed(M, K, seed=600 + K, frac=0.02)
+    W = synth.weights_gaussian(K, N, seed=601 + K, sigma=0.04)
+    Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
+    s, _, O, _, _ = osm.calibrate([Xd], Wd, 0.6, k)
+    up = osm.Plan(K, N, k, s, O, osm.WSCALE_STRIP128x1)
+    ac, asc, ah = up.alloc_packed(M)
+    osm.quantize_act(up, Xd, ac, asc, ah)
+    wc, wsc, wh = up.alloc_packed(N)
+    osm.pack_weights(up, Wd, wc, wsc, wh)
+    H = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(up, ac, asc, ah, M, wc, wsc, wh, H, epi=osm.EPI_GELU_BF16)
+    Wn = synth.weights_gaussian(N, 256, seed=602 + K, sigma=0.02)
+    sn, _, On, _, _ = osm.calibrate([H], to_dev_bf16(Wn), 0.5, kn)
+    nxt = osm.Plan(N, 256, kn, sn, On, osm.WSCALE_TILE32x32)
+    c1, s1, h1 = nxt.alloc_packed(M)
+    osm.quantize_act(nxt, H, c1, s1, h1)
+    wc2, wsc2, wh2 = up.alloc_packed(N)
+    osm.pack_weights_for_next(up, nxt, Wd, wc2, wsc2, wh2)
+    c2, s2, h2 = nxt.alloc_packed(M)
+    for t in (c2, s2):
+        t.fill_(0xAB)          # stale bytes must all be overwritten
+    h2.fill_(3.0)
+    osm.dual_gemm(up, ac, asc, ah, M, wc2, wsc2, wh2, None, epi=osm.EPI_GELU_REQUANT, next_plan=nxt,
+                  next_buffers=(c2, s2, h2))
+    torch.cuda.synchronize()
+    assert up.status() == 0
+    assert torch.equal(c1, c2)
+    assert torch.equal(s1, s2)
+    assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
+
+
+def test_gelu_bf16_epilogue_tracks_the_oracle_on_real_data():
+    # Accumulators differ from the FP64 sums by FP32 rounding, so compare the
+    # GELU outputs within the accumulation bound pushed through GELU
+    # (|GELU'| <= 1.13) plus one BF16 rounding.
+    M, K, N, k = 200, 768, 512, 48
+    X = synth.acts_heavy_tailed(M, K, seed=611, frac=0.02)
+    W = synth.weights_gaussian(K, N, seed=612, sigma=0.04)
+    Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
+    s, inv_s, O, _, _ = osm.calibrate([Xd], Wd, 0.6, k)
+    plan = osm.Plan(K, N, k, s, O, osm.WSCALE_1x32)
+    ac, asc, ah = plan.alloc_packed(M)
+    osm.quantize_act(plan, Xd, ac, asc, ah)
+    wc, wsc, wh = plan.alloc_packed(N)
+    osm.pack_weights(plan, Wd, wc, wsc, wh)
+    H = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(plan, ac, asc, ah, M, wc, wsc, wh, H, epi=osm.EPI_GELU_BF16)
+    torch.cuda.synchronize()
+    so, inv_so, Oo = oracle.calibrate(oracle.act_amax(X), oracle.weight_amax(W), 0.6, k)
+    ac_o, asc_o, ah_o = oracle.quantize_act(X, inv_so, Oo)
+    wc_o, wsc_o, wh_o = oracle.pack_weights(W, so, Oo, 0)
+    y, T = oracle.dual_gemm_rows(ac_o, asc_o, ah_o, np.arange(M), wc_o, wsc_o, wh_o)
+    h_ref = synth.bf16_bits_to_f32(oracle.gelu_bf16(y)).astype(np.float64)
+    h = H.float().cpu().numpy().astype(np.float64)
+    tol = 1.13 * (1e-5 * T + 1e-6) + 2.0 ** -8 * np.abs(h_ref) + 1e-6
+    assert np.all(np.abs(h - h_ref) <= tol)

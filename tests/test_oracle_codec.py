@@ -115,8 +115,33 @@ def test_gelu_tanh_close_to_libm(x):
     assert abs(got - want) <= 4e-7 * abs(x) + 1e-7 * abs(want) + 1e-30
 
 
+def test_gelu_recip_within_one_ulp_on_one_to_two():
+    # Newton's iteration from the linear seed: 1/d to within one FP32 ulp of
+    # the exact reciprocal over [1, 2] (dense sample plus both ends).
+    rng = np.random.default_rng(17)
+    ds = np.concatenate([np.linspace(1.0, 2.0, 20001), rng.uniform(1.0, 2.0, 20000), [1.0, 2.0]]).astype(np.float32)
+    for d in ds:
+        got = np.float32(oracle.gelu_recip(float(d)))
+        exact = 1.0 / float(d)
+        ulp = float(np.spacing(np.float32(exact)))
+        assert abs(float(got) - exact) <= ulp, (float(d), float(got), exact)
+    assert oracle.gelu_recip(1.0) == 1.0 and oracle.gelu_recip(2.0) == 0.5
+
+
+def test_gelu_tanh_dense_against_fp64_formula():
+    # Over the range the FFN accumulators span, the FP32 routine stays within
+    # a few FP32 ulps of the FP64 formula (and is exactly 0 at 0).
+    xs = np.concatenate([np.linspace(-12, 12, 24001), np.linspace(-1e-3, 1e-3, 2001)]).astype(np.float32)
+    for x in xs:
+        x = float(x)
+        want = 0.5 * x * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+        got = oracle.gelu_tanh_f32(x)
+        assert abs(got - want) <= 5e-7 * abs(want) + 2e-8 * abs(x) + 1e-37, (x, got, want)
+    assert oracle.gelu_tanh_f32(0.0) == 0.0
+
+
 def test_gelu_exp_close_to_libm():
-    for x in np.linspace(-88, 0, 2001):
+    for x in np.linspace(-86, 0, 2001):
         want = math.exp(float(np.float32(x)))
         got = oracle.gelu_exp_neg(float(x))
         assert abs(got - want) <= 3e-7 * want + 1e-38, x

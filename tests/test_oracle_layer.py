@@ -256,3 +256,41 @@ def test_error_falls_as_k_grows():
         errs.append(np.linalg.norm(y - ref) / np.linalg.norm(ref))
     assert errs[-1] < errs[0]
     assert errs[2] < errs[0]
+
+
+def test_channel_reordering_is_invisible_to_quantize_act():
+    # Permuting the channels to [J | O] (bulk ascending, then outliers
+    # ascending), permuting inv_s alike and declaring the last k channels the
+    # outliers gives the same codes, scales and slots as the natural layout:
+    # the reading under which an FFN up-projection may emit its output columns
+    # pre-ordered for the down-projection.
+    M, K, k = 24, 320, 37
+    X = synth.acts_heavy_tailed(M, K, seed=81, frac=0.03)
+    rng = np.random.default_rng(82)
+    inv_s = np.exp(rng.uniform(-0.6, 0.6, K)).astype(np.float32)
+    O = np.sort(rng.choice(K, k, replace=False)).astype(np.int32)
+    order = np.concatenate([np.setdiff1d(np.arange(K), O), O])
+    nat = oracle.quantize_act(X, inv_s, O)
+    perm = oracle.quantize_act(X[:, order], inv_s[order], np.arange(K - k, K, dtype=np.int32))
+    for a, b in zip(nat, perm):
+        assert np.array_equal(a, b)
+    # ...while reversing the bulk channels (a different compaction) changes them
+    other = np.concatenate([np.setdiff1d(np.arange(K), O)[::-1], O])
+    moved = oracle.quantize_act(X[:, other], inv_s[other], np.arange(K - k, K, dtype=np.int32))
+    assert not np.array_equal(moved[0], nat[0])
+    assert np.array_equal(moved[2], nat[2])
+
+
+def test_gelu_bf16_special_values():
+    # GELU(0) = 0; for large |x| the tanh saturates to +-1 exactly in FP32,
+    # giving GELU(x) = x and GELU(-x) = -0; values match the scalar routine
+    # rounded to BF16 and stay within a BF16 ulp of the FP64 formula.
+    y = np.array([0.0, 12.0, 300.0, -12.0, -300.0, 1.0, -1.0, 0.5, 3.0, -2.5])
+    h = oracle.gelu_bf16(y)
+    f = synth.bf16_bits_to_f32(h).astype(np.float64)
+    assert f[0] == 0.0 and f[1] == 12.0 and f[2] == 300.0
+    assert f[3] == 0.0 and f[4] == 0.0
+    for yi, hi, fi in zip(y, h, f):
+        assert hi == oracle.f32_to_bf16(oracle.gelu_tanh_f32(yi))
+        want = 0.5 * yi * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (yi + 0.044715 * yi ** 3)))
+        assert abs(fi - want) <= 2.0 ** -8 * abs(want) + 1e-30, yi
