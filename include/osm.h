@@ -91,7 +91,7 @@ typedef enum {
  * this library specifies it, with only IEEE round-to-nearest-even adds,
  * multiplies and fused multiply-adds: 0.5 (1 + tanh(u)) = sigma(2u) is
  * 1/(1 + E) for x >= 0 and E/(1 + E) for x < 0, E = exp(-2|u|) (Cody-Waite
- * reduction, degree-7 Taylor polynomial, 0 below exp(-86)), the reciprocal
+ * reduction, degree-7 Taylor polynomial, 0 below 2^-126), the reciprocal
  * by a linear seed and three Newton steps. */
 typedef enum {
     OSM_EPI_F32 = 0,          /* Y [M][N] float32                                     */

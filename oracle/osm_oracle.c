@@ -467,20 +467,20 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
 /* ------------------------------------------------------------------ */
 
 /*
- * exp(a) for a <= 0 in FP32, taken as exactly 0 below -86 (where exp(a) <
- * 2^-124); on [-86, 0] with explicit operations: Cody-Waite
- * reduction a = n*ln2 + r (|r| <= ln2/2) with ln2 split into a 12-bit high
- * part and a low remainder; exp(r) by its Taylor series to degree 7 in
- * Horner form with fused multiply-adds (fmaf, one rounding each); the
- * result scaled by 2^n. n is a*log2(e) rounded to the nearest integer (ties
- * to even) in one fused step: t = fmaf(a, LOG2E, 1.5*2^23) lies in
- * [2^23, 2^24), where the FP32 spacing is 1, and n = t - 1.5*2^23 exactly.
- * On that range 2^n (and the result) stay normal, so the scaling is exact.
- * Constants are the binary32 values of log2(e), ln2 split, and 1/k!.
+ * exp(a) for a <= 0 in FP32, with explicit operations: a is first clamped
+ * to -100; Cody-Waite reduction a = n*ln2 + r (|r| <= ln2/2) with ln2 split
+ * into a 12-bit high part and a low remainder; exp(r) by its Taylor series
+ * to degree 7 in Horner form with fused multiply-adds (fmaf, one rounding
+ * each). n is a*log2(e) rounded to the nearest integer (ties to even) in one
+ * fused step: t = fmaf(a, LOG2E, 1.5*2^23) lies in [2^23, 2^24), where the
+ * FP32 spacing is 1, and n = t - 1.5*2^23 exactly. The result is 0 for
+ * n < -126 (exp(a) < 2^-126), else p * 2^n rounded once (exact unless it
+ * is subnormal). Constants are the binary32 values of log2(e), ln2 split,
+ * and 1/k!.
  */
 float oracle_gelu_exp_neg(float a)
 {
-    if (a < -86.0f) return 0.0f;
+    if (a < -100.0f) a = -100.0f;
     if (a > 0.0f) a = 0.0f;
     const float LOG2E = 0x1.715476p+0f;
     const float LN2_HI = 0x1.62e4p-1f;      /* 12 significant bits */
@@ -498,7 +498,8 @@ float oracle_gelu_exp_neg(float a)
     p = fmaf(p, r, 0.5f);
     p = fmaf(p, r, 1.0f);
     p = fmaf(p, r, 1.0f);
-    return ldexpf(p, (int)n);
+    if (n < -126.0f) return 0.0f;
+    return p * ldexpf(1.0f, (int)n);
 }
 
 /*
@@ -522,10 +523,11 @@ float oracle_gelu_recip(float d)
  * GELU in its tanh form, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi)(x + 0.044715
  * x^3), for finite x, evaluated through the identity 0.5 (1 + tanh(u)) =
  * sigma(2u) = 1 / (1 + exp(-2u)): with E = exp(-2|u|),
- *   sigma(2u) = 1 / (1 + E)  for u >= 0,   E / (1 + E)  for u < 0,
- * and u has the sign of x. Every operation in FP32 in the order written:
- * x2 = x*x; k = fmaf(C1, x2, 1); u = (C0*x)*k; E = exp(-2|u|) as above;
- * y = recip(1 + E); result (x * (x < 0 ? E : 1)) * y.
+ *   x sigma(2u) = x / (1 + E)  for u >= 0,   x E / (1 + E)  for u < 0,
+ * and u has the sign of x, so the numerator is max(x, x E) (0 <= E <= 1).
+ * Every operation in FP32 in the order written: x2 = x*x;
+ * k = fmaf(C1, x2, 1); u = (C0*x)*k; E = exp(-2|u|) as above;
+ * y = recip(1 + E); result fmaxf(x, x*E) * y.
  */
 float oracle_gelu_tanh_f32(float x)
 {
@@ -536,8 +538,7 @@ float oracle_gelu_tanh_f32(float x)
     float u = (C0 * x) * k;
     float E = oracle_gelu_exp_neg(-2.0f * fabsf(u));
     float y = oracle_gelu_recip(1.0f + E);
-    float s = x < 0.0f ? E : 1.0f;
-    return (x * s) * y;
+    return fmaxf(x, x * E) * y;
 }
 
 /* FFN hidden activations from FP64 accumulators: h = bf16(GELU(fp32(y))),

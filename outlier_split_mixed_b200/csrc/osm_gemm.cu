@@ -225,41 +225,18 @@ __device__ __forceinline__ void release_accumulator(uint32_t acc_empty_leader, i
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
 }
-// OSM_EPI_GELU_REQUANT, step 1: the lane's 128 accumulators (one row,
-// columns c_base .. c_base+127) become x' = bf16(bf16(GELU(acc)) * inv_s) of
-// the next layer, packed as BF16 pairs (element 2i in the low half of word
-// i). Column c of this layer is channel order[c] of the next layer, whose
-// reciprocal smoothing factor is inv_s_ord[c]. Columns >= N are not read.
-__device__ __forceinline__ void requant_convert(const GemmParams& p, int64_t c_base, const uint32_t (&r)[128],
-                                                uint32_t (&hw)[64]) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        if (c_base + 4 * i >= p.N) break;
-        const float4 sv = __ldg(reinterpret_cast<const float4*>(p.inv_s_ord + c_base) + i);
-        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
-        uint32_t xs[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t hb = mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])));
-            xs[j] = mx::f32_to_bf16_bits(__fmul_rn(mx::bf16_bits_to_f32(hb), s4[j]));
-        }
-        hw[2 * i] = xs[0] | (xs[1] << 16);
-        hw[2 * i + 1] = xs[2] | (xs[3] << 16);
-    }
-}
-// Step 2, one 32-column group G (columns c0 = c_base + 32G ..): column
-// c < nKb is bulk position c, column c >= nKb is outlier slot c - nKb. The
-// bulk part is MXFP4-encoded as one block (codes 16 bytes, one scale byte;
-// in a partial last block the positions >= nKb are padding, code 0) and
-// the outlier part goes to next_hp. The group holding the last bulk position
-// also writes the next layer's padding blocks (code 0, scale 0), the group
-// holding the last column the outlier padding slots, and lanes of padding
-// rows (M <= row < M rounded up to 128) write scale 0.
-template <int G>
-__device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, int64_t c_base, const uint32_t (&hwall)[64]) {
-    const int64_t c0 = c_base + 32 * G;
-    if (c0 >= p.N) return;
-    const uint32_t* hw = hwall + 16 * G;
+// OSM_EPI_GELU_REQUANT for one 32-column group of one row (the lane's row),
+// columns c0 .. c0+31 (c0 < N; N % 32 == 0, so all 32 are real). Column c
+// of this layer is channel order[c] of the next layer, with reciprocal
+// smoothing factor inv_s_ord[c]; column c < nKb is bulk position c, column
+// c >= nKb is outlier slot c - nKb. h = bf16(GELU(acc)), x' = bf16(h * inv_s),
+// then the bulk part is MXFP4-encoded as one block (codes 16 bytes, one scale
+// byte; in a partial last block the positions >= nKb are padding, code 0)
+// and the outlier part goes to next_hp. The group holding the last bulk
+// position also writes the next layer's padding blocks (code 0, scale 0),
+// the group holding the last column the outlier padding slots, and lanes of
+// padding rows (M <= row < M rounded up to 128) write scale 0 only.
+__device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, int64_t c0, const uint32_t* r) {
     const int katoms = p.nKbp >> 7;
     const bool holds_last_bulk = p.nKb > 0 && c0 <= p.nKb - 1 && p.nKb - 1 < c0 + 32;
     if (row >= p.M) {
@@ -269,6 +246,21 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
                 for (int b = (p.nKb + 31) >> 5; b < (p.nKbp >> 5); ++b) p.next_scales[mx::sf_offset(row, b, katoms)] = 0;
         }
         return;
+    }
+    uint32_t hw[16];  // x' as BF16 pairs, element 2i in the low half of word i
+    const float4* iv = reinterpret_cast<const float4*>(p.inv_s_ord + c0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 sv = __ldg(iv + i);
+        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+        uint32_t xs[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t hb = mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])));
+            xs[j] = mx::f32_to_bf16_bits(__fmul_rn(mx::bf16_bits_to_f32(hb), s4[j]));
+        }
+        hw[2 * i] = xs[0] | (xs[1] << 16);
+        hw[2 * i + 1] = xs[2] | (xs[3] << 16);
     }
     if (c0 < p.nKb) {
         const int nreal = static_cast<int>(p.nKb - c0 < 32 ? p.nKb - c0 : 32);
@@ -313,6 +305,17 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
         if (p.nkp > p.nk && c0 <= p.N - 1 && p.N - 1 < c0 + 32)
             for (int i = p.nk; i < p.nkp; ++i) hp[i] = 0;
     }
+}
+
+// The epilogue code for a whole 128-column strip, unrolled, does not fit
+// the instruction cache; the strips are processed in a rolled loop over
+// column groups instead. Registers cannot be indexed at run time, so after
+// each step the accumulator array shifts down by the step's width (register
+// moves) and the loop body always reads r[0 ..].
+template <int STEP, int N>
+__device__ __forceinline__ void shift_down(uint32_t (&r)[N]) {
+#pragma unroll
+    for (int j = 0; j + STEP < N; ++j) r[j] = r[j + STEP];
 }
 
 // TMA producer, one elected thread in each CTA of the pair.
@@ -475,12 +478,12 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int 
             ptx::tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
             ptx::tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
             release_accumulator(acc_empty_leader, lane);
-            uint32_t hw[64];
-            requant_convert(p, x0, r, hw);
-            requant_group<0>(p, y0 + lane, x0, hw);
-            requant_group<1>(p, y0 + lane, x0, hw);
-            requant_group<2>(p, y0 + lane, x0, hw);
-            requant_group<3>(p, y0 + lane, x0, hw);
+#pragma unroll 1
+            for (int g = 0; g < 4; g += 2) {
+                if (x0 + 32 * g < p.N) requant_group(p, y0 + lane, x0 + 32 * g, r);
+                if (x0 + 32 * g + 32 < p.N) requant_group(p, y0 + lane, x0 + 32 * g + 32, r + 32);
+                shift_down<64>(r);
+            }
         } else {
             // four lanes per row: full 32-byte sectors per store
             uint32_t r[128];
@@ -488,8 +491,11 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int 
             tmem_ld_16x256b_x16(taddr + (16u << 16), r + 64);
             release_accumulator(acc_empty_leader, lane);
             if (x0 < p.N) {
-                store_slab<EPI>(p, y0, x0, lane, r);
-                store_slab<EPI>(p, y0 + 16, x0, lane, r + 64);
+#pragma unroll 1
+                for (int sl = 0; sl < 2; ++sl) {
+                    store_slab<EPI>(p, y0 + 16 * sl, x0, lane, r);
+                    shift_down<64>(r);
+                }
             }
         }
         acc_phase ^= 1u;

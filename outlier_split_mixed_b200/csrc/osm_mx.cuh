@@ -66,17 +66,17 @@ __device__ __forceinline__ uint32_t encode8_words(uint32_t w0, uint32_t w1, uint
     return out;
 }
 
-// exp(a) for a <= 0 in FP32, exactly 0 below -86 (exp(a) < 2^-124 there).
-// On [-86, 0]: Cody-Waite reduction a = n ln2 + r with ln2 split into a
-// 12-bit high part and a low remainder, the degree-7 Taylor polynomial of
-// exp(r) in Horner form with fused multiply-adds, and an exact scaling by
-// 2^n. n = round(a log2 e) comes from one fused multiply-add onto 1.5*2^23
-// (FP32 spacing 1 there), so its integer value is read off the low bits of
-// the sum and no conversion instruction is needed. Every operation is an
-// explicitly rounded intrinsic so that no contraction or reassociation
-// changes the result.
+// exp(a) for a <= 0 in FP32: a clamped to -100, Cody-Waite reduction
+// a = n ln2 + r with ln2 split into a 12-bit high part and a low remainder,
+// the degree-7 Taylor polynomial of exp(r) in Horner form with fused
+// multiply-adds, then p * 2^n rounded once, or 0 for n < -126. n =
+// round(a log2 e) comes from one fused multiply-add onto 1.5*2^23 (FP32
+// spacing 1 there), so its integer value is read off the low bits of the sum
+// and the factor 2^n is built from bits (an exponent field clamped at 0
+// gives the factor 0). Every operation is an explicitly rounded intrinsic so
+// that no contraction or reassociation changes the result.
 __device__ __forceinline__ float gelu_exp_neg(float a) {
-    const float ac = fminf(fmaxf(a, -86.0f), 0.0f);
+    const float ac = fmaxf(a, -100.0f);
     const float t = __fmaf_rn(ac, 0x1.715476p+0f, 0x1.8p+23f);
     const float n = __fsub_rn(t, 0x1.8p+23f);
     float r = __fmaf_rn(-n, 0x1.62e4p-1f, ac);
@@ -89,10 +89,9 @@ __device__ __forceinline__ float gelu_exp_neg(float a) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    // t = 1.5*2^23 + n with n in [-124, 0]: its bit pattern is that of 1.5*2^23 plus n
-    const uint32_t e = (__float_as_uint(t) - 0x4B400000u + 127u) << 23;
-    const float v = __fmul_rn(p, __uint_as_float(e));
-    return a < -86.0f ? 0.0f : v;
+    // t = 1.5*2^23 + n with n in [-145, 0]: its bit pattern is that of 1.5*2^23 plus n
+    const int e = max(static_cast<int>(__float_as_uint(t) - 0x4B400000u) + 127, 0);
+    return __fmul_rn(p, __uint_as_float(static_cast<uint32_t>(e) << 23));
 }
 
 // 1/d for d in [1, 2]: linear seed 24/17 - (8/17) d, then three Newton
@@ -109,9 +108,10 @@ __device__ __forceinline__ float gelu_recip(float d) {
 
 // GELU_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), for
 // finite x, through 0.5 (1 + tanh(u)) = sigma(2u): with E = exp(-2|u|),
-// sigma(2u) = 1/(1+E) for u >= 0 and E/(1+E) for u < 0 (u has the sign of
-// x). Operations in this order: x2 = x x; k = fma(C1, x2, 1); u = (C0 x) k;
-// E; y = recip(1 + E); (x (x < 0 ? E : 1)) y. No division, no branch.
+// x sigma(2u) = x/(1+E) for u >= 0 and x E/(1+E) for u < 0; u has the sign
+// of x and 0 <= E <= 1, so the numerator is max(x, x E). Operations in this
+// order: x2 = x x; k = fma(C1, x2, 1); u = (C0 x) k; E; y = recip(1 + E);
+// max(x, x E) y. No division, no branch.
 __device__ __forceinline__ float gelu_tanh(float x) {
     const float C0 = 0x1.988454p-1f;  // sqrt(2/pi)
     const float C1 = 0x1.6e4e26p-5f;  // 0.044715
@@ -120,8 +120,7 @@ __device__ __forceinline__ float gelu_tanh(float x) {
     const float u = __fmul_rn(__fmul_rn(C0, x), k);
     const float E = gelu_exp_neg(__fmul_rn(-2.0f, fabsf(u)));
     const float y = gelu_recip(__fadd_rn(1.0f, E));
-    const float s = x < 0.0f ? E : 1.0f;
-    return __fmul_rn(__fmul_rn(x, s), y);
+    return __fmul_rn(fmaxf(x, __fmul_rn(x, E)), y);
 }
 
 // Byte offset of E8M0 scale (row r, 32-block b) in the tcgen05 block-scale
