@@ -8,7 +8,11 @@ up-projection, 4096 tokens x 5120 -> 13824, alpha 0.6, k = 128 outliers,
 128x1 weight stripes, FP32 output.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload up|down|long|tiny]
+                  [--workload up|down|long|tiny|ffn]
+
+`--workload ffn` runs four FFN blocks of 32760 tokens (up 5120 -> 13824
+with GELU, smoothing and requantisation fused into its epilogue, then down
+13824 -> 5120 to BF16); one step is all four blocks.
 
 Multi-GPU (torchrun, one rank per GPU): tokens are data-parallel, each rank
 runs its own batch with no collective on the data path (weak scaling); the
@@ -49,7 +53,39 @@ def load_peaks():
 
 def workloads():
     from outlier_split_mixed_b200 import synth
-    return {"up": synth.UP, "down": synth.DOWN, "long": synth.LONG, "tiny": synth.TINY}
+    return {"up": synth.UP, "down": synth.DOWN, "long": synth.LONG, "tiny": synth.TINY, "ffn": synth.FFN}
+
+
+METRIC = "dual-branch W4A4 GEMM effective TFLOP/s (+act quantize)"
+
+
+WSCALE_NAMES = {0: "1x32", 1: "32x32", 2: "128x1"}
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one dual_gemm
+# launch, from one ncu capture of the current kernel on the workload; a
+# workload without a capture of the current kernel reports null.
+DUAL_GEMM_TRAFFIC = {"wan_ffn_up_4096x5120x13824": 92.180992e6 + 179.756544e6}
+
+
+def workload_config(cfg):
+    if hasattr(cfg, "layers"):
+        return {"workload": cfg.name, "layers": cfg.layers, "M": cfg.M, "d_model": cfg.d_model, "d_ff": cfg.d_ff,
+                "k_up": cfg.k_up, "k_down": cfg.k_down, "alpha_up": cfg.alpha_up, "alpha_down": cfg.alpha_down,
+                "wscale_up": WSCALE_NAMES[cfg.wmode_up], "wscale_down": WSCALE_NAMES[cfg.wmode_down],
+                "calib_tokens": cfg.calib_tokens}
+    return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "k": cfg.k, "alpha": cfg.alpha}
+
+
+def blended_peak(peaks, parts):
+    """Tensor-pipe peak for a mix of FP4 and BF16 MMAs: parts is a list of
+    (fp4_flops, bf16_flops); FP4 runs at the measured BF16 burst x 4 (the
+    nominal dense ratio), BF16 at the measured BF16 burst."""
+    p16 = peaks["bf16_tflops"]
+    p4 = p16 * FP4_PER_BF16
+    f4 = sum(a for a, _ in parts)
+    f16 = sum(b for _, b in parts)
+    t_ideal = f4 / (p4 * 1e12) + f16 / (p16 * 1e12)
+    return (f4 + f16) / t_ideal / 1e12, p16
 
 
 # ------------------------------------------------------------------ clocks
@@ -139,19 +175,65 @@ def oracle_sample_throughput(cfg, rows_per_step: int, steps: int, warmup: int):
     return flops / t / 1e12, t, cores
 
 
+def oracle_ffn_throughput(cfg, rows_per_step: int, steps: int, warmup: int, calib_rows: int = 64):
+    """Time the CPU oracle on the FFN chain: per block quantize (up),
+    dual-branch product, GELU to BF16, quantize (down), dual-branch product,
+    on `rows_per_step` tokens per block per step. Calibration (on the first
+    `calib_rows` tokens of each block's calibration batch; down-projection
+    statistics from the unquantised GELU(X W_up)) and weight packing are
+    offline, outside the timed region."""
+    import oracle
+    preps = []
+    for l in range(cfg.layers):
+        Xc = cfg.make_calib(l)[:calib_rows]
+        Wu, Wd = cfg.make_w_up(l), cfg.make_w_down(l)
+        s_u, inv_u, O_u = oracle.calibrate(oracle.act_amax(Xc), oracle.weight_amax(Wu), cfg.alpha_up, cfg.k_up)
+        allc = np.arange(cfg.d_model, dtype=np.int32)
+        ones = np.ones(cfg.d_model, np.float32)
+        fa = oracle.quantize_act(Xc, ones, allc)
+        fw = oracle.pack_weights(Wu, ones, allc, cfg.wmode_up)
+        y, _ = oracle.dual_gemm_rows(*fa, np.arange(Xc.shape[0]), *fw)
+        Hc = oracle.gelu_bf16(y)
+        s_d, inv_d, O_d = oracle.calibrate(oracle.act_amax(Hc), oracle.weight_amax(Wd), cfg.alpha_down, cfg.k_down)
+        preps.append(dict(inv_u=inv_u, O_u=O_u, wu=oracle.pack_weights(Wu, s_u, O_u, cfg.wmode_up),
+                          inv_d=inv_d, O_d=O_d, wd=oracle.pack_weights(Wd, s_d, O_d, cfg.wmode_down),
+                          X=cfg.make_x(l, max(256, rows_per_step * (steps + warmup)))))
+    times = []
+    r = np.arange(rows_per_step)
+    for i in range(steps + warmup):
+        t0 = time.perf_counter()
+        for pr in preps:
+            lo = (i * rows_per_step) % max(1, pr["X"].shape[0] - rows_per_step)
+            a = oracle.quantize_act(pr["X"][lo:lo + rows_per_step], pr["inv_u"], pr["O_u"])
+            y, _ = oracle.dual_gemm_rows(*a, r, *pr["wu"])
+            h = oracle.gelu_bf16(y)
+            a2 = oracle.quantize_act(h, pr["inv_d"], pr["O_d"])
+            oracle.dual_gemm_rows(*a2, r, *pr["wd"])
+        t1 = time.perf_counter()
+        if i >= warmup:
+            times.append(t1 - t0)
+    t = float(np.mean(times))
+    flops = cfg.layers * 2.0 * 2.0 * rows_per_step * cfg.d_model * cfg.d_ff
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return flops / t / 1e12, t, cores
+
+
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return 0
-    rows = max(1, args.ref_rows)
-    tflops, t, cores = oracle_sample_throughput(cfg, rows, args.steps, args.warmup)
+    is_ffn = cfg.name == workloads()["ffn"].name
+    rows = max(1, args.ref_rows if not is_ffn else max(1, args.ref_rows // 8))
+    if is_ffn:
+        tflops, t, cores = oracle_ffn_throughput(cfg, rows, args.steps, args.warmup)
+    else:
+        tflops, t, cores = oracle_sample_throughput(cfg, rows, args.steps, args.warmup)
     line = {
         "impl": "reference",
-        "metric": "dual-branch W4A4 GEMM effective TFLOP/s (+act quantize)",
+        "metric": METRIC,
         "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "k": cfg.k, "alpha": cfg.alpha,
-                   "sample_rows_per_step": rows},
+        "config": dict(workload_config(cfg), sample_rows_per_step=rows),
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows} of {cfg.M} tokens per step, weights packed offline"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -266,7 +348,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         q_bytes = M * K * 2 + cb + sb + hb
         q_gbs = q_bytes / quant_s / 1e9
         line = {
-            "metric": "dual-branch W4A4 GEMM effective TFLOP/s (+act quantize)",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
@@ -283,7 +365,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                                  "frac_hbm": q_gbs / peaks["hbm_gbs"]},
             },
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
-                         "frac": achieved / peak_blend, "traffic": None, "kernel": "dual_gemm",
+                         "frac": achieved / peak_blend, "traffic": DUAL_GEMM_TRAFFIC.get(cfg.name),
+                         "traffic_unit": "bytes per launch", "kernel": "dual_gemm",
                          "peak_source": f"{peak_src}: bf16 burst {p16} x4 for the FP4 share, x1 for the "
                                         f"BF16 share (k={plan.k} of K={K})"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
@@ -302,13 +385,196 @@ def run_ours(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_ffn(args, cfg, rank, world, local_rank):
+    """Four FFN blocks on one stream. Per block and step: quantize_act of the
+    block input for the up-projection; dual_gemm up with the fused GELU +
+    smoothing + MXFP4 requantisation epilogue, writing the down-projection's
+    packed activations; dual_gemm down to BF16."""
+    import torch
+    import torch.distributed as dist
+
+    import outlier_split_mixed_b200 as osm
+    from outlier_split_mixed_b200 import dist as odist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    M, D, F = cfg.M, cfg.d_model, cfg.d_ff
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    blocks = []
+    for l in range(cfg.layers):
+        Xc, Wu, Wd = to_dev(cfg.make_calib(l)), to_dev(cfg.make_w_up(l)), to_dev(cfg.make_w_down(l))
+        # up-projection statistics
+        amax = torch.zeros(D, dtype=torch.float32, device=dev)
+        wmax = torch.empty(D, dtype=torch.float32, device=dev)
+        osm.act_amax_accumulate(Xc, amax)
+        osm.weight_amax(Wu, wmax)
+        s_u, _, O_u = odist.calibrate_from_local_stats(amax, wmax, cfg.alpha_up, cfg.k_up)
+        # down-projection statistics from the unquantised GELU(Xc W_up): k = K, s = 1
+        full = osm.Plan(D, F, D, np.ones(D, np.float32), np.arange(D, dtype=np.int32), cfg.wmode_up)
+        fa = full.alloc_packed(Xc.shape[0], dev)
+        fw = full.alloc_packed(F, dev)
+        osm.quantize_act(full, Xc, *fa)
+        osm.pack_weights(full, Wu, *fw)
+        Hc = torch.empty((Xc.shape[0], F), dtype=torch.bfloat16, device=dev)
+        osm.dual_gemm(full, *fa, Xc.shape[0], *fw, Hc, epi=osm.EPI_GELU_BF16)
+        amax_d = torch.zeros(F, dtype=torch.float32, device=dev)
+        wmax_d = torch.empty(F, dtype=torch.float32, device=dev)
+        osm.act_amax_accumulate(Hc, amax_d)
+        osm.weight_amax(Wd, wmax_d)
+        s_d, _, O_d = odist.calibrate_from_local_stats(amax_d, wmax_d, cfg.alpha_down, cfg.k_down)
+        full.close()
+        del fa, fw, Hc
+        up = osm.Plan(D, F, cfg.k_up, s_u, O_u, cfg.wmode_up)
+        down = osm.Plan(F, D, cfg.k_down, s_d, O_d, cfg.wmode_down)
+        wu = up.alloc_packed(F, dev)
+        osm.pack_weights_for_next(up, down, Wu, *wu)
+        wd = down.alloc_packed(D, dev)
+        osm.pack_weights(down, Wd, *wd)
+        del Wu, Wd, Xc
+        blocks.append(dict(up=up, down=down, wu=wu, wd=wd, X=cfg.make_x(l)))
+    # activation buffers shared by the blocks; each block has its own input and output
+    a_up = blocks[0]["up"].alloc_packed(M, dev)
+    a_dn = blocks[0]["down"].alloc_packed(M, dev)
+    for b in blocks:
+        b["Xd"] = to_dev(b["X"])
+        b["Y"] = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def block(b, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        osm.quantize_act(b["up"], b["Xd"], *a_up)
+        if ev is not None:
+            ev[1].record(stream)
+        osm.dual_gemm(b["up"], *a_up, M, *b["wu"], None, epi=osm.EPI_GELU_REQUANT, next_plan=b["down"],
+                      next_buffers=a_dn)
+        if ev is not None:
+            ev[2].record(stream)
+        osm.dual_gemm(b["down"], *a_dn, M, *b["wd"], b["Y"], epi=osm.EPI_BF16)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        for b in blocks:
+            block(b)
+    torch.cuda.synchronize()
+
+    n = args.steps
+    L = cfg.layers
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)] for _ in range(n)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(n):
+            flush.fill_(float(i))                    # evict L2 between timed steps (untimed)
+            for l, b in enumerate(blocks):
+                block(b, ev[i][l])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for b in blocks:
+        if b["up"].status() != 0 or b["down"].status() != 0:
+            raise RuntimeError("device status reports a timeout during the timed region")
+    t = np.array([[[ev[i][l][j].elapsed_time(ev[i][l][j + 1]) * 1e-3 for j in range(3)] for l in range(L)]
+                  for i in range(n)])  # [step][block][quantize, up, down]
+    t_step = np.array([ev[i][0][0].elapsed_time(ev[i][L - 1][3]) * 1e-3 for i in range(n)])
+    loc = torch.tensor([t_step.mean(), t[:, :, 0].sum(1).mean(), t[:, :, 1].sum(1).mean(), t[:, :, 2].sum(1).mean()],
+                       dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(loc, op=dist.ReduceOp.MAX)
+    step_s, quant_s, up_s, down_s = (float(x) for x in loc.cpu())
+
+    # end to end through the public API: every block input copied in from
+    # pinned host memory and every block output copied out, inside the region
+    Xh = [torch.from_numpy(b["X"].view(np.int16)).view(torch.bfloat16).pin_memory() for b in blocks]
+    Yh = [torch.empty((M, D), dtype=torch.bfloat16).pin_memory() for _ in blocks]
+
+    def e2e_step():
+        for b, xh, yh in zip(blocks, Xh, Yh):
+            b["Xd"].copy_(xh, non_blocking=True)
+            block(b)
+            yh.copy_(b["Y"], non_blocking=True)
+
+    e2e_steps = max(3, min(10, n))
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_t = torch.tensor([e0.elapsed_time(e1) * 1e-3 / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_s = float(e2e_t.item())
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops = cfg.flops
+        value = world * flops / step_s / 1e12
+        up0, dn0 = blocks[0]["up"], blocks[0]["down"]
+        f_up = L * 2.0 * M * F * D
+        f_dn = L * 2.0 * M * D * F
+        parts = [(L * 2.0 * M * F * b["up"].Kb, L * 2.0 * M * F * b["up"].k) for b in blocks[:1]] + \
+                [(L * 2.0 * M * D * b["down"].Kb, L * 2.0 * M * D * b["down"].k) for b in blocks[:1]]
+        peak_blend, p16 = blended_peak(peaks, parts)
+        gemm_s = up_s + down_s
+        achieved = (f_up + f_dn) / gemm_s / 1e12
+        cb, sb, hb = up0.sizes(M)
+        q_bytes = L * (M * D * 2 + cb + sb + hb)
+        line = {
+            "metric": METRIC,
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
+            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
+                           parallelism=f"dp{world} (token shards, no data-path collective)"),
+            "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
+            "kernels": {
+                "dual_gemm_up_gelu_requant": {"ms": up_s * 1e3, "tflops": f_up / up_s / 1e12},
+                "dual_gemm_down_bf16": {"ms": down_s * 1e3, "tflops": f_dn / down_s / 1e12},
+                "quantize_act": {"ms": quant_s * 1e3, "gbs": q_bytes / quant_s / 1e9, "bytes": q_bytes,
+                                 "frac_hbm": q_bytes / quant_s / 1e9 / peaks["hbm_gbs"]},
+            },
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
+                         "frac": achieved / peak_blend, "traffic": None, "kernel": "dual_gemm (up + down)",
+                         "peak_source": f"{peak_src}: bf16 burst {p16} x4 for the FP4 share, x1 for the BF16 "
+                                        f"share (k_up={up0.k}, k_down={dn0.k})"},
+            "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": L * M * D * 2, "d2h_bytes_per_step": L * M * D * 2,
+                    "api": "quantize_act + dual_gemm (Python binding), pinned host copies"},
+            "gpu_launches": 3 * L * n,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            rows = max(1, args.cpu_rows // 16)
+            tf, t1, cores = oracle_ffn_throughput(cfg, rows, 2, 1)
+            line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{rows} of {M} tokens per block per step (2 steps), calibration "
+                                              f"on 64 tokens, weights packed offline"}
+        print(json.dumps(line), flush=True)
+    for b in blocks:
+        b["up"].close()
+        b["down"].close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["up", "down", "long", "tiny"], default="up")
+    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn"], default="up")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -332,6 +598,8 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
+        if args.workload == "ffn":
+            return run_ffn(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
