@@ -70,7 +70,7 @@ extern "C" {
 #define OSM_ERR_NOMEM          6  /* plan allocation failed                               */
 
 /* device status bits, returned by osm_plan_status() */
-#define OSM_STATUS_TIMEOUT     1u  /* a pipeline wait in osm_dual_gemm ran out of time */
+#define OSM_STATUS_TIMEOUT     1u  /* a pipeline wait of a plan's kernel ran out of time */
 
 typedef struct osm_plan osm_plan;
 
@@ -152,10 +152,20 @@ OSM_API int osm_plan_dims(const osm_plan* plan, int64_t* K, int64_t* N, int64_t*
 OSM_API int osm_plan_status(const osm_plan* plan, void* stream, uint32_t* status_host, int clear);
 
 /* Debug knob for failure-detection tests: the wait limit, in nanoseconds,
- * of every pipeline wait inside osm_dual_gemm for this plan (default
- * 2e9). A wait that runs out sets OSM_STATUS_TIMEOUT and the kernel
- * returns early; the context stays usable. */
+ * of every pipeline wait inside osm_dual_gemm and osm_quantize_act for this
+ * plan (default 2e9). A wait that runs out sets OSM_STATUS_TIMEOUT and the
+ * kernel returns early (its outputs are then incomplete); the context stays
+ * usable. */
 OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
+
+/* Debug flags for failure-detection tests (no counterpart in the paper).
+ * OSM_DEBUG_STARVE_QUANTIZE: osm_quantize_act expects 16 bytes more per row
+ * group than its copies deliver, so every wait on a row group runs out after
+ * the wait limit: the kernel sets OSM_STATUS_TIMEOUT, waits (bounded) for
+ * its copies and returns; its outputs are incomplete. Nothing faults: the
+ * copies themselves complete. 0 restores normal operation. */
+#define OSM_DEBUG_STARVE_QUANTIZE 1u
+OSM_API int osm_plan_set_debug(osm_plan* plan, uint32_t flags);
 
 /* Channel order in which a previous layer must produce this plan's input
  * for OSM_EPI_GELU_REQUANT: order_host[c] = J[c] for c < Kb (bulk channels
@@ -193,7 +203,10 @@ OSM_API int osm_pack_weights_for_next(const osm_plan* plan, const osm_plan* next
  *   bulk x'[J_p] -> MXFP4 with the exponent floor(log2 amax_b) - 2 of each
  *   32-block (clamped to [-127,127]; amax 0 -> -127), elements E2M1 RNE,
  *   saturating at 6; the sign bit is the sign of x'.
- * Writes a_codes [M][Kbp/2], a_scales (rows padded to 128), a_hp [M][kp]. */
+ * Writes a_codes [M][Kbp/2], a_scales (rows padded to 128), a_hp [M][kp].
+ * Rows stream through shared memory by asynchronous bulk copies; a copy
+ * that does not arrive within the plan's wait limit sets OSM_STATUS_TIMEOUT
+ * in the plan status (osm_plan_status). */
 OSM_API int osm_quantize_act(const osm_plan* plan, const uint16_t* X, int64_t M, uint8_t* a_codes,
                      uint8_t* a_scales, uint16_t* a_hp, void* stream);
 

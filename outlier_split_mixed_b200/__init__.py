@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libosm.so")
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
 STATUS_TIMEOUT = 1
+DEBUG_STARVE_QUANTIZE = 1
 WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
 EPI_F32, EPI_BF16, EPI_GELU_REQUANT, EPI_GELU_BF16 = 0, 1, 2, 3
 
@@ -40,6 +41,7 @@ _SIGNATURES = {
     "osm_plan_dims": (_I, [_P] + [ctypes.POINTER(_I64)] * 6),
     "osm_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _I]),
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
+    "osm_plan_set_debug": (_I, [_P, ctypes.c_uint32]),
     "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
     "osm_pack_weights_for_next": (_I, [_P, _P, _P, _P, _P, _P, _P]),
     "osm_plan_channel_order": (_I, [_P, _P]),
@@ -173,6 +175,9 @@ class Plan:
 
     def set_wait_limit(self, ns: int):
         _check(lib().osm_plan_set_wait_limit(self._h, int(ns)))
+
+    def set_debug(self, flags: int):
+        _check(lib().osm_plan_set_debug(self._h, int(flags)))
 
     def alloc_packed(self, rows: int, device="cuda"):
         """Allocate (codes, scales, hp) torch buffers for `rows` rows."""

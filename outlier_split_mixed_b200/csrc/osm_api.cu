@@ -164,6 +164,7 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
     p->kp = round_up(k, 64);
     p->wmode = wscale_mode;
     p->wait_limit_ns = 2000000000ull;
+    p->debug_flags = 0;
 
     std::vector<float> inv_s(static_cast<size_t>(K));
     for (int64_t j = 0; j < K; ++j) inv_s[j] = 1.0f / s_host[j];
@@ -268,6 +269,14 @@ int osm_plan_set_wait_limit(osm_plan* p, uint64_t ns) {
     OSM_REQUIRE(p, "plan_set_wait_limit: plan is NULL");
     OSM_REQUIRE(ns >= 1000ull, "plan_set_wait_limit: limit below 1 us");
     p->wait_limit_ns = ns;
+    return OSM_OK;
+}
+
+int osm_plan_set_debug(osm_plan* p, uint32_t flags) {
+    g_err[0] = 0;
+    OSM_REQUIRE(p, "plan_set_debug: plan is NULL");
+    OSM_REQUIRE((flags & ~static_cast<uint32_t>(OSM_DEBUG_STARVE_QUANTIZE)) == 0, "plan_set_debug: unknown flag");
+    p->debug_flags = flags;
     return OSM_OK;
 }
 

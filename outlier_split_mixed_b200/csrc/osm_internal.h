@@ -23,6 +23,7 @@ struct osm_plan {
     float* d_inv_s_ord;  // [K]  inv_s in that order: inv_s[d_order[c]]
     uint32_t* d_status;  // OSM_STATUS_* bits written by kernels
     uint64_t wait_limit_ns;
+    uint32_t debug_flags;  // OSM_DEBUG_* (failure-detection tests)
 };
 
 namespace osm {

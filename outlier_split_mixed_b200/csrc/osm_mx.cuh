@@ -18,6 +18,13 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
+// Two FP32 values -> BF16 pair (RNE each, one cvt.rn.bf16x2.f32): lo in
+// bits 0-15, hi in bits 16-31.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return static_cast<uint32_t>(__bfloat16_as_ushort(h.x)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h.y)) << 16);
+}
+
 // MX shared exponent X = floor(log2 amax) - 2, clamped to [-127, 127],
 // amax == 0 -> -127. amax is a finite, non-negative float; floor(log2) is
 // read from the exponent field (subnormals from the leading mantissa bit).
@@ -53,16 +60,23 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
 
 // Eight BF16 values (4 packed words, element 0 in the low half of word 0)
 // scaled by `inv` (a power of two, so exact) -> eight E2M1 codes, element i
-// in nibble i.
+// in nibble i. The scaling is two packed FP32 multiplies per word (each lane
+// an IEEE multiply), and the four code bytes are packed in one step.
 __device__ __forceinline__ uint32_t encode8_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float inv) {
-    const uint32_t w[4] = {w0, w1, w2, w3};
-    uint32_t out = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16) * inv;
-        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
-        out |= e2m1x2(lo, hi) << (8 * i);
-    }
+    const float2 iv = make_float2(inv, inv);
+    const float2 v0 = __fmul2_rn(make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u)), iv);
+    const float2 v1 = __fmul2_rn(make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u)), iv);
+    const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(w2 << 16), __uint_as_float(w2 & 0xFFFF0000u)), iv);
+    const float2 v3 = __fmul2_rn(make_float2(__uint_as_float(w3 << 16), __uint_as_float(w3 & 0xFFFF0000u)), iv);
+    uint32_t out;
+    asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+        "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+        : "=r"(out)
+        : "f"(v0.x), "f"(v0.y), "f"(v1.x), "f"(v1.y), "f"(v2.x), "f"(v2.y), "f"(v3.x), "f"(v3.y));
     return out;
 }
 

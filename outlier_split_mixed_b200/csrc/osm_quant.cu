@@ -13,6 +13,7 @@
 
 #include "osm_internal.h"
 #include "osm_mx.cuh"
+#include "osm_ptx.cuh"
 
 namespace osm {
 namespace {
@@ -49,6 +50,13 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 }
 
 __device__ __forceinline__ uint32_t encode8_words(uint4 q, float inv) { return mx::encode8_words(q.x, q.y, q.z, q.w, inv); }
+
+// Two BF16 inputs (one packed word) times their inv_s -> two BF16 x' values
+// (packed): x' = bf16(fp32(x) * inv_s), one IEEE multiply per lane.
+__device__ __forceinline__ uint32_t smooth2(uint32_t w, float2 s) {
+    const float2 v = __fmul2_rn(make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)), s);
+    return mx::bf16x2_bits(v.x, v.y);
+}
 
 // ------------------------------------------------------------ calibration
 
@@ -197,6 +205,9 @@ struct QuantParams {
     uint8_t* codes;          // [M][Kbp/2]
     uint8_t* scales;         // layout, rows padded to 128
     uint16_t* hp;            // [M][kp]
+    uint32_t* status;        // OSM_STATUS_* bits
+    uint64_t wait_limit_ns;  // bound of every wait on an incoming row group
+    uint32_t extra_tx;       // bytes expected beyond each group's copy (0; 16 when starved for a test)
 };
 
 constexpr int QA_THREADS = 256;
@@ -209,9 +220,11 @@ __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * Q
 // threads hit distinct banks.
 //  phase 1: each lane loads 2 channels (32-bit) of each of the R rows -- a
 //           warp reads 128 contiguous bytes per row -- computes
-//           x' = bf16(x * inv_s) and stores both values at their routed
-//           offsets (bulk position or outlier slot); consecutive lanes write
-//           into one 128-byte window, so the stores are conflict-free;
+//           x' = bf16(x * inv_s) (a packed pair of IEEE multiplies) and
+//           stores both values at their routed offsets (bulk position or
+//           outlier slot); consecutive lanes write into one 128-byte window,
+//           so the stores are conflict-free (eight channels per lane would
+//           put a warp's stores 16 bytes apart: a 4-way bank conflict);
 //  phase 2: one thread per (row, 32-block): four 128-bit shared loads,
 //           amax by packed u16 max, E8M0 exponent, sixteen E2M1x2
 //           conversions, one 128-bit code store and one scale byte;
@@ -219,7 +232,6 @@ __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * Q
 template <int R>
 __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p) {
     extern __shared__ __align__(16) uint8_t sbuf[];
-    constexpr int UNROLL = 16 / R;
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
     const int row0 = blockIdx.x * R;
@@ -237,38 +249,39 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
         }
     }
 
-    // phase 1
+    // phase 1: each lane takes channel pairs c = tid, tid + 256, ... (a warp
+    // reads 128 contiguous bytes of each row); the pair's inv_s and routes
+    // are loaded once and serve all R rows. Consecutive lanes store into one
+    // 128-byte window of the staged row, so the routed stores do not conflict.
     const int npairs = p.K >> 1;
-    const uint32_t* X32 = reinterpret_cast<const uint32_t*>(p.X);
-    const float2* is2 = reinterpret_cast<const float2*>(p.inv_s);
-    const int2* rt2 = reinterpret_cast<const int2*>(p.route);
-    for (int c0 = tid; c0 < npairs; c0 += QA_THREADS * UNROLL) {
-        uint32_t w[UNROLL][R];
-        float2 sv[UNROLL];
-        int2 dv[UNROLL];
+    const uint32_t* xrow[R];
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
+    for (int r = 0; r < R; ++r)
+        xrow[r] = reinterpret_cast<const uint32_t*>(p.X) + static_cast<size_t>(row0 + r < p.M ? row0 + r : row0) * npairs;
+    constexpr int U = 4;
+    for (int c0 = tid; c0 < npairs; c0 += U * QA_THREADS) {
+        uint32_t w[U][R];
+        float2 sv[U];
+        int2 dv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
             const int c = c0 + u * QA_THREADS;
             if (c < npairs) {
-                sv[u] = __ldg(is2 + c);
-                dv[u] = __ldg(rt2 + c);
+                sv[u] = __ldg(reinterpret_cast<const float2*>(p.inv_s) + c);
+                dv[u] = __ldg(reinterpret_cast<const int2*>(p.route) + c);
 #pragma unroll
-                for (int r = 0; r < R; ++r)
-                    w[u][r] = (row0 + r < p.M) ? ldg_nc_u32(X32 + static_cast<size_t>(row0 + r) * npairs + c) : 0u;
+                for (int r = 0; r < R; ++r) w[u][r] = ldg_nc_u32(xrow[r] + c);
             }
         }
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int c = c0 + u * QA_THREADS;
             if (c < npairs) {
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const float lo = __uint_as_float(w[u][r] << 16) * sv[u].x;
-                    const float hi = __uint_as_float(w[u][r] & 0xFFFF0000u) * sv[u].y;
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-                    const uint32_t pk = *reinterpret_cast<const uint32_t*>(&h);
-                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].x) = static_cast<uint16_t>(pk);
-                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].y) = static_cast<uint16_t>(pk >> 16);
+                    const uint32_t h = smooth2(w[u][r], sv[u]);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].x) = static_cast<uint16_t>(h);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].y) = static_cast<uint16_t>(h >> 16);
                 }
             }
         }
@@ -277,8 +290,13 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
 
     // phase 2
     const int katoms = p.Kbp >> 7;
+    const float inv_nb = 1.0f / static_cast<float>(nb);
     for (int wi = tid; wi < R * nb; wi += QA_THREADS) {
-        const int r = wi / nb, b = wi - r * nb;
+        // r = wi / nb (exact: wi < 2^20 and the quotient is below 8)
+        int r = static_cast<int>((static_cast<float>(wi) + 0.5f) * inv_nb);
+        r -= (r * nb > wi);
+        r += ((r + 1) * nb <= wi);
+        const int b = wi - r * nb;
         const int t = row0 + r;
         if (t >= p.M) continue;
         const uint8_t* src = sbuf + r * stride + b * QA_BLOCK_BYTES;
@@ -320,6 +338,170 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
             *reinterpret_cast<uint32_t*>(p.scales + sf_offset(tile * 128 + rr, a * 4, katoms)) = 0u;
         }
     }
+}
+
+
+// Encode the staged rows [0, nrows) of a routed buffer: one thread per
+// (row, 32-block) -- four 128-bit shared loads, amax by packed u16 max, the
+// E8M0 exponent, sixteen E2M1x2 conversions, one 16-byte code store and one
+// scale byte -- then the outlier slots as 16-byte copies. Rows are
+// row0 + r of the output.
+__device__ __forceinline__ void encode_staged(const QuantParams& p, const uint8_t* sbuf, int stride, int row0,
+                                              int nrows) {
+    const int nb = p.Kbp >> 5;
+    const int katoms = p.Kbp >> 7;
+    const int tid = threadIdx.x;
+    const float inv_nb = 1.0f / static_cast<float>(nb);
+    for (int wi = tid; wi < nrows * nb; wi += blockDim.x) {
+        // r = wi / nb (exact: wi < 2^20 and the quotient is below 8)
+        int r = static_cast<int>((static_cast<float>(wi) + 0.5f) * inv_nb);
+        r -= (r * nb > wi);
+        r += ((r + 1) * nb <= wi);
+        const int b = wi - r * nb;
+        const int t = row0 + r;
+        const uint8_t* src = sbuf + r * stride + b * QA_BLOCK_BYTES;
+        const uint4 q0 = lds128(src), q1 = lds128(src + 16), q2 = lds128(src + 32), q3 = lds128(src + 48);
+        uint32_t m = vmax_u16x2(vmax_u16x2(q0.x & 0x7FFF7FFFu, q0.y & 0x7FFF7FFFu),
+                                vmax_u16x2(q0.z & 0x7FFF7FFFu, q0.w & 0x7FFF7FFFu));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q1.x & 0x7FFF7FFFu, q1.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q1.z & 0x7FFF7FFFu, q1.w & 0x7FFF7FFFu)));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q2.x & 0x7FFF7FFFu, q2.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q2.z & 0x7FFF7FFFu, q2.w & 0x7FFF7FFFu)));
+        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q3.x & 0x7FFF7FFFu, q3.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(q3.z & 0x7FFF7FFFu, q3.w & 0x7FFF7FFFu)));
+        const uint32_t amax = max(m & 0xFFFFu, m >> 16);
+        const int X = mx_exponent(bf16_bits_to_f32(amax));
+        const float inv = exp2_neg(X);
+        const uint4 out = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv), encode8_words(q2, inv),
+                                     encode8_words(q3, inv));
+        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16) = out;
+        p.scales[sf_offset(t, b, katoms)] = static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
+    }
+    const int hv = p.kp >> 3;
+    for (int i = tid; i < nrows * hv; i += blockDim.x) {
+        const int r = i / hv, c = i - r * hv;
+        *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(row0 + r) * p.kp + c * 8) =
+            lds128(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
+    }
+}
+
+// Scale bytes of the padding rows [M, round_up(M, 128)) are zero; done by
+// the CTA that handles row M - 1.
+__device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
+    const int katoms = p.Kbp >> 7;
+    const int tile = (p.M - 1) >> 7;
+    const int rem = p.M & 127;
+    if (rem == 0) return;
+    const int nwords = (128 - rem) * katoms;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) {
+        const int a = i / (128 - rem), rr = rem + (i - a * (128 - rem));
+        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(tile * 128 + rr, a * 4, katoms)) = 0u;
+    }
+}
+
+// The streaming form. Persistent CTAs take groups of R consecutive rows
+// g = blockIdx.x, blockIdx.x + gridDim.x, ...; the R rows of a group are
+// contiguous in X, so one bulk asynchronous copy (issued by thread 0, S
+// groups ahead, into a ring of S raw slots, completion on an mbarrier) brings
+// them into shared memory while the CTA works on earlier groups. Per group:
+//  route: each thread takes channel pairs c = tid, tid + 256, ... of each row
+//         from the raw slot (conflict-free 32-bit shared loads), computes
+//         x' = bf16(x * inv_s) and stores the two values at their routed
+//         offsets in the staged buffer ([bulk blocks | outlier slots], a
+//         32-block in 80 bytes); consecutive lanes write one 128-byte window;
+//  then the raw slot is refilled with the group S ahead, and the staged rows
+//  are encoded (encode_staged).
+// Every wait on a slot is bounded; a wait that runs out sets
+// OSM_STATUS_TIMEOUT, and the CTA lets its copies land before it returns.
+template <int R, int S>
+__global__ void __launch_bounds__(QA_THREADS) quantize_act_stream_kernel(QuantParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nb = p.Kbp >> 5;
+    const int stride = qa_row_stride(nb, p.kp);
+    const int raw_bytes = R * p.K * 2;
+    uint8_t* raw = smem;
+    uint8_t* sbuf = smem + S * raw_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + R * stride);
+    __shared__ int never;  // a flag nothing sets
+    const int tid = threadIdx.x;
+    const int ngroups = (p.M + R - 1) / R;
+    const int mine = blockIdx.x < ngroups ? (ngroups - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+
+    auto issue = [&](int i) {
+        const int g = blockIdx.x + i * gridDim.x;
+        const int rows = min(R, p.M - g * R);
+        const uint32_t bar = ptx::smem_u32(&full[i % S]);
+        const uint32_t bytes = static_cast<uint32_t>(rows) * p.K * 2u;
+        ptx::mbar_arrive_expect_tx(bar, bytes + p.extra_tx);
+        ptx::bulk_load(ptx::smem_u32(raw + (i % S) * raw_bytes), p.X + static_cast<size_t>(g) * R * p.K, bytes, bar);
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+        never = 0;
+        ptx::fence_mbar_init();
+    }
+    // the padding positions of the staged rows (bulk [Kb, Kbp), slots [k, kp))
+    // are never written by the routing step: zero them once
+    {
+        const int npb = p.Kbp - p.Kb, npad = npb + (p.kp - p.k);
+        for (int i = tid; i < R * npad; i += QA_THREADS) {
+            const int r = i / npad, c = i - r * npad;
+            const int pos = p.Kb + c;
+            const int off = c < npb ? (pos >> 5) * QA_BLOCK_BYTES + (pos & 31) * 2
+                                    : nb * QA_BLOCK_BYTES + (p.k + c - npb) * 2;
+            *reinterpret_cast<uint16_t*>(sbuf + r * stride + off) = 0;
+        }
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int i = 0; i < S && i < mine; ++i) issue(i);
+
+    const int npairs = p.K >> 1;
+    const float2* is2 = reinterpret_cast<const float2*>(p.inv_s);
+    const int2* rt2 = reinterpret_cast<const int2*>(p.route);
+    int issued = min(S, mine);
+    for (int i = 0; i < mine; ++i) {
+        const int g = blockIdx.x + i * gridDim.x;
+        const int rows = min(R, p.M - g * R);
+        const uint32_t bar = ptx::smem_u32(&full[i % S]);
+        const bool ok = ptx::mbar_wait_bounded(bar, static_cast<uint32_t>((i / S) & 1), p.wait_limit_ns, &never);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(p.status, OSM_STATUS_TIMEOUT);
+                // let every copy already issued land in this CTA's shared memory
+                for (int j = i; j < issued; ++j)
+                    if (!ptx::mbar_wait_bounded(ptx::smem_u32(&full[j % S]), static_cast<uint32_t>((j / S) & 1),
+                                                20000000ull, &never))
+                        ptx::spin_ns(1000000);
+            }
+            __syncthreads();
+            return;
+        }
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(raw + (i % S) * raw_bytes);
+        for (int c = tid; c < npairs; c += QA_THREADS) {
+            const float2 sv = __ldg(is2 + c);
+            const int2 dv = __ldg(rt2 + c);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (r < rows) {
+                    const uint32_t h = smooth2(src[r * npairs + c], sv);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv.x) = static_cast<uint16_t>(h);
+                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv.y) = static_cast<uint16_t>(h >> 16);
+                }
+            }
+        }
+        __syncthreads();  // raw slot consumed, staged rows complete
+        if (tid == 0 && issued < mine) issue(issued++);
+        encode_staged(p, sbuf, stride, g * R, rows);
+        if (g * R <= p.M - 1 && p.M - 1 < g * R + rows) zero_padding_scale_rows(p);
+        __syncthreads();  // staged rows free for the next group
+    }
+}
+
+template <int R, int S>
+size_t stream_smem_bytes(int K, int stride) {
+    return static_cast<size_t>(S) * R * K * 2 + static_cast<size_t>(R) * stride + 8 * S;
 }
 
 }  // namespace
@@ -372,13 +554,42 @@ static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
+template <int R, int S>
+static int launch_stream(const QuantParams& p, int stride, cudaStream_t st) {
+    const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
+    auto kern = quantize_act_stream_kernel<R, S>;
+    int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem)),
+                        "quantize_act smem attribute");
+    if (rc) return rc;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+    if ((rc = check_cuda(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count"))) return rc;
+    if ((rc = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QA_THREADS, smem),
+                         "quantize_act occupancy")))
+        return rc;
+    if (per_sm < 1) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: no CTA fits");
+    const int64_t groups = ceil_div(p.M, R);
+    const int64_t grid = groups < static_cast<int64_t>(sms) * per_sm ? groups : static_cast<int64_t>(sms) * per_sm;
+    kern<<<static_cast<unsigned>(grid), QA_THREADS, smem, st>>>(p);
+    return check_cuda(cudaGetLastError(), "quantize_act launch");
+}
+
 int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st) {
     if (M > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: M too large");
     QuantParams p{X, pl->d_inv_s, pl->d_route, static_cast<int>(M), static_cast<int>(pl->K),
                   static_cast<int>(pl->k), static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp),
-                  static_cast<int>(pl->kp), codes, scales, hp};
-    const size_t row_bytes = static_cast<size_t>(qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp)));
+                  static_cast<int>(pl->kp), codes, scales, hp, pl->d_status, pl->wait_limit_ns,
+                  (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u};
+    const int stride = qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp));
+    // streaming form: two CTAs of at most 110 KB per SM
+    const size_t two_per_sm = 110 * 1024;
+    if (stream_smem_bytes<2, 3>(p.K, stride) <= two_per_sm) return launch_stream<2, 3>(p, stride, st);
+    if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3>(p, stride, st);
+    if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2>(p, stride, st);
+    // very wide rows: the staged, phase-serial form
+    const size_t row_bytes = static_cast<size_t>(stride);
     const size_t budget = 72 * 1024;
     if (row_bytes * 8 <= budget) return launch_qa<8>(p, row_bytes * 8, st);
     if (row_bytes * 4 <= budget) return launch_qa<4>(p, row_bytes * 4, st);

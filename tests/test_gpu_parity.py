@@ -31,6 +31,8 @@ SMALL = [
     ("bf16_out_bias", 257, 768, 512, 0.7, 48, osm.WSCALE_1x32, osm.EPI_BF16, True, "gelu"),
     ("long_k_wraps_ring", 257, 5120, 512, 0.6, 128, osm.WSCALE_STRIP128x1, osm.EPI_F32, False, "heavy"),
     ("k_all_but_32", 96, 512, 256, 0.5, 480, osm.WSCALE_TILE32x32, osm.EPI_F32, False, "heavy"),
+    # rows too wide for the streaming quantize_act ring: the staged form
+    ("wide_k_staged", 40, 32768, 64, 0.5, 64, osm.WSCALE_1x32, osm.EPI_F32, False, "heavy"),
 ]
 
 
@@ -120,6 +122,36 @@ def test_short_wait_limit_reports_timeout_and_context_survives():
     osm.dual_gemm(plan, ac, asc, ah, M, wc, wsc, wh, Y3)
     torch.cuda.synchronize()
     assert torch.equal(Y2, Y3)  # deterministic and complete
+
+
+def test_quantize_act_wait_limit_reports_timeout_and_recovers():
+    # Failure detection without a fault: with the starve flag every row
+    # group's wait expects bytes that never come, so each bounded wait runs
+    # out (1 ms limit); the kernel reports OSM_STATUS_TIMEOUT, lets its copies
+    # land and returns; the context stays usable and a normal run right after
+    # equals a run on a fresh plan.
+    cfg = synth.UP
+    M = 1024
+    X = cfg.make_x(M)
+    Xd = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    rng = np.random.default_rng(11)
+    s = np.exp(rng.uniform(-0.5, 0.5, cfg.K)).astype(np.float32)
+    O = np.sort(rng.choice(cfg.K, cfg.k, replace=False)).astype(np.int32)
+    plan = osm.Plan(cfg.K, cfg.N, cfg.k, s, O, cfg.wmode)
+    ac, asc, ah = plan.alloc_packed(M)
+    plan.set_wait_limit(1_000_000)
+    plan.set_debug(osm.DEBUG_STARVE_QUANTIZE)
+    osm.quantize_act(plan, Xd, ac, asc, ah)
+    assert plan.status(clear=True) & osm.STATUS_TIMEOUT
+    plan.set_debug(0)
+    plan.set_wait_limit(2_000_000_000)
+    osm.quantize_act(plan, Xd, ac, asc, ah)
+    assert plan.status(clear=True) == 0
+    fresh = osm.Plan(cfg.K, cfg.N, cfg.k, s, O, cfg.wmode)
+    bc, bsc, bh = fresh.alloc_packed(M)
+    osm.quantize_act(fresh, Xd, bc, bsc, bh)
+    torch.cuda.synchronize()
+    assert torch.equal(ac, bc) and torch.equal(asc, bsc) and torch.equal(ah.view(torch.int16), bh.view(torch.int16))
 
 
 def test_quant_linear_and_host_entry_point_agree():
