@@ -21,8 +21,29 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
 // Two FP32 values -> BF16 pair (RNE each, one cvt.rn.bf16x2.f32): lo in
 // bits 0-15, hi in bits 16-31.
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return static_cast<uint32_t>(__bfloat16_as_ushort(h.x)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h.y)) << 16);
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// max(|a|, |b|) of each BF16 half of two packed words; the sign bits of the
+// result are the XOR of the inputs' signs (mask them off before use).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// For a BF16 block maximum (bit pattern, sign clear): the MX exponent
+// X = floor(log2 amax) - 2 clamped to [-127, 127] (amax 0 -> -127) is
+// max(e - 129, -127) with e the biased exponent field -- a subnormal or zero
+// amax is below 2^-126, so its X clamps to -127, and e <= 254 keeps X <= 125.
+// Returns X; *inv receives 2^-X (exact, normal).
+__device__ __forceinline__ int bf16_block_exponent(uint32_t amax_bits, float* inv) {
+    const int e = static_cast<int>(amax_bits >> 7);
+    const int X = max(e - 129, -127);
+    *inv = __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
+    return X;
 }
 
 // MX shared exponent X = floor(log2 amax) - 2, clamped to [-127, 127],

@@ -10,6 +10,9 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "osm_internal.h"
 #include "osm_mx.cuh"
@@ -211,6 +214,7 @@ struct QuantParams {
 };
 
 constexpr int QA_THREADS = 256;
+constexpr int STREAM_NT = 512;  // threads of the streaming form
 
 __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * QA_BLOCK_BYTES + kp * 2 + 15) & ~15; }
 
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
 // E8M0 exponent, sixteen E2M1x2 conversions, one 16-byte code store and one
 // scale byte -- then the outlier slots as 16-byte copies. Rows are
 // row0 + r of the output.
-__device__ __forceinline__ void encode_staged(const QuantParams& p, const uint8_t* sbuf, int stride, int row0,
+__device__ __forceinline__ void encode_staged(const QuantParams& p, uint32_t sbuf, int stride, int row0,
                                               int nrows) {
     const int nb = p.Kbp >> 5;
     const int katoms = p.Kbp >> 7;
@@ -359,19 +363,18 @@ __device__ __forceinline__ void encode_staged(const QuantParams& p, const uint8_
         r += ((r + 1) * nb <= wi);
         const int b = wi - r * nb;
         const int t = row0 + r;
-        const uint8_t* src = sbuf + r * stride + b * QA_BLOCK_BYTES;
-        const uint4 q0 = lds128(src), q1 = lds128(src + 16), q2 = lds128(src + 32), q3 = lds128(src + 48);
-        uint32_t m = vmax_u16x2(vmax_u16x2(q0.x & 0x7FFF7FFFu, q0.y & 0x7FFF7FFFu),
-                                vmax_u16x2(q0.z & 0x7FFF7FFFu, q0.w & 0x7FFF7FFFu));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q1.x & 0x7FFF7FFFu, q1.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q1.z & 0x7FFF7FFFu, q1.w & 0x7FFF7FFFu)));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q2.x & 0x7FFF7FFFu, q2.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q2.z & 0x7FFF7FFFu, q2.w & 0x7FFF7FFFu)));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q3.x & 0x7FFF7FFFu, q3.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q3.z & 0x7FFF7FFFu, q3.w & 0x7FFF7FFFu)));
-        const uint32_t amax = max(m & 0xFFFFu, m >> 16);
-        const int X = mx_exponent(bf16_bits_to_f32(amax));
-        const float inv = exp2_neg(X);
+        const uint32_t src = sbuf + r * stride + b * QA_BLOCK_BYTES;
+        const uint4 q0 = ptx::ld_shared_v4(src), q1 = ptx::ld_shared_v4(src + 16), q2 = ptx::ld_shared_v4(src + 32),
+                    q3 = ptx::ld_shared_v4(src + 48);
+        using mx::bf16x2_absmax;
+        const uint32_t m = bf16x2_absmax(
+            bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q0.x, q0.y), bf16x2_absmax(q0.z, q0.w)),
+                          bf16x2_absmax(bf16x2_absmax(q1.x, q1.y), bf16x2_absmax(q1.z, q1.w))),
+            bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q2.x, q2.y), bf16x2_absmax(q2.z, q2.w)),
+                          bf16x2_absmax(bf16x2_absmax(q3.x, q3.y), bf16x2_absmax(q3.z, q3.w))));
+        const uint32_t amax = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
+        float inv;
+        const int X = mx::bf16_block_exponent(amax, &inv);
         const uint4 out = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv), encode8_words(q2, inv),
                                      encode8_words(q3, inv));
         *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16) = out;
@@ -381,7 +384,7 @@ __device__ __forceinline__ void encode_staged(const QuantParams& p, const uint8_
     for (int i = tid; i < nrows * hv; i += blockDim.x) {
         const int r = i / hv, c = i - r * hv;
         *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(row0 + r) * p.kp + c * 8) =
-            lds128(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
+            ptx::ld_shared_v4(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
     }
 }
 
@@ -413,8 +416,8 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 //  are encoded (encode_staged).
 // Every wait on a slot is bounded; a wait that runs out sets
 // OSM_STATUS_TIMEOUT, and the CTA lets its copies land before it returns.
-template <int R, int S>
-__global__ void __launch_bounds__(QA_THREADS) quantize_act_stream_kernel(QuantParams p) {
+template <int R, int S, int NT, int TR>
+__global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_stream_kernel(QuantPa
     // are never written by the routing step: zero them once
     {
         const int npb = p.Kbp - p.Kb, npad = npb + (p.kp - p.k);
-        for (int i = tid; i < R * npad; i += QA_THREADS) {
+        for (int i = tid; i < R * npad; i += NT) {
             const int r = i / npad, c = i - r * npad;
             const int pos = p.Kb + c;
             const int off = c < npb ? (pos >> 5) * QA_BLOCK_BYTES + (pos & 31) * 2
@@ -460,6 +463,23 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_stream_kernel(QuantPa
     const int npairs = p.K >> 1;
     const float2* is2 = reinterpret_cast<const float2*>(p.inv_s);
     const int2* rt2 = reinterpret_cast<const int2*>(p.route);
+    // with TR > 0 (npairs <= TR * NT) each thread keeps its pairs' inv_s and
+    // routes in registers for all its groups
+    const uint32_t raw_u32 = ptx::smem_u32(raw), sbuf_u32 = ptx::smem_u32(sbuf);
+    const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
+    // with TR > 0 (npairs <= TR * NT) each thread keeps its pairs' inv_s and
+    // the shared addresses of their routed slots (row 0) in registers
+    float2 tsv[TR > 0 ? TR : 1];
+    uint2 tad[TR > 0 ? TR : 1];
+    if constexpr (TR > 0) {
+#pragma unroll
+        for (int j = 0; j < TR; ++j) {
+            const int c = tid + j * NT;
+            tsv[j] = c < npairs ? __ldg(is2 + c) : make_float2(0.f, 0.f);
+            const int2 dv = c < npairs ? __ldg(rt2 + c) : make_int2(0, 0);
+            tad[j] = make_uint2(sbuf_u32 + dv.x, sbuf_u32 + dv.y);
+        }
+    }
     int issued = min(S, mine);
     for (int i = 0; i < mine; ++i) {
         const int g = blockIdx.x + i * gridDim.x;
@@ -478,22 +498,38 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_stream_kernel(QuantPa
             __syncthreads();
             return;
         }
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(raw + (i % S) * raw_bytes);
-        for (int c = tid; c < npairs; c += QA_THREADS) {
-            const float2 sv = __ldg(is2 + c);
-            const int2 dv = __ldg(rt2 + c);
+        const uint32_t src = raw_u32 + (i % S) * raw_bytes + tid * 4;  // this thread's first pair, row 0
+        if constexpr (TR > 0) {
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                if (r < rows) {
-                    const uint32_t h = smooth2(src[r * npairs + c], sv);
-                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv.x) = static_cast<uint16_t>(h);
-                    *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv.y) = static_cast<uint16_t>(h >> 16);
+            for (int j = 0; j < TR; ++j) {
+                if (tid + j * NT < npairs) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        if (r < rows) {
+                            const uint32_t h = smooth2(ptx::ld_shared_u32(src + r * row_bytes + j * NT * 4), tsv[j]);
+                            ptx::st_shared_u16(tad[j].x + r * stride, h);
+                            ptx::st_shared_u16(tad[j].y + r * stride, h >> 16);
+                        }
+                    }
+                }
+            }
+        } else {
+            for (int c = tid; c < npairs; c += NT) {
+                const float2 sv = __ldg(is2 + c);
+                const int2 dv = __ldg(rt2 + c);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if (r < rows) {
+                        const uint32_t h = smooth2(ptx::ld_shared_u32(src + r * row_bytes + (c - tid) * 4), sv);
+                        ptx::st_shared_u16(sbuf_u32 + r * stride + dv.x, h);
+                        ptx::st_shared_u16(sbuf_u32 + r * stride + dv.y, h >> 16);
+                    }
                 }
             }
         }
         __syncthreads();  // raw slot consumed, staged rows complete
         if (tid == 0 && issued < mine) issue(issued++);
-        encode_staged(p, sbuf, stride, g * R, rows);
+        encode_staged(p, sbuf_u32, stride, g * R, rows);
         if (g * R <= p.M - 1 && p.M - 1 < g * R + rows) zero_padding_scale_rows(p);
         __syncthreads();  // staged rows free for the next group
     }
@@ -540,38 +576,71 @@ int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* co
     return OSM_OK;
 }
 
+// Per device and kernel, once: raise the dynamic shared-memory limit to
+// what a launch needs and look up CTAs per SM for that size and the SM
+// count, so that a launch costs no driver queries after the first.
+static int prepare_kernel(const void* kern, int threads, size_t smem, int* per_sm_out, int* sms_out) {
+    struct Setup {
+        size_t smem_set = 0;
+        std::map<size_t, int> per_sm;
+    };
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, Setup> cache;
+    static int sms_cache[64] = {};
+    int dev = 0;
+    int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+    if (rc) return rc;
+    if (dev < 0 || dev >= 64) return fail(OSM_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    Setup& su = cache[{kern, dev}];
+    if (smem > 48 * 1024 && su.smem_set < smem) {
+        if ((rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)),
+                             "quantize_act smem attribute")))
+            return rc;
+        su.smem_set = smem;
+    }
+    if (per_sm_out) {
+        auto it = su.per_sm.find(smem);
+        if (it == su.per_sm.end()) {
+            int n = 0;
+            if ((rc = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem),
+                                 "quantize_act occupancy")))
+                return rc;
+            it = su.per_sm.emplace(smem, n).first;
+        }
+        *per_sm_out = it->second;
+    }
+    if (sms_out) {
+        if (!sms_cache[dev] &&
+            (rc = check_cuda(cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev), "SM count")))
+            return rc;
+        *sms_out = sms_cache[dev];
+    }
+    return OSM_OK;
+}
+
 template <int R>
 static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
     auto kern = quantize_act_kernel<R>;
-    if (smem > 48 * 1024) {
-        int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem)),
-                            "quantize_act smem attribute");
-        if (rc) return rc;
-    }
+    int rc = prepare_kernel(reinterpret_cast<const void*>(kern), QA_THREADS, smem, nullptr, nullptr);
+    if (rc) return rc;
     const int64_t grid = ceil_div(p.M, R);
     kern<<<static_cast<unsigned>(grid), QA_THREADS, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
-template <int R, int S>
+template <int R, int S, int NT, int TR>
 static int launch_stream(const QuantParams& p, int stride, cudaStream_t st) {
     const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
-    auto kern = quantize_act_stream_kernel<R, S>;
-    int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem)),
-                        "quantize_act smem attribute");
+    auto kern = quantize_act_stream_kernel<R, S, NT, TR>;
+    int per_sm = 0, sms = 0;
+    int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
     if (rc) return rc;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
-    if ((rc = check_cuda(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count"))) return rc;
-    if ((rc = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QA_THREADS, smem),
-                         "quantize_act occupancy")))
-        return rc;
     if (per_sm < 1) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: no CTA fits");
     const int64_t groups = ceil_div(p.M, R);
     const int64_t grid = groups < static_cast<int64_t>(sms) * per_sm ? groups : static_cast<int64_t>(sms) * per_sm;
-    kern<<<static_cast<unsigned>(grid), QA_THREADS, smem, st>>>(p);
+    kern<<<static_cast<unsigned>(grid), NT, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
@@ -585,9 +654,13 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
     const int stride = qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp));
     // streaming form: two CTAs of at most 110 KB per SM
     const size_t two_per_sm = 110 * 1024;
-    if (stream_smem_bytes<2, 3>(p.K, stride) <= two_per_sm) return launch_stream<2, 3>(p, stride, st);
-    if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3>(p, stride, st);
-    if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2>(p, stride, st);
+    const int npairs = p.K / 2;
+    if (stream_smem_bytes<2, 3>(p.K, stride) <= two_per_sm) {
+        if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, stride, st);
+        return launch_stream<2, 3, STREAM_NT, 0>(p, stride, st);
+    }
+    if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3, STREAM_NT, 0>(p, stride, st);
+    if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2, STREAM_NT, 0>(p, stride, st);
     // very wide rows: the staged, phase-serial form
     const size_t row_bytes = static_cast<size_t>(stride);
     const size_t budget = 72 * 1024;
