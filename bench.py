@@ -568,13 +568,87 @@ def run_ffn(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_refresh(args, cfg, rank, world, local_rank):
+    """Dynamic outlier set: one step re-calibrates the layer on the device
+    from the current batch (activation maxima, osm_plan_refresh) and packs
+    the weights again for the new s and O; inputs resident in HBM."""
+    import torch
+    import outlier_split_mixed_b200 as osm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    M, K, N = cfg.M, cfg.K, cfg.N
+    X, W = cfg.make_x(), cfg.make_w()
+    Xd = torch.from_numpy(X.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+    wmax = torch.empty(K, dtype=torch.float32, device=dev)
+    osm.weight_amax(Wd, wmax)
+    amax = torch.zeros(K, dtype=torch.float32, device=dev)
+    plan = osm.Plan(K, N, cfg.k, np.ones(K, np.float32), np.arange(cfg.k, dtype=np.int32), cfg.wmode)
+    wc, wsc, wh = plan.alloc_packed(N, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        amax.zero_()
+        osm.act_amax_accumulate(Xd, amax)
+        if ev is not None:
+            ev[1].record(stream)
+        plan.refresh(amax, wmax, cfg.alpha)
+        if ev is not None:
+            ev[2].record(stream)
+        osm.pack_weights(plan, Wd, wc, wsc, wh)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    n = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(n):
+            flush.fill_(float(i))
+            step(ev[i])
+        torch.cuda.synchronize()
+    if plan.status() != 0:
+        raise RuntimeError("plan status reports an error")
+    t = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) * 1e-3 for j in range(3)] for i in range(n)]).mean(0)
+    step_s = float(t.sum())
+    if rank == 0:
+        peaks, _ = load_peaks()
+        cb, sb, hb = plan.sizes(N)
+        pack_bytes = K * N * 2 + cb + sb + hb
+        line = {
+            "metric": "dynamic re-calibration time per step (activation maxima + plan refresh + weight repack)",
+            "value": step_s * 1e6, "unit": "us", "n_gpus": world, "steps": n, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in, mxfp4+bf16 out", "data": "synthetic",
+            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)"),
+            "kernels": {
+                "act_amax": {"us": t[0] * 1e6, "gbs": M * K * 2 / t[0] / 1e9},
+                "plan_refresh": {"us": t[1] * 1e6},
+                "pack_weights": {"us": t[2] * 1e6, "gbs": pack_bytes / t[2] / 1e9, "bytes": pack_bytes,
+                                 "frac_hbm": pack_bytes / t[2] / 1e9 / peaks["hbm_gbs"]},
+            },
+            "gpu_launches": 4 * n,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn"], default="up")
+    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn", "refresh"], default="up")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -585,7 +659,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = workloads()[args.workload]
+    cfg = workloads()[args.workload if args.workload != "refresh" else "up"]
 
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)
@@ -600,6 +674,8 @@ def main():
     try:
         if args.workload == "ffn":
             return run_ffn(args, cfg, rank, world, local_rank)
+        if args.workload == "refresh":
+            return run_refresh(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:

@@ -71,6 +71,7 @@ extern "C" {
 
 /* device status bits, returned by osm_plan_status() */
 #define OSM_STATUS_TIMEOUT     1u  /* a pipeline wait of a plan's kernel ran out of time */
+#define OSM_STATUS_NONFINITE   2u  /* osm_plan_refresh saw a non-finite statistic          */
 
 typedef struct osm_plan osm_plan;
 
@@ -193,6 +194,27 @@ OSM_API int osm_pack_weights(const osm_plan* plan, const uint16_t* W, uint8_t* w
  * in the permuted order. */
 OSM_API int osm_pack_weights_for_next(const osm_plan* plan, const osm_plan* next, const uint16_t* W,
                                       uint8_t* w_codes, uint8_t* w_scales, uint16_t* w_hp, void* stream);
+
+/* ---- dynamic outlier set (on-device re-calibration) -----------------------
+ * Eq. (2) and Eq. (4) recomputed on the device from device statistics, so
+ * that the outlier set can follow the activations per batch or per
+ * denoising step (the paper leaves a dynamic set to future work; MixQ keeps
+ * it online). amax, wmax: device float[K], the same statistics
+ * osm_calibrate_finalize takes (osm_act_amax_accumulate, osm_weight_amax).
+ * The plan keeps K, N, k and its weight-scale mode; s, inv_s, O, J and
+ * every routing table are rebuilt in place with osm_calibrate_finalize's
+ * arithmetic (FP64 pow may differ from the host's in the last double bit,
+ * so s can differ by one FP32 ulp in rare cases; O is exact). Stream-
+ * ordered, no host synchronisation. Afterwards the weights must be packed
+ * again (osm_pack_weights): s is folded into them and J has changed; data
+ * packed for the old plan must not be used with the new one. A non-finite
+ * statistic sets OSM_STATUS_NONFINITE and leaves the plan unchanged.
+ * alpha in (0, 1). */
+OSM_API int osm_plan_refresh(osm_plan* plan, const float* amax, const float* wmax, float alpha, void* stream);
+
+/* Copies of the plan's s, inv_s (float[K]) and O (int32[k], ascending) to
+ * host memory; any pointer may be NULL. Synchronous. */
+OSM_API int osm_plan_tables(const osm_plan* plan, float* s_host, float* inv_s_host, int32_t* O_host);
 
 /* ---- runtime activation path ----------------------------------------------
  * "activations are divided in-place by s, quantized ..., and routed through

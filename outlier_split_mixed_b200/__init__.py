@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libosm.so")
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
 STATUS_TIMEOUT = 1
+STATUS_NONFINITE = 2
 DEBUG_STARVE_QUANTIZE = 1
 WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
 EPI_F32, EPI_BF16, EPI_GELU_REQUANT, EPI_GELU_BF16 = 0, 1, 2, 3
@@ -42,6 +43,8 @@ _SIGNATURES = {
     "osm_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _I]),
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
     "osm_plan_set_debug": (_I, [_P, ctypes.c_uint32]),
+    "osm_plan_refresh": (_I, [_P, _P, _P, ctypes.c_float, _P]),
+    "osm_plan_tables": (_I, [_P, _P, _P, _P]),
     "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
     "osm_pack_weights_for_next": (_I, [_P, _P, _P, _P, _P, _P, _P]),
     "osm_plan_channel_order": (_I, [_P, _P]),
@@ -178,6 +181,22 @@ class Plan:
 
     def set_debug(self, flags: int):
         _check(lib().osm_plan_set_debug(self._h, int(flags)))
+
+    def refresh(self, amax, wmax, alpha: float, stream=None):
+        """Re-calibrate on the device from device statistics (osm_plan_refresh):
+        s, inv_s, O and the routing tables are rebuilt; pack the weights again."""
+        import torch
+        _check(lib().osm_plan_refresh(self._h, _ptr(amax, "amax", (torch.float32,), self.K * 4),
+                                      _ptr(wmax, "wmax", (torch.float32,), self.K * 4), float(alpha),
+                                      _stream(stream)))
+
+    def tables(self):
+        """(s, inv_s, O) copied to host numpy arrays (osm_plan_tables)."""
+        s = np.empty(self.K, np.float32)
+        inv_s = np.empty(self.K, np.float32)
+        O = np.empty(max(self.k, 1), np.int32)
+        _check(lib().osm_plan_tables(self._h, _host_ptr(s), _host_ptr(inv_s), _host_ptr(O)))
+        return s, inv_s, O[:self.k].copy()
 
     def alloc_packed(self, rows: int, device="cuda"):
         """Allocate (codes, scales, hp) torch buffers for `rows` rows."""

@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libosm.so")
 
-SOURCES = ["osm_api.cu", "osm_quant.cu", "osm_gemm.cu", "osm_noalloc.cu"]
+SOURCES = ["osm_api.cu", "osm_quant.cu", "osm_gemm.cu", "osm_noalloc.cu", "osm_refresh.cu"]
 HEADERS = ["osm_internal.h", "osm_ptx.cuh", "osm_mx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -315,6 +315,28 @@ int osm_plan_channel_order(const osm_plan* p, int32_t* order_host) {
                       "plan_channel_order: read");
 }
 
+int osm_plan_refresh(osm_plan* p, const float* amax, const float* wmax, float alpha, void* stream) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(p));
+    OSM_REQUIRE(amax && wmax && (reinterpret_cast<uintptr_t>(amax) & 3) == 0 &&
+                    (reinterpret_cast<uintptr_t>(wmax) & 3) == 0,
+                "plan_refresh: amax / wmax null or misaligned");
+    OSM_REQUIRE(alpha > 0.0f && alpha < 1.0f, "plan_refresh: alpha must lie in (0, 1)");
+    return launch_plan_refresh(p, amax, wmax, alpha, static_cast<cudaStream_t>(stream));
+}
+
+int osm_plan_tables(const osm_plan* p, float* s_host, float* inv_s_host, int32_t* O_host) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(p));
+    cudaError_t e = cudaSuccess;
+    if (s_host) e = cudaMemcpy(s_host, p->d_s, sizeof(float) * p->K, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && inv_s_host)
+        e = cudaMemcpy(inv_s_host, p->d_inv_s, sizeof(float) * p->K, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && O_host && p->k > 0)
+        e = cudaMemcpy(O_host, p->d_O, sizeof(int32_t) * p->k, cudaMemcpyDeviceToHost);
+    return check_cuda(e, "plan_tables: read");
+}
+
 int osm_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* a_codes, uint8_t* a_scales,
                      uint16_t* a_hp, void* stream) {
     g_err[0] = 0;

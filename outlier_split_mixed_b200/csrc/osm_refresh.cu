@@ -1,0 +1,185 @@
+// On-device plan refresh: the calibration of "W4A4 Quantization for
+// Inference on Wan2.2-I2V-A14B" (Eq. (2) smoothing vector, Eq. (4) top-k
+// outlier set) recomputed from device-resident statistics, and every plan
+// table derived from it rebuilt in place, so that a new outlier set can be
+// adopted per batch or per denoising step without a host round trip. The
+// arithmetic is that of osm_calibrate_finalize followed by osm_plan_create.
+//
+// One CTA of 1024 threads (K <= 65536):
+//  1. any non-finite statistic -> OSM_STATUS_NONFINITE, tables untouched;
+//  2. s_j = fp32(max(amax_j,1e-5)^alpha / max(wmax_j,1e-5)^(1-alpha)) in
+//     FP64, inv_s_j = 1.0f / s_j;
+//  3. O = the k channels with the largest key (amax, mapped to an unsigned
+//     integer of the same order, << 16 | 0xFFFF - j): keys are unique, and
+//     their order is amax descending, then channel index ascending.
+//     The k-th largest key is found by a radix select over the 48 key bits,
+//     8 bits per pass, with a shared 256-bin histogram;
+//  4. J (unselected, ascending) and O (selected, ascending) by block-wide
+//     ballot scans over chunks of 1024 channels; route, order and
+//     inv_s in that order follow from each channel's rank.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "osm_internal.h"
+
+namespace osm {
+namespace {
+
+constexpr int RF_THREADS = 1024;
+
+struct RefreshParams {
+    const float* amax;
+    const float* wmax;
+    double alpha;
+    int K, k, Kb, Kbp;
+    float* s;
+    float* inv_s;
+    int32_t* route;
+    int32_t* J;
+    int32_t* O;
+    int32_t* order;
+    float* inv_s_ord;
+    uint32_t* status;
+};
+
+// 48-bit key: the statistic mapped to an unsigned integer of the same order
+// (-0 taken as +0, so that equal values tie), then 0xFFFF - j.
+__device__ __forceinline__ uint64_t rf_key(const float* amax, int j) {
+    uint32_t u = __float_as_uint(amax[j]);
+    if (u == 0x80000000u) u = 0u;
+    u ^= (u >> 31) ? 0xFFFFFFFFu : 0x80000000u;
+    return (static_cast<uint64_t>(u) << 16) | static_cast<uint64_t>(0xFFFF - j);
+}
+
+// Exclusive prefix of `flag` over the CTA (thread order), and the total.
+__device__ __forceinline__ int block_exclusive_scan(int flag, int* warp_tot, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned b = __ballot_sync(0xffffffffu, flag);
+    const int in_warp = __popc(b & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(b);
+    __syncthreads();
+    if (warp == 0) {
+        const int v = warp_tot[lane];
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        warp_tot[lane] = incl - v;  // exclusive
+        if (lane == 31) *total = incl;
+    }
+    __syncthreads();
+    const int r = warp_tot[warp] + in_warp;
+    __syncthreads();  // warp_tot is reused by the next call
+    return r;
+}
+
+__global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams p) {
+    __shared__ int bad;
+    __shared__ unsigned hist[256];
+    __shared__ int warp_tot[32];
+    __shared__ int total;
+    __shared__ uint64_t prefix_sh;
+    __shared__ int need_sh;
+    const int tid = threadIdx.x;
+
+    // 1. statistics must be finite
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    for (int j = tid; j < p.K; j += RF_THREADS)
+        if (!isfinite(p.amax[j]) || !isfinite(p.wmax[j])) bad = 1;
+    __syncthreads();
+    if (bad) {
+        if (tid == 0) atomicOr(p.status, OSM_STATUS_NONFINITE);
+        return;
+    }
+
+    // 2. Eq. (2)
+    for (int j = tid; j < p.K; j += RF_THREADS) {
+        const double am = fmax(static_cast<double>(p.amax[j]), 1e-5);
+        const double wm = fmax(static_cast<double>(p.wmax[j]), 1e-5);
+        const float s = static_cast<float>(pow(am, p.alpha) / pow(wm, 1.0 - p.alpha));
+        p.s[j] = s;
+        p.inv_s[j] = __fdiv_rn(1.0f, s);
+    }
+
+    // 3. the k-th largest key (k = 0: none selected; k = K: all)
+    uint64_t thresh = 0;  // selected <=> key >= thresh
+    if (p.k == 0) {
+        thresh = ~0ull;
+    } else if (p.k < p.K) {
+        if (tid == 0) {
+            prefix_sh = 0;
+            need_sh = p.k;
+        }
+        __syncthreads();
+        for (int shift = 40; shift >= 0; shift -= 8) {
+            for (int b = tid; b < 256; b += RF_THREADS) hist[b] = 0;
+            __syncthreads();
+            const uint64_t prefix = prefix_sh;
+            const uint64_t hi_mask = shift == 40 ? 0ull : (~0ull << (shift + 8)) & 0xFFFFFFFFFFFFull;
+            for (int j = tid; j < p.K; j += RF_THREADS) {
+                const uint64_t key = rf_key(p.amax, j);
+                if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int need = need_sh;
+                int d = 255;
+                for (; d > 0; --d) {
+                    if (static_cast<int>(hist[d]) >= need) break;
+                    need -= static_cast<int>(hist[d]);
+                }
+                prefix_sh = prefix | (static_cast<uint64_t>(d) << shift);
+                need_sh = need;
+            }
+            __syncthreads();
+        }
+        thresh = prefix_sh;  // exact: keys are unique, so the k-th largest is one key
+    }
+
+    // 4. ranks, J, O, route, order, inv_s in order
+    __syncthreads();
+    const int nbp = p.Kbp / 32;
+    int base_o = 0, base_j = 0;
+    for (int c0 = 0; c0 < p.K; c0 += RF_THREADS) {
+        const int j = c0 + tid;
+        const bool valid = j < p.K;
+        const int sel = valid && rf_key(p.amax, valid ? j : 0) >= thresh ? 1 : 0;
+        const int r_o = block_exclusive_scan(sel, warp_tot, &total) + base_o;
+        const int n_sel = total;
+        const int r_j = base_j + tid - (r_o - base_o);  // unselected channels before j
+        if (valid) {
+            const float iv = p.inv_s[j];
+            if (sel) {
+                p.O[r_o] = j;
+                p.route[j] = nbp * QA_BLOCK_BYTES + 2 * r_o;
+                p.order[p.Kb + r_o] = j;
+                p.inv_s_ord[p.Kb + r_o] = iv;
+            } else {
+                p.J[r_j] = j;
+                p.route[j] = (r_j / 32) * QA_BLOCK_BYTES + (r_j % 32) * 2;
+                p.order[r_j] = j;
+                p.inv_s_ord[r_j] = iv;
+            }
+        }
+        base_o += n_sel;
+        base_j += min(RF_THREADS, p.K - c0) - n_sel;
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+int launch_plan_refresh(osm_plan* pl, const float* amax, const float* wmax, float alpha, cudaStream_t st) {
+    RefreshParams p{amax, wmax, static_cast<double>(alpha), static_cast<int>(pl->K), static_cast<int>(pl->k),
+                    static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp), pl->d_s, pl->d_inv_s, pl->d_route,
+                    pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status};
+    plan_refresh_kernel<<<1, RF_THREADS, 0, st>>>(p);
+    return check_cuda(cudaGetLastError(), "plan_refresh launch");
+}
+
+}  // namespace osm
