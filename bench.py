@@ -652,6 +652,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (small cases for profiler captures)")
+    ap.add_argument("--blocks", type=int, default=0, help="override the number of FFN blocks (ffn workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -660,6 +663,15 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = workloads()[args.workload if args.workload != "refresh" else "up"]
+    if args.tokens or args.blocks:
+        import dataclasses
+        changes = {}
+        if args.tokens:
+            changes["M"] = args.tokens
+        if args.blocks and hasattr(cfg, "layers"):
+            changes["layers"] = args.blocks
+        changes["name"] = cfg.name + "".join(f"_{k}{v}" for k, v in sorted(changes.items()))
+        cfg = dataclasses.replace(cfg, **changes)
 
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)

@@ -63,30 +63,48 @@ __device__ __forceinline__ uint32_t smooth2(uint32_t w, float2 s) {
 
 // ------------------------------------------------------------ calibration
 
-constexpr int AMAX_ROWS = 64;
+constexpr int AMAX_ROWS = 32;
 
 // amax[j] = max(amax[j], max_t |X[t][j]|). One thread per 8 channels and
-// AMAX_ROWS rows; the per-thread maxima are merged with atomicMax on the
-// IEEE bit pattern (monotone for non-negative floats).
+// AMAX_ROWS rows, eight 16-byte row loads in flight; the maxima are kept as
+// packed u16 pairs of |x| bit patterns (integer order, so a NaN pattern
+// propagates and the finiteness check of the calibration sees it) and
+// merged with atomicMax on the IEEE bit pattern of the FP32 value
+// (monotone for non-negative floats).
 __global__ void __launch_bounds__(128) act_amax_kernel(const uint16_t* __restrict__ X, int64_t T,
                                                        int64_t K, float* __restrict__ amax) {
     const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (v * 8 >= K) return;
     const int64_t t0 = static_cast<int64_t>(blockIdx.y) * AMAX_ROWS;
     const int64_t t1 = min(T, t0 + AMAX_ROWS);
-    uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // |x| bit patterns (bf16 << 16)
-    for (int64_t t = t0; t < t1; ++t) {
-        const uint4 q = ldg_nc_v4(X + t * K + v * 8);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t m[4] = {0, 0, 0, 0};
+    const uint16_t* src = X + v * 8;
+    int64_t t = t0;
+    for (; t + 8 <= t1; t += 8) {
+        uint4 q[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            m[2 * i] = max(m[2 * i], (w[i] & 0x7FFFu) << 16);
-            m[2 * i + 1] = max(m[2 * i + 1], (w[i] >> 16 & 0x7FFFu) << 16);
+        for (int u = 0; u < 8; ++u) q[u] = ldg_nc_v4(src + (t + u) * K);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            m[0] = vmax_u16x2(m[0], q[u].x & 0x7FFF7FFFu);
+            m[1] = vmax_u16x2(m[1], q[u].y & 0x7FFF7FFFu);
+            m[2] = vmax_u16x2(m[2], q[u].z & 0x7FFF7FFFu);
+            m[3] = vmax_u16x2(m[3], q[u].w & 0x7FFF7FFFu);
         }
+    }
+    for (; t < t1; ++t) {
+        const uint4 q = ldg_nc_v4(src + t * K);
+        m[0] = vmax_u16x2(m[0], q.x & 0x7FFF7FFFu);
+        m[1] = vmax_u16x2(m[1], q.y & 0x7FFF7FFFu);
+        m[2] = vmax_u16x2(m[2], q.z & 0x7FFF7FFFu);
+        m[3] = vmax_u16x2(m[3], q.w & 0x7FFF7FFFu);
     }
     unsigned int* dst = reinterpret_cast<unsigned int*>(amax) + v * 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) atomicMax(dst + i, m[i]);
+    for (int i = 0; i < 4; ++i) {
+        atomicMax(dst + 2 * i, (m[i] & 0xFFFFu) << 16);
+        atomicMax(dst + 2 * i + 1, m[i] & 0xFFFF0000u);
+    }
 }
 
 // wmax[j] = max_n |W[j][n]|: one block per input channel row.
@@ -128,74 +146,140 @@ struct PackParams {
     uint16_t* hp;       // [N][kp]
 };
 
-// One thread per (output channel n, 128-wide bulk strip). Threads of a warp
-// take 32 consecutive n, so every W row read is a coalesced 64-byte segment
-// and a 32x32 tile is exactly one warp.
-__global__ void __launch_bounds__(256) pack_bulk_kernel(PackParams p) {
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.x;
-    const int64_t strip = static_cast<int64_t>(blockIdx.y) * 8 + threadIdx.y;
-    const int64_t katoms = p.Kbp / 128;
-    if (strip >= katoms) return;  // uniform per warp
-    const bool nvalid = n < p.N;
-    uint32_t h[64];  // 128 folded BF16 weights, two per word
-    float am[4] = {0.f, 0.f, 0.f, 0.f};
+// Tiled forms of the two packing kernels: a CTA gathers whole W rows (input
+// channels) with coalesced 16-byte loads, folds s and rounds to BF16 on the
+// way into shared memory, and reads the tile back transposed, so that every
+// global access is wide and contiguous whatever the packing order.
+
+constexpr int PK_THREADS = 256;
+
+// Load rows src_row(r) of W (r < nrows; a negative row is zero), columns
+// n0 .. n0+127 (packed order: W column col_order[n] when col_order is set),
+// as w' = bf16(fp32(w) * s[row]) into tile[r][0..63] (BF16 pairs).
+template <typename RowOf>
+__device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0, int nrows, RowOf src_row,
+                                                 uint32_t (*tile)[64]) {
+    for (int t = threadIdx.x; t < nrows * 16; t += PK_THREADS) {
+        const int r = t >> 4, c = t & 15;
+        const int64_t j = src_row(r);
+        const int64_t n = n0 + 8 * c;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j >= 0 && n < p.N) {
+            const float sj = __ldg(p.s + j);
+            const float2 s2 = make_float2(sj, sj);
+            uint4 w;
+            if (p.col_order == nullptr) {
+                w = ldg_nc_v4(p.W + j * p.N + n);
+            } else {
+                uint32_t e[8];
 #pragma unroll
-    for (int i = 0; i < 128; ++i) {
-        const int64_t pos = strip * 128 + i;
-        uint32_t bits = 0;
-        if (nvalid && pos < p.Kb) {
-            const int32_t j = __ldg(p.J + pos);
-            const int64_t src = p.col_order ? __ldg(p.col_order + n) : n;
-            const float w = bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + src]);
-            bits = f32_to_bf16_bits(w * __ldg(p.s + j));
+                for (int i = 0; i < 8; ++i) e[i] = p.W[j * p.N + __ldg(p.col_order + n + i)];
+                w = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+            }
+            v = make_uint4(smooth2(w.x, s2), smooth2(w.y, s2), smooth2(w.z, s2), smooth2(w.w, s2));
         }
-        if (i & 1) h[i >> 1] |= bits << 16; else h[i >> 1] = bits;
-        am[i >> 5] = fmaxf(am[i >> 5], bf16_bits_to_f32(bits & 0x7FFFu));
-    }
-    if (p.mode == OSM_WSCALE_STRIP128x1) {
-        const float m = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-        am[0] = am[1] = am[2] = am[3] = m;
-    } else if (p.mode == OSM_WSCALE_TILE32x32) {
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-#pragma unroll
-            for (int o = 16; o; o >>= 1) am[b] = fmaxf(am[b], __shfl_xor_sync(0xffffffffu, am[b], o));
-    }
-    uint32_t sc = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const int X = mx_exponent(am[b]);
-        const int64_t pos0 = strip * 128 + b * 32;
-        const uint32_t code = (nvalid && pos0 < p.Kb) ? static_cast<uint32_t>(X + 127) : 0u;
-        sc |= code << (8 * b);
-        if (nvalid) {
-            const float inv = exp2_neg(X);
-            uint4 out;
-            out.x = encode8_words(make_uint4(h[16 * b + 0], h[16 * b + 1], h[16 * b + 2], h[16 * b + 3]), inv);
-            out.y = encode8_words(make_uint4(h[16 * b + 4], h[16 * b + 5], h[16 * b + 6], h[16 * b + 7]), inv);
-            out.z = encode8_words(make_uint4(h[16 * b + 8], h[16 * b + 9], h[16 * b + 10], h[16 * b + 11]), inv);
-            out.w = encode8_words(make_uint4(h[16 * b + 12], h[16 * b + 13], h[16 * b + 14], h[16 * b + 15]), inv);
-            *reinterpret_cast<uint4*>(p.codes + n * (p.Kbp / 2) + strip * 64 + b * 16) = out;
-        }
-    }
-    // four scales of this strip are contiguous bytes of one atom row
-    if (n < (p.N + 127) / 128 * 128) {
-        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, strip * 4, katoms)) = sc;
+        *reinterpret_cast<uint4*>(&tile[r][4 * c]) = v;
     }
 }
 
-// w_hp[n][i] = bf16(w[O_i][n] * s[O_i]) for i < k, zero for k <= i < kp.
-__global__ void __launch_bounds__(256) pack_hp_kernel(PackParams p) {
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.x;
-    const int64_t i = static_cast<int64_t>(blockIdx.y) * 8 + threadIdx.y;
-    if (n >= p.N || i >= p.kp) return;
-    uint32_t bits = 0;
-    if (i < p.k) {
-        const int32_t j = p.O[i];
-        const int64_t src = p.col_order ? p.col_order[n] : n;
-        bits = f32_to_bf16_bits(bf16_bits_to_f32(p.W[static_cast<int64_t>(j) * p.N + src]) * p.s[j]);
+// Bulk channels: CTA = 128 bulk positions (one strip, four MX blocks) x 128
+// packed output channels. Warp w encodes block q = w / 2 for the 64 channel
+// pairs 32 (w % 2) + lane: its 32 words are (channel n, channel n + 1) pairs
+// down the block, so one packed abs-max chain gives both channels' block
+// maxima. 1x32: the block maximum; 32x32: the maximum over 32 channels (16
+// lanes); 128x1: the maximum over the strip's four blocks (four warps, via
+// shared memory). Codes and scales as in pack_bulk_kernel.
+__global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams p) {
+    __shared__ __align__(16) uint32_t tile[128][64];
+    __shared__ uint32_t red[4][64];
+    __shared__ uint32_t sxs[4][64];  // exponent codes, (lo | hi << 8) per quarter and pair
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
+    const int64_t p0 = static_cast<int64_t>(blockIdx.y) * 128;
+    const int64_t katoms = p.Kbp / 128;
+    load_folded_rows(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; }, tile);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp >> 1;
+    const int c = 32 * (warp & 1) + lane;  // channel pair: columns n0 + 2c, n0 + 2c + 1
+    uint32_t wv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) wv[i] = tile[32 * q + i][c];
+    using mx::bf16x2_absmax;
+    uint32_t m = wv[0];
+#pragma unroll
+    for (int i = 1; i < 32; ++i) m = bf16x2_absmax(m, wv[i]);
+    if (p.mode == OSM_WSCALE_TILE32x32) {
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) m = bf16x2_absmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const uint32_t mm = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
+        m = mm | (mm << 16);
+    } else if (p.mode == OSM_WSCALE_STRIP128x1) {
+        red[q][c] = m;
+        __syncthreads();
+        m = bf16x2_absmax(bf16x2_absmax(red[0][c], red[1][c]), bf16x2_absmax(red[2][c], red[3][c]));
     }
-    p.hp[n * p.kp + i] = static_cast<uint16_t>(bits);
+    const bool real = p0 + 32 * q < p.Kb;  // the block holds at least one real position
+    float inv_lo, inv_hi;
+    const int X_lo = mx::bf16_block_exponent(m & 0x7FFFu, &inv_lo);
+    const int X_hi = mx::bf16_block_exponent((m >> 16) & 0x7FFFu, &inv_hi);
+    const int64_t n = n0 + 2 * c;
+    if (n < p.N) {
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int k2 = 0; k2 < 16; ++k2) {
+            lo[k2] = __byte_perm(wv[2 * k2], wv[2 * k2 + 1], 0x5410);
+            hi[k2] = __byte_perm(wv[2 * k2], wv[2 * k2 + 1], 0x7632);
+        }
+        const uint4 clo = make_uint4(mx::encode8_words(lo[0], lo[1], lo[2], lo[3], inv_lo),
+                                     mx::encode8_words(lo[4], lo[5], lo[6], lo[7], inv_lo),
+                                     mx::encode8_words(lo[8], lo[9], lo[10], lo[11], inv_lo),
+                                     mx::encode8_words(lo[12], lo[13], lo[14], lo[15], inv_lo));
+        const uint4 chi = make_uint4(mx::encode8_words(hi[0], hi[1], hi[2], hi[3], inv_hi),
+                                     mx::encode8_words(hi[4], hi[5], hi[6], hi[7], inv_hi),
+                                     mx::encode8_words(hi[8], hi[9], hi[10], hi[11], inv_hi),
+                                     mx::encode8_words(hi[12], hi[13], hi[14], hi[15], inv_hi));
+        *reinterpret_cast<uint4*>(p.codes + n * (p.Kbp / 2) + p0 / 2 + 16 * q) = clo;
+        *reinterpret_cast<uint4*>(p.codes + (n + 1) * (p.Kbp / 2) + p0 / 2 + 16 * q) = chi;
+    }
+    sxs[q][c] = real ? static_cast<uint32_t>(X_lo + 127) | (static_cast<uint32_t>(X_hi + 127) << 8) : 0u;
+    __syncthreads();
+    if (warp < 2) {  // the four scale bytes of a channel are one word of its atom row; padding rows get 0
+        uint32_t wlo = 0, whi = 0;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            wlo |= (sxs[qq][c] & 0xFFu) << (8 * qq);
+            whi |= ((sxs[qq][c] >> 8) & 0xFFu) << (8 * qq);
+        }
+        if (n >= p.N) wlo = 0;
+        if (n + 1 >= p.N) whi = 0;
+        const int64_t strip = blockIdx.y;
+        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, strip * 4, katoms)) = wlo;
+        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n + 1, strip * 4, katoms)) = whi;
+    }
+}
+
+// Outlier channels: CTA = 64 outlier slots x 128 packed output channels;
+// w_hp[n][i] = bf16(fp32(w[O_i][n]) * s[O_i]) for i < k, 0 for k <= i < kp.
+// Thread (n, 8-slot group) gathers its eight values down the tile and writes
+// them as one 16-byte store.
+__global__ void __launch_bounds__(PK_THREADS) pack_hp_tiled_kernel(PackParams p) {
+    __shared__ __align__(16) uint32_t tile[64][64];
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
+    const int64_t i0 = static_cast<int64_t>(blockIdx.y) * 64;
+    load_folded_rows(p, n0, 64, [&](int r) -> int64_t { return i0 + r < p.k ? __ldg(p.O + i0 + r) : -1; }, tile);
+    __syncthreads();
+    const uint16_t* t16 = reinterpret_cast<const uint16_t*>(&tile[0][0]);
+    for (int t = threadIdx.x; t < 128 * 8; t += PK_THREADS) {
+        const int nl = t & 127, g = t >> 7;  // channel, group of 8 slots
+        const int64_t n = n0 + nl;
+        if (n >= p.N) continue;
+        uint32_t e[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = t16[(8 * g + i) * 128 + nl];
+        *reinterpret_cast<uint4*>(p.hp + n * p.kp + i0 + 8 * g) =
+            make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+    }
 }
 
 // ------------------------------------------------------------ quantize_act
@@ -562,15 +646,14 @@ int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* co
     PackParams p{W, col_order, pl->d_s, pl->d_J, pl->d_O, pl->K, pl->N, pl->k, pl->Kb, pl->Kbp, pl->kp,
                  pl->wmode, codes, scales, hp};
     if (pl->Kbp > 0) {
-        dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 32),
-                  static_cast<unsigned>(ceil_div(pl->Kbp / 128, 8)));
-        pack_bulk_kernel<<<grid, dim3(32, 8), 0, st>>>(p);
+        dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 128), static_cast<unsigned>(pl->Kbp / 128));
+        pack_bulk_tiled_kernel<<<grid, PK_THREADS, 0, st>>>(p);
         int rc = check_cuda(cudaGetLastError(), "pack_bulk launch");
         if (rc) return rc;
     }
     if (pl->kp > 0) {
-        dim3 grid(static_cast<unsigned>(ceil_div(pl->N, 32)), static_cast<unsigned>(ceil_div(pl->kp, 8)));
-        pack_hp_kernel<<<grid, dim3(32, 8), 0, st>>>(p);
+        dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 128), static_cast<unsigned>(pl->kp / 64));
+        pack_hp_tiled_kernel<<<grid, PK_THREADS, 0, st>>>(p);
         return check_cuda(cudaGetLastError(), "pack_hp launch");
     }
     return OSM_OK;

@@ -5,15 +5,18 @@
 // adopted per batch or per denoising step without a host round trip. The
 // arithmetic is that of osm_calibrate_finalize followed by osm_plan_create.
 //
-// One CTA of 1024 threads (K <= 65536):
-//  1. any non-finite statistic -> OSM_STATUS_NONFINITE, tables untouched;
-//  2. s_j = fp32(max(amax_j,1e-5)^alpha / max(wmax_j,1e-5)^(1-alpha)) in
-//     FP64, inv_s_j = 1.0f / s_j;
+// Kernel 1 (one thread per channel): s_j = fp32(max(amax_j,1e-5)^alpha /
+// max(wmax_j,1e-5)^(1-alpha)) in FP64 and inv_s_j = 1.0f / s_j into plan
+// scratch, and a flag if any statistic is not finite.
+// Kernel 2, one CTA of 1024 threads (K <= 65536):
+//  1. flag set -> OSM_STATUS_NONFINITE, every table untouched;
+//  2. s, inv_s adopted from scratch;
 //  3. O = the k channels with the largest key (amax, mapped to an unsigned
 //     integer of the same order, << 16 | 0xFFFF - j): keys are unique, and
 //     their order is amax descending, then channel index ascending.
 //     The k-th largest key is found by a radix select over the 48 key bits,
-//     8 bits per pass, with a shared 256-bin histogram;
+//     8 bits per pass: a shared 256-bin histogram (one increment per
+//     distinct digit of a warp) and a warp-parallel search from the top;
 //  4. J (unselected, ascending) and O (selected, ascending) by block-wide
 //     ballot scans over chunks of 1024 channels; route, order and
 //     inv_s in that order follow from each channel's rank.
@@ -34,6 +37,8 @@ struct RefreshParams {
     const float* wmax;
     double alpha;
     int K, k, Kb, Kbp;
+    const float* s_new;    // [2K]: s, then inv_s
+    const uint32_t* bad;
     float* s;
     float* inv_s;
     int32_t* route;
@@ -44,12 +49,20 @@ struct RefreshParams {
     uint32_t* status;
 };
 
-// 48-bit key: the statistic mapped to an unsigned integer of the same order
-// (-0 taken as +0, so that equal values tie), then 0xFFFF - j.
-__device__ __forceinline__ uint64_t rf_key(const float* amax, int j) {
-    uint32_t u = __float_as_uint(amax[j]);
+constexpr int RF_SMEM_KEYS = 32768;  // statistics staged in shared memory (128 KB)
+
+// The statistic mapped to an unsigned integer of the same order (-0 taken
+// as +0, so that equal values tie).
+__device__ __forceinline__ uint32_t rf_ord(float a) {
+    uint32_t u = __float_as_uint(a);
     if (u == 0x80000000u) u = 0u;
-    u ^= (u >> 31) ? 0xFFFFFFFFu : 0x80000000u;
+    return u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);
+}
+
+// 48-bit key of channel j: its ordered statistic, then 0xFFFF - j. `sk`
+// holds the ordered statistics of channels below RF_SMEM_KEYS.
+__device__ __forceinline__ uint64_t rf_key(const uint32_t* sk, const float* amax, int j) {
+    const uint32_t u = j < RF_SMEM_KEYS ? sk[j] : rf_ord(amax[j]);
     return (static_cast<uint64_t>(u) << 16) | static_cast<uint64_t>(0xFFFF - j);
 }
 
@@ -77,8 +90,25 @@ __device__ __forceinline__ int block_exclusive_scan(int flag, int* warp_tot, int
     return r;
 }
 
+__global__ void __launch_bounds__(256) refresh_smooth_kernel(const float* __restrict__ amax,
+                                                             const float* __restrict__ wmax, double alpha, int K,
+                                                             float* __restrict__ s_new, uint32_t* __restrict__ bad) {
+    const int j = blockIdx.x * 256 + threadIdx.x;
+    if (j >= K) return;
+    const float a = amax[j], w = wmax[j];
+    if (!isfinite(a) || !isfinite(w)) {
+        atomicOr(bad, 1u);
+        return;
+    }
+    const double am = fmax(static_cast<double>(a), 1e-5);
+    const double wm = fmax(static_cast<double>(w), 1e-5);
+    const float s = static_cast<float>(pow(am, alpha) / pow(wm, 1.0 - alpha));
+    s_new[j] = s;
+    s_new[K + j] = __fdiv_rn(1.0f, s);
+}
+
 __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams p) {
-    __shared__ int bad;
+    extern __shared__ uint32_t sk[];  // ordered statistics of the first min(K, RF_SMEM_KEYS) channels
     __shared__ unsigned hist[256];
     __shared__ int warp_tot[32];
     __shared__ int total;
@@ -87,24 +117,18 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     const int tid = threadIdx.x;
 
     // 1. statistics must be finite
-    if (tid == 0) bad = 0;
-    __syncthreads();
-    for (int j = tid; j < p.K; j += RF_THREADS)
-        if (!isfinite(p.amax[j]) || !isfinite(p.wmax[j])) bad = 1;
-    __syncthreads();
-    if (bad) {
+    if (*p.bad) {
         if (tid == 0) atomicOr(p.status, OSM_STATUS_NONFINITE);
         return;
     }
 
-    // 2. Eq. (2)
+    // 2. Eq. (2), computed by refresh_smooth_kernel; stage the keys
     for (int j = tid; j < p.K; j += RF_THREADS) {
-        const double am = fmax(static_cast<double>(p.amax[j]), 1e-5);
-        const double wm = fmax(static_cast<double>(p.wmax[j]), 1e-5);
-        const float s = static_cast<float>(pow(am, p.alpha) / pow(wm, 1.0 - p.alpha));
-        p.s[j] = s;
-        p.inv_s[j] = __fdiv_rn(1.0f, s);
+        p.s[j] = p.s_new[j];
+        p.inv_s[j] = p.s_new[p.K + j];
+        if (j < RF_SMEM_KEYS) sk[j] = rf_ord(p.amax[j]);
     }
+    __syncthreads();
 
     // 3. the k-th largest key (k = 0: none selected; k = K: all)
     uint64_t thresh = 0;  // selected <=> key >= thresh
@@ -121,20 +145,42 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
             __syncthreads();
             const uint64_t prefix = prefix_sh;
             const uint64_t hi_mask = shift == 40 ? 0ull : (~0ull << (shift + 8)) & 0xFFFFFFFFFFFFull;
-            for (int j = tid; j < p.K; j += RF_THREADS) {
-                const uint64_t key = rf_key(p.amax, j);
-                if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
+            for (int j0 = 0; j0 < p.K; j0 += RF_THREADS) {  // uniform trip count: whole warps stay converged
+                const int j = j0 + tid;
+                const uint64_t key = j < p.K ? rf_key(sk, p.amax, j) : 0;
+                const bool in = j < p.K && (key & hi_mask) == prefix;
+                const unsigned digit = in ? static_cast<unsigned>((key >> shift) & 0xFF) : 256u;
+                // one shared-memory increment per distinct digit of the warp
+                const unsigned peers = __match_any_sync(0xffffffffu, digit);
+                if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
             }
             __syncthreads();
-            if (tid == 0) {
-                int need = need_sh;
-                int d = 255;
-                for (; d > 0; --d) {
-                    if (static_cast<int>(hist[d]) >= need) break;
-                    need -= static_cast<int>(hist[d]);
+            if (tid < 32) {
+                // lane l owns digits 255 - 8l .. 248 - 8l; a prefix sum over lanes
+                // runs from the top digit down
+                const int lane = tid;
+                int own = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) own += static_cast<int>(hist[255 - 8 * lane - i]);
+                int incl = own;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += o;
                 }
-                prefix_sh = prefix | (static_cast<uint64_t>(d) << shift);
-                need_sh = need;
+                const int need = need_sh;
+                const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+                const int l = __ffs(hit) - 1;  // first lane whose digits reach the k-th key
+                if (lane == l) {
+                    int rem = need - (incl - own);
+                    int d = 255 - 8 * lane;
+                    for (int i = 0; i < 7; ++i, --d) {
+                        if (static_cast<int>(hist[d]) >= rem) break;
+                        rem -= static_cast<int>(hist[d]);
+                    }
+                    prefix_sh = prefix | (static_cast<uint64_t>(d) << shift);
+                    need_sh = rem;
+                }
             }
             __syncthreads();
         }
@@ -148,7 +194,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     for (int c0 = 0; c0 < p.K; c0 += RF_THREADS) {
         const int j = c0 + tid;
         const bool valid = j < p.K;
-        const int sel = valid && rf_key(p.amax, valid ? j : 0) >= thresh ? 1 : 0;
+        const int sel = valid && rf_key(sk, p.amax, valid ? j : 0) >= thresh ? 1 : 0;
         const int r_o = block_exclusive_scan(sel, warp_tot, &total) + base_o;
         const int n_sel = total;
         const int r_j = base_j + tid - (r_o - base_o);  // unselected channels before j
@@ -175,10 +221,27 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
 }  // namespace
 
 int launch_plan_refresh(osm_plan* pl, const float* amax, const float* wmax, float alpha, cudaStream_t st) {
-    RefreshParams p{amax, wmax, static_cast<double>(alpha), static_cast<int>(pl->K), static_cast<int>(pl->k),
-                    static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp), pl->d_s, pl->d_inv_s, pl->d_route,
+    const int K = static_cast<int>(pl->K);
+    int rc = check_cuda(cudaMemsetAsync(pl->d_bad, 0, sizeof(uint32_t), st), "plan_refresh flag");
+    if (rc) return rc;
+    refresh_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(amax, wmax, static_cast<double>(alpha), K, pl->d_s_new,
+                                                          pl->d_bad);
+    if ((rc = check_cuda(cudaGetLastError(), "plan_refresh smooth launch"))) return rc;
+    RefreshParams p{amax, wmax, static_cast<double>(alpha), K, static_cast<int>(pl->k), static_cast<int>(pl->Kb),
+                    static_cast<int>(pl->Kbp), pl->d_s_new, pl->d_bad, pl->d_s, pl->d_inv_s, pl->d_route,
                     pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status};
-    plan_refresh_kernel<<<1, RF_THREADS, 0, st>>>(p);
+    const size_t smem = sizeof(uint32_t) * static_cast<size_t>(K < RF_SMEM_KEYS ? K : RF_SMEM_KEYS);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if ((rc = check_cuda(cudaFuncSetAttribute(plan_refresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(sizeof(uint32_t) * RF_SMEM_KEYS)),
+                             "plan_refresh smem attribute")))
+            return rc;
+        attr_set[dev] = true;
+    }
+    plan_refresh_kernel<<<1, RF_THREADS, smem, st>>>(p);
     return check_cuda(cudaGetLastError(), "plan_refresh launch");
 }
 
