@@ -12,7 +12,8 @@ library ``outlier_split_mixed_b200``; only the seeded input generators
 arithmetic) feed both.
 
 Pinned functions (see tests/test_oracle_*.py): BF16 rounding, E2M1 codec,
-MX scale exponent, calibration (Eq. (2), Eq. (4)), smoothing/folding
+MX scale exponent, calibration (Eq. (2), Eq. (4), the tail-aware percentile
+score), smoothing/folding
 (Eq. (1)), quantize_act, pack_weights (all three block-scale modes),
 dual_gemm_rows (Eq. (5)). The FP32 tanh-form GELU is pinned only to libm
 within an error bound ("parity unpinned" for its exact bits).
@@ -72,6 +73,11 @@ def _load():
             lib.oracle_weight_amax.argtypes = [P, I64, I64, P]
             lib.oracle_calibrate.restype = ctypes.c_int
             lib.oracle_calibrate.argtypes = [P, P, I64, ctypes.c_float, I64, P, P, P]
+            lib.oracle_calibrate_scored.restype = ctypes.c_int
+            lib.oracle_calibrate_scored.argtypes = [P, P, P, I64, ctypes.c_float, I64, P, P, P]
+            lib.oracle_percentile_rank.restype = I64
+            lib.oracle_percentile_rank.argtypes = [ctypes.c_double, I64]
+            lib.oracle_act_percentile.argtypes = [P, I64, I64, I64, P]
             lib.oracle_smooth_act.argtypes = [P, I64, I64, P, P]
             lib.oracle_fold_weights.argtypes = [P, I64, I64, P, P]
             lib.oracle_quantize_act.argtypes = [P, I64, I64, I64, P, P, P, P, P]
@@ -186,6 +192,35 @@ def calibrate(amax: np.ndarray, wmax: np.ndarray, alpha: float, k: int):
     if rc != 0:
         raise ValueError("non-finite calibration statistics")
     return s, inv_s, O[:k].copy()
+
+
+def calibrate_scored(amax: np.ndarray, score: np.ndarray, wmax: np.ndarray, alpha: float, k: int):
+    """Eq. (2) from the maxima, Eq. (4)'s top-k by a separate score."""
+    amax = _c(amax, np.float32)
+    score = _c(score, np.float32)
+    wmax = _c(wmax, np.float32)
+    K = amax.shape[0]
+    s = np.empty(K, np.float32)
+    inv_s = np.empty(K, np.float32)
+    O = np.empty(max(k, 1), np.int32)
+    rc = _load().oracle_calibrate_scored(_p(amax), _p(score), _p(wmax), K, float(alpha), k, _p(s), _p(inv_s), _p(O))
+    if rc != 0:
+        raise ValueError("non-finite calibration statistics")
+    return s, inv_s, O[:k].copy()
+
+
+def percentile_rank(q: float, T: int) -> int:
+    """Nearest rank ceil(q T), clamped to [1, T]."""
+    return int(_load().oracle_percentile_rank(float(q), int(T)))
+
+
+def act_percentile(X: np.ndarray, rank: int) -> np.ndarray:
+    """score[j] = the rank-th smallest |x_tj| (rank 1-based)."""
+    X = _c(X, np.uint16)
+    T, K = X.shape
+    out = np.empty(K, np.float32)
+    _load().oracle_act_percentile(_p(X), T, K, int(rank), _p(out))
+    return out
 
 
 def smooth_act(X: np.ndarray, inv_s: np.ndarray) -> np.ndarray:

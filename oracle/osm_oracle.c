@@ -196,14 +196,16 @@ static int cmp_i32(const void* pa, const void* pb)
  * Eq. (2): s_j = act_scale_j^alpha / weight_scale_j^(1-alpha), evaluated in
  * FP64 with both statistics floored at 1e-5, then rounded to FP32;
  * inv_s_j = 1/s_j in FP32. Eq. (4): O = the k channels with the largest
- * act_scale (ties: lower channel index first), returned ascending.
- * Returns 0, or 1 if a statistic is not finite.
+ * score (ties: lower channel index first), returned ascending; the paper's
+ * score is act_scale itself (oracle_calibrate), the tail-aware variant a
+ * percentile of |x| (oracle_act_percentile). Returns 0, or 1 if a
+ * statistic is not finite.
  */
-int oracle_calibrate(const float* amax, const float* wmax, int64_t K, float alpha,
-                     int64_t k, float* s, float* inv_s, int32_t* O)
+int oracle_calibrate_scored(const float* amax, const float* score, const float* wmax, int64_t K, float alpha,
+                            int64_t k, float* s, float* inv_s, int32_t* O)
 {
     for (int64_t j = 0; j < K; ++j)
-        if (!isfinite(amax[j]) || !isfinite(wmax[j])) return 1;
+        if (!isfinite(amax[j]) || !isfinite(wmax[j]) || !isfinite(score[j])) return 1;
     double a = (double)alpha;
     for (int64_t j = 0; j < K; ++j) {
         double am = (double)amax[j] < 1e-5 ? 1e-5 : (double)amax[j];
@@ -215,13 +217,53 @@ int oracle_calibrate(const float* amax, const float* wmax, int64_t K, float alph
     if (k > 0) {
         int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
         for (int64_t j = 0; j < K; ++j) idx[j] = j;
-        g_sort_amax = amax;
+        g_sort_amax = score;
         qsort(idx, (size_t)K, sizeof(int64_t), cmp_score_desc);
         for (int64_t i = 0; i < k; ++i) O[i] = (int32_t)idx[i];
         qsort(O, (size_t)k, sizeof(int32_t), cmp_i32);
         free(idx);
     }
     return 0;
+}
+
+int oracle_calibrate(const float* amax, const float* wmax, int64_t K, float alpha,
+                     int64_t k, float* s, float* inv_s, int32_t* O)
+{
+    return oracle_calibrate_scored(amax, amax, wmax, K, alpha, k, s, inv_s, O);
+}
+
+/*
+ * Tail-aware channel score (the activation-tail-aware percentile
+ * calibration of the Tail-Aware HiFloat4 page, used to build the channel
+ * mask): the nearest-rank q-percentile of |x_tj| over the T calibration
+ * tokens, i.e. the value of rank r in ascending order with
+ * r = ceil(q T) clamped to [1, T], evaluated in FP64. q = 1 gives the
+ * maximum, the score of Eq. (4).
+ */
+int64_t oracle_percentile_rank(double q, int64_t T)
+{
+    double r = ceil(q * (double)T);
+    if (r < 1.0) r = 1.0;
+    if (r > (double)T) r = (double)T;
+    return (int64_t)r;
+}
+
+static int cmp_f32_asc(const void* pa, const void* pb)
+{
+    float a = *(const float*)pa, b = *(const float*)pb;
+    return (a > b) - (a < b);
+}
+
+/* score[j] = the rank-th smallest |x_tj| over t (rank 1-based). */
+void oracle_act_percentile(const uint16_t* X, int64_t T, int64_t K, int64_t rank, float* score)
+{
+    float* col = (float*)malloc(sizeof(float) * (size_t)T);
+    for (int64_t j = 0; j < K; ++j) {
+        for (int64_t t = 0; t < T; ++t) col[t] = fabsf(oracle_bf16_to_f32(X[t * K + j]));
+        qsort(col, (size_t)T, sizeof(float), cmp_f32_asc);
+        score[j] = col[rank - 1];
+    }
+    free(col);
 }
 
 /* J = ascending complement of O in [0, K). Returns Kb. */

@@ -4,6 +4,7 @@ import numpy as np
 import pytest
 
 import oracle
+from conftest import golden_path
 from outlier_split_mixed_b200 import synth
 
 
@@ -104,3 +105,75 @@ def test_eq1_wrong_channel_would_be_caught(small_layer):
     x, w = _f32(X), _f32(W)
     bound = (2.0 ** -8 + 2.0 ** -17) * (np.abs(x) @ np.abs(w))
     assert np.any(np.abs(_f32(Xs) @ _f32(Ws) - x @ w) > bound)
+
+
+# ---- tail-aware (percentile) channel score -------------------------------
+
+def _golden_percentiles():
+    rows = []
+    with open(golden_path("percentile_rank.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                q, r, v = line.split()
+                rows.append((float(q), int(r), float(v)))
+    return rows
+
+
+def test_percentile_golden_column():
+    col = np.array([3, -1, 4, 1, -5, 9, 2, 6], np.float32)
+    X = synth.to_bf16_bits(col[:, None] * np.ones((1, 32), np.float32))
+    for q, r, v in _golden_percentiles():
+        assert oracle.percentile_rank(q, 8) == r, q
+        score = oracle.act_percentile(X, r)
+        assert np.all(score == np.float32(v)), (q, score[0], v)
+
+
+def test_percentile_at_q1_is_the_maximum_and_monotone_in_q():
+    X = synth.acts_heavy_tailed(200, 96, seed=31, frac=0.05)
+    T = X.shape[0]
+    amax = oracle.act_amax(X)
+    assert np.array_equal(oracle.act_percentile(X, oracle.percentile_rank(1.0, T)), amax)
+    prev = None
+    for q in (0.5, 0.9, 0.99, 0.999, 1.0):
+        sc = oracle.act_percentile(X, oracle.percentile_rank(q, T))
+        assert np.all(sc <= amax)
+        if prev is not None:
+            assert np.all(sc >= prev)
+        prev = sc
+
+
+def test_scored_calibration_reduces_to_eq4_with_the_maximum():
+    rng = np.random.default_rng(41)
+    K, k = 300, 17
+    amax = np.exp(rng.normal(0, 1, K)).astype(np.float32)
+    wmax = rng.uniform(0.01, 0.5, K).astype(np.float32)
+    a = oracle.calibrate(amax, wmax, 0.55, k)
+    b = oracle.calibrate_scored(amax, amax, wmax, 0.55, k)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    # s does not depend on the score; O does
+    score = rng.permutation(amax)
+    c = oracle.calibrate_scored(amax, score, wmax, 0.55, k)
+    assert np.array_equal(c[0], a[0]) and np.array_equal(c[1], a[1])
+    assert np.array_equal(c[2], np.sort(np.argsort(-score, kind="stable")[:k]))
+
+
+def test_percentile_score_ignores_a_single_token_spike():
+    # The purpose of the tail-aware score: a channel whose maximum comes from
+    # one rare token is an outlier for Eq. (4)'s max score but not for a
+    # percentile score, while a channel with a consistently heavy tail is
+    # an outlier for both.
+    T, K = 512, 64
+    rng = np.random.default_rng(5)
+    x = rng.normal(0, 0.3, (T, K)).astype(np.float32)
+    x[7, 10] = 40.0                                   # one spike
+    x[:, 20] = rng.standard_t(2, T).astype(np.float32) * 3.0   # heavy tail throughout
+    X = synth.to_bf16_bits(x)
+    amax = oracle.act_amax(X)
+    score = oracle.act_percentile(X, oracle.percentile_rank(0.99, T))
+    wmax = np.full(K, 0.3, np.float32)
+    O_max = oracle.calibrate(amax, wmax, 0.5, 2)[2]
+    O_pct = oracle.calibrate_scored(amax, score, wmax, 0.5, 2)[2]
+    assert 10 in O_max and 20 in O_max
+    assert 10 not in O_pct and 20 in O_pct
