@@ -589,14 +589,21 @@ def run_refresh(args, cfg, rank, world, local_rank):
     wc, wsc, wh = plan.alloc_packed(N, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
+    score = torch.empty(K, dtype=torch.float32, device=dev) if args.percentile else None
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
         amax.zero_()
         osm.act_amax_accumulate(Xd, amax)
+        if score is not None:
+            osm.act_percentile(Xd, args.percentile, score)
         if ev is not None:
             ev[1].record(stream)
-        plan.refresh(amax, wmax, cfg.alpha)
+        if score is not None:
+            plan.refresh_scored(amax, score, wmax, cfg.alpha)
+        else:
+            plan.refresh(amax, wmax, cfg.alpha)
         if ev is not None:
             ev[2].record(stream)
         osm.pack_weights(plan, Wd, wc, wsc, wh)
@@ -623,13 +630,14 @@ def run_refresh(args, cfg, rank, world, local_rank):
         cb, sb, hb = plan.sizes(N)
         pack_bytes = K * N * 2 + cb + sb + hb
         line = {
-            "metric": "dynamic re-calibration time per step (activation maxima + plan refresh + weight repack)",
+            "metric": "dynamic re-calibration time per step (activation statistics + plan refresh + weight repack)",
             "value": step_s * 1e6, "unit": "us", "n_gpus": world, "steps": n, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 in, mxfp4+bf16 out", "data": "synthetic",
-            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)"),
+            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
+                           channel_score=f"percentile {args.percentile}" if args.percentile else "maximum"),
             "kernels": {
-                "act_amax": {"us": t[0] * 1e6, "gbs": M * K * 2 / t[0] / 1e9},
+                "act_stats": {"us": t[0] * 1e6, "gbs": M * K * 2 * (2 if args.percentile else 1) / t[0] / 1e9},
                 "plan_refresh": {"us": t[1] * 1e6},
                 "pack_weights": {"us": t[2] * 1e6, "gbs": pack_bytes / t[2] / 1e9, "bytes": pack_bytes,
                                  "frac_hbm": pack_bytes / t[2] / 1e9 / peaks["hbm_gbs"]},
@@ -655,6 +663,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiler captures)")
     ap.add_argument("--blocks", type=int, default=0, help="override the number of FFN blocks (ffn workload)")
+    ap.add_argument("--percentile", type=float, default=0.0,
+                    help="refresh workload: score channels by this percentile of |x| (0: by the maximum)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -127,6 +127,23 @@ OSM_API int osm_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax
 OSM_API int osm_calibrate_finalize(const float* amax_host, const float* wmax_host, int64_t K, float alpha,
                            int64_t k, float* s_host, float* inv_s_host, int32_t* O_host);
 
+/* Tail-aware channel score (the activation-tail-aware percentile
+ * calibration of the Tail-Aware HiFloat4 page, which builds the channel
+ * mask from the tail of the activation distribution so that rare
+ * calibration spikes do not decide the outlier set). score[j] = the
+ * nearest-rank q-percentile of |x_tj| over the T tokens of X [T][K] BF16:
+ * the value of rank ceil(q T) (clamped to [1, T], computed in FP64) in
+ * ascending order. q in (0, 1]; q = 1 gives the maximum. score: device
+ * float[K]. All T tokens in one call (percentiles do not merge across
+ * batches). K % 32 == 0. */
+OSM_API int osm_act_percentile(const uint16_t* X, int64_t T, int64_t K, float q, float* score, void* stream);
+
+/* As osm_calibrate_finalize, with Eq. (4)'s top-k taken by score_host
+ * (e.g. osm_act_percentile) while Eq. (2) keeps amax_host. Host arrays. */
+OSM_API int osm_calibrate_finalize_scored(const float* amax_host, const float* score_host, const float* wmax_host,
+                                          int64_t K, float alpha, int64_t k, float* s_host, float* inv_s_host,
+                                          int32_t* O_host);
+
 /* ---- plans ------------------------------------------------------------ */
 
 /* Build a plan for one linear map with K input and N output channels,
@@ -211,6 +228,11 @@ OSM_API int osm_pack_weights_for_next(const osm_plan* plan, const osm_plan* next
  * statistic sets OSM_STATUS_NONFINITE and leaves the plan unchanged.
  * alpha in (0, 1). */
 OSM_API int osm_plan_refresh(osm_plan* plan, const float* amax, const float* wmax, float alpha, void* stream);
+
+/* As osm_plan_refresh, with the top-k taken by a separate device score
+ * (e.g. osm_act_percentile) while s follows amax. */
+OSM_API int osm_plan_refresh_scored(osm_plan* plan, const float* amax, const float* score, const float* wmax,
+                                    float alpha, void* stream);
 
 /* Copies of the plan's s, inv_s (float[K]) and O (int32[k], ascending) to
  * host memory; any pointer may be NULL. Synchronous. */

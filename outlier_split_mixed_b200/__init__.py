@@ -44,6 +44,9 @@ _SIGNATURES = {
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
     "osm_plan_set_debug": (_I, [_P, ctypes.c_uint32]),
     "osm_plan_refresh": (_I, [_P, _P, _P, ctypes.c_float, _P]),
+    "osm_plan_refresh_scored": (_I, [_P, _P, _P, _P, ctypes.c_float, _P]),
+    "osm_act_percentile": (_I, [_P, _I64, _I64, ctypes.c_float, _P, _P]),
+    "osm_calibrate_finalize_scored": (_I, [_P, _P, _P, _I64, ctypes.c_float, _I64, _P, _P, _P]),
     "osm_plan_tables": (_I, [_P, _P, _P, _P]),
     "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
     "osm_pack_weights_for_next": (_I, [_P, _P, _P, _P, _P, _P, _P]),
@@ -190,6 +193,14 @@ class Plan:
                                       _ptr(wmax, "wmax", (torch.float32,), self.K * 4), float(alpha),
                                       _stream(stream)))
 
+    def refresh_scored(self, amax, score, wmax, alpha: float, stream=None):
+        """As refresh, with the top-k by `score` (osm_plan_refresh_scored)."""
+        import torch
+        f32 = (torch.float32,)
+        _check(lib().osm_plan_refresh_scored(self._h, _ptr(amax, "amax", f32, self.K * 4),
+                                             _ptr(score, "score", f32, self.K * 4),
+                                             _ptr(wmax, "wmax", f32, self.K * 4), float(alpha), _stream(stream)))
+
     def tables(self):
         """(s, inv_s, O) copied to host numpy arrays (osm_plan_tables)."""
         s = np.empty(self.K, np.float32)
@@ -229,6 +240,14 @@ def act_amax_accumulate(X, amax, stream=None):
                                          _ptr(amax, "amax", (torch.float32,), K * 4), _stream(stream)))
 
 
+def act_percentile(X, q: float, score, stream=None):
+    """score[j] = nearest-rank q-percentile of |X[:, j]| on the device (osm_act_percentile)."""
+    T, K = X.shape
+    import torch
+    _check(lib().osm_act_percentile(_ptr(X, "X", _bf16_types()), T, K, float(q),
+                                    _ptr(score, "score", (torch.float32,), K * 4), _stream(stream)))
+
+
 def weight_amax(W, wmax, stream=None):
     """wmax[j] = max_n |W[j][n]| (osm_weight_amax)."""
     K, N = W.shape
@@ -247,6 +266,21 @@ def calibrate_finalize(amax_host: np.ndarray, wmax_host: np.ndarray, alpha: floa
     O = np.empty(max(k, 1), np.int32)
     _check(lib().osm_calibrate_finalize(_host_ptr(amax_host), _host_ptr(wmax_host), K, float(alpha), int(k),
                                         _host_ptr(s), _host_ptr(inv_s), _host_ptr(O)))
+    return s, inv_s, O[:k].copy()
+
+
+def calibrate_finalize_scored(amax_host: np.ndarray, score_host: np.ndarray, wmax_host: np.ndarray, alpha: float,
+                              k: int):
+    """Eq. (2) from amax, Eq. (4)'s top-k by score -> (s, inv_s, O) (osm_calibrate_finalize_scored)."""
+    amax_host = np.ascontiguousarray(amax_host, dtype=np.float32)
+    score_host = np.ascontiguousarray(score_host, dtype=np.float32)
+    wmax_host = np.ascontiguousarray(wmax_host, dtype=np.float32)
+    K = amax_host.shape[0]
+    s = np.empty(K, np.float32)
+    inv_s = np.empty(K, np.float32)
+    O = np.empty(max(k, 1), np.int32)
+    _check(lib().osm_calibrate_finalize_scored(_host_ptr(amax_host), _host_ptr(score_host), _host_ptr(wmax_host), K,
+                                               float(alpha), int(k), _host_ptr(s), _host_ptr(inv_s), _host_ptr(O)))
     return s, inv_s, O[:k].copy()
 
 

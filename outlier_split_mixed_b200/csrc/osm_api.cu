@@ -97,15 +97,15 @@ int osm_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, void* 
     return launch_weight_amax(W, K, N, wmax, static_cast<cudaStream_t>(stream));
 }
 
-int osm_calibrate_finalize(const float* amax_host, const float* wmax_host, int64_t K, float alpha, int64_t k,
-                           float* s_host, float* inv_s_host, int32_t* O_host) {
+int osm_calibrate_finalize_scored(const float* amax_host, const float* score_host, const float* wmax_host, int64_t K,
+                                  float alpha, int64_t k, float* s_host, float* inv_s_host, int32_t* O_host) {
     g_err[0] = 0;
-    OSM_REQUIRE(amax_host && wmax_host && s_host && inv_s_host, "calibrate_finalize: null pointer");
+    OSM_REQUIRE(amax_host && score_host && wmax_host && s_host && inv_s_host, "calibrate_finalize: null pointer");
     OSM_REQUIRE(K > 0 && k >= 0 && k <= K, "calibrate_finalize: need 0 <= k <= K");
     OSM_REQUIRE(k == 0 || O_host, "calibrate_finalize: O_host is NULL");
     OSM_REQUIRE(alpha > 0.0f && alpha < 1.0f, "calibrate_finalize: alpha must lie in (0, 1)");
     for (int64_t j = 0; j < K; ++j)
-        if (!std::isfinite(amax_host[j]) || !std::isfinite(wmax_host[j]))
+        if (!std::isfinite(amax_host[j]) || !std::isfinite(wmax_host[j]) || !std::isfinite(score_host[j]))
             return fail(OSM_ERR_NONFINITE, "calibrate_finalize: statistic of channel %lld is not finite",
                         (long long)j);
     // Eq. (2) in double, statistics floored at 1e-5, rounded once to float
@@ -116,18 +116,35 @@ int osm_calibrate_finalize(const float* amax_host, const float* wmax_host, int64
         s_host[j] = static_cast<float>(std::pow(am, a) / std::pow(wm, 1.0 - a));
         inv_s_host[j] = 1.0f / s_host[j];
     }
-    // Eq. (4): top-k by activation maximum, ties to the lower channel index
+    // Eq. (4): top-k by score, ties to the lower channel index
     if (k > 0) {
         std::vector<int32_t> idx(static_cast<size_t>(K));
         std::iota(idx.begin(), idx.end(), 0);
         std::partial_sort(idx.begin(), idx.begin() + k, idx.end(), [&](int32_t x, int32_t y) {
-            if (amax_host[x] != amax_host[y]) return amax_host[x] > amax_host[y];
+            if (score_host[x] != score_host[y]) return score_host[x] > score_host[y];
             return x < y;
         });
         std::sort(idx.begin(), idx.begin() + k);
         std::copy(idx.begin(), idx.begin() + k, O_host);
     }
     return OSM_OK;
+}
+
+int osm_calibrate_finalize(const float* amax_host, const float* wmax_host, int64_t K, float alpha, int64_t k,
+                           float* s_host, float* inv_s_host, int32_t* O_host) {
+    return osm_calibrate_finalize_scored(amax_host, amax_host, wmax_host, K, alpha, k, s_host, inv_s_host, O_host);
+}
+
+int osm_act_percentile(const uint16_t* X, int64_t T, int64_t K, float q, float* score, void* stream) {
+    g_err[0] = 0;
+    OSM_REQUIRE(T >= 1 && K > 0 && K % 32 == 0 && K <= 0x7FFFFFFF, "act_percentile: need T >= 1, K %% 32 == 0");
+    OSM_REQUIRE(q > 0.0f && q <= 1.0f, "act_percentile: q must lie in (0, 1]");
+    OSM_REQUIRE(X && aligned16(X) && score, "act_percentile: null or misaligned pointer");
+    OSM_TRY(check_device());
+    double r = std::ceil(static_cast<double>(q) * static_cast<double>(T));
+    if (r < 1.0) r = 1.0;
+    if (r > static_cast<double>(T)) r = static_cast<double>(T);
+    return launch_act_percentile(X, T, K, static_cast<int64_t>(r), score, static_cast<cudaStream_t>(stream));
 }
 
 int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const int32_t* O_host, int wscale_mode,
@@ -319,14 +336,18 @@ int osm_plan_channel_order(const osm_plan* p, int32_t* order_host) {
                       "plan_channel_order: read");
 }
 
-int osm_plan_refresh(osm_plan* p, const float* amax, const float* wmax, float alpha, void* stream) {
+int osm_plan_refresh_scored(osm_plan* p, const float* amax, const float* score, const float* wmax, float alpha,
+                            void* stream) {
     g_err[0] = 0;
     OSM_TRY(check_plan(p));
-    OSM_REQUIRE(amax && wmax && (reinterpret_cast<uintptr_t>(amax) & 3) == 0 &&
-                    (reinterpret_cast<uintptr_t>(wmax) & 3) == 0,
-                "plan_refresh: amax / wmax null or misaligned");
+    auto ok = [](const float* x) { return x && (reinterpret_cast<uintptr_t>(x) & 3) == 0; };
+    OSM_REQUIRE(ok(amax) && ok(score) && ok(wmax), "plan_refresh: amax / score / wmax null or misaligned");
     OSM_REQUIRE(alpha > 0.0f && alpha < 1.0f, "plan_refresh: alpha must lie in (0, 1)");
-    return launch_plan_refresh(p, amax, wmax, alpha, static_cast<cudaStream_t>(stream));
+    return launch_plan_refresh(p, amax, score, wmax, alpha, static_cast<cudaStream_t>(stream));
+}
+
+int osm_plan_refresh(osm_plan* p, const float* amax, const float* wmax, float alpha, void* stream) {
+    return osm_plan_refresh_scored(p, amax, amax, wmax, alpha, stream);
 }
 
 int osm_plan_tables(const osm_plan* p, float* s_host, float* inv_s_host, int32_t* O_host) {

@@ -51,10 +51,12 @@ inline int64_t scales_bytes(int64_t rows, int64_t Kbp) {
 
 // launchers (return OSM_OK or an error code; arguments already validated)
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st);
+int launch_act_percentile(const uint16_t* X, int64_t T, int64_t K, int64_t rank, float* score, cudaStream_t st);
 int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cudaStream_t st);
 int launch_pack_weights(const osm_plan* p, const uint16_t* W, const int32_t* col_order, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st);
-int launch_plan_refresh(osm_plan* p, const float* amax, const float* wmax, float alpha, cudaStream_t st);
+int launch_plan_refresh(osm_plan* p, const float* amax, const float* score, const float* wmax, float alpha,
+                        cudaStream_t st);
 int launch_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st);
 int launch_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_scales,

@@ -107,6 +107,53 @@ __global__ void __launch_bounds__(128) act_amax_kernel(const uint16_t* __restric
     }
 }
 
+// Tail-aware channel score (the activation-tail-aware percentile
+// calibration of the Tail-Aware HiFloat4 page): score[j] = the rank-th
+// smallest |x_tj| over the T tokens (rank 1-based; the host derives it from
+// the percentile q as ceil(q T)). One CTA per 32 channels, lane = channel,
+// warps over rows; a two-pass radix select on the 15-bit |x| pattern (high
+// 8 bits, then the low 7 within the chosen bucket) with per-channel shared
+// histograms padded so that equal buckets of different channels fall in
+// different banks.
+constexpr int PCT_THREADS = 256;
+
+__global__ void __launch_bounds__(PCT_THREADS) act_percentile_kernel(const uint16_t* __restrict__ X, int64_t T,
+                                                                     int64_t K, int64_t rank,
+                                                                     float* __restrict__ score) {
+    __shared__ unsigned hist[32][257];
+    __shared__ unsigned pick[32], rem[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;  // K % 32 == 0
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int i = threadIdx.x; i < 32 * 257; i += PCT_THREADS) (&hist[0][0])[i] = 0;
+        __syncthreads();
+        const unsigned hi = pass ? pick[lane] : 0u;
+        for (int64_t t = warp; t < T; t += PCT_THREADS / 32) {
+            const unsigned key = X[t * K + j] & 0x7FFFu;
+            if (pass == 0) atomicAdd(&hist[lane][key >> 7], 1u);
+            else if ((key >> 7) == hi) atomicAdd(&hist[lane][key & 127u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int c = threadIdx.x;
+            unsigned need = pass ? rem[c] : static_cast<unsigned>(rank);
+            const int nb = pass ? 128 : 256;
+            int b = 0;
+            for (; b < nb - 1; ++b) {
+                if (hist[c][b] >= need) break;
+                need -= hist[c][b];
+            }
+            if (pass == 0) {
+                pick[c] = static_cast<unsigned>(b);
+                rem[c] = need;
+            } else {
+                score[static_cast<int64_t>(blockIdx.x) * 32 + c] = __uint_as_float(((pick[c] << 7) | b) << 16);
+            }
+        }
+        __syncthreads();
+    }
+}
+
 // wmax[j] = max_n |W[j][n]|: one block per input channel row.
 __global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t* __restrict__ W, int64_t N,
                                                           float* __restrict__ wmax) {
@@ -634,6 +681,11 @@ int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaSt
     if (grid.y > 65535u) return fail(OSM_ERR_UNSUPPORTED, "act_amax: T too large for one launch");
     act_amax_kernel<<<grid, 128, 0, st>>>(X, T, K, amax);
     return check_cuda(cudaGetLastError(), "act_amax launch");
+}
+
+int launch_act_percentile(const uint16_t* X, int64_t T, int64_t K, int64_t rank, float* score, cudaStream_t st) {
+    act_percentile_kernel<<<static_cast<unsigned>(K / 32), PCT_THREADS, 0, st>>>(X, T, K, rank, score);
+    return check_cuda(cudaGetLastError(), "act_percentile launch");
 }
 
 int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cudaStream_t st) {

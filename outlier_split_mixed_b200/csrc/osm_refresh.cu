@@ -11,9 +11,10 @@
 // Kernel 2, one CTA of 1024 threads (K <= 65536):
 //  1. flag set -> OSM_STATUS_NONFINITE, every table untouched;
 //  2. s, inv_s adopted from scratch;
-//  3. O = the k channels with the largest key (amax, mapped to an unsigned
-//     integer of the same order, << 16 | 0xFFFF - j): keys are unique, and
-//     their order is amax descending, then channel index ascending.
+//  3. O = the k channels with the largest key (the score -- amax for Eq. (4),
+//     or a tail-aware percentile -- mapped to an unsigned integer of the
+//     same order, << 16 | 0xFFFF - j): keys are unique, and their order is
+//     score descending, then channel index ascending.
 //     The k-th largest key is found by a radix select over the 48 key bits,
 //     8 bits per pass: a shared 256-bin histogram (one increment per
 //     distinct digit of a warp) and a warp-parallel search from the top;
@@ -33,7 +34,8 @@ namespace {
 constexpr int RF_THREADS = 1024;
 
 struct RefreshParams {
-    const float* amax;
+    const float* amax;     // Eq. (2)
+    const float* score;    // Eq. (4)
     const float* wmax;
     double alpha;
     int K, k, Kb, Kbp;
@@ -91,12 +93,13 @@ __device__ __forceinline__ int block_exclusive_scan(int flag, int* warp_tot, int
 }
 
 __global__ void __launch_bounds__(256) refresh_smooth_kernel(const float* __restrict__ amax,
+                                                             const float* __restrict__ score,
                                                              const float* __restrict__ wmax, double alpha, int K,
                                                              float* __restrict__ s_new, uint32_t* __restrict__ bad) {
     const int j = blockIdx.x * 256 + threadIdx.x;
     if (j >= K) return;
     const float a = amax[j], w = wmax[j];
-    if (!isfinite(a) || !isfinite(w)) {
+    if (!isfinite(a) || !isfinite(w) || !isfinite(score[j])) {
         atomicOr(bad, 1u);
         return;
     }
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     for (int j = tid; j < p.K; j += RF_THREADS) {
         p.s[j] = p.s_new[j];
         p.inv_s[j] = p.s_new[p.K + j];
-        if (j < RF_SMEM_KEYS) sk[j] = rf_ord(p.amax[j]);
+        if (j < RF_SMEM_KEYS) sk[j] = rf_ord(p.score[j]);
     }
     __syncthreads();
 
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
             const uint64_t hi_mask = shift == 40 ? 0ull : (~0ull << (shift + 8)) & 0xFFFFFFFFFFFFull;
             for (int j0 = 0; j0 < p.K; j0 += RF_THREADS) {  // uniform trip count: whole warps stay converged
                 const int j = j0 + tid;
-                const uint64_t key = j < p.K ? rf_key(sk, p.amax, j) : 0;
+                const uint64_t key = j < p.K ? rf_key(sk, p.score, j) : 0;
                 const bool in = j < p.K && (key & hi_mask) == prefix;
                 const unsigned digit = in ? static_cast<unsigned>((key >> shift) & 0xFF) : 256u;
                 // one shared-memory increment per distinct digit of the warp
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     for (int c0 = 0; c0 < p.K; c0 += RF_THREADS) {
         const int j = c0 + tid;
         const bool valid = j < p.K;
-        const int sel = valid && rf_key(sk, p.amax, valid ? j : 0) >= thresh ? 1 : 0;
+        const int sel = valid && rf_key(sk, p.score, valid ? j : 0) >= thresh ? 1 : 0;
         const int r_o = block_exclusive_scan(sel, warp_tot, &total) + base_o;
         const int n_sel = total;
         const int r_j = base_j + tid - (r_o - base_o);  // unselected channels before j
@@ -220,14 +223,15 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
 
 }  // namespace
 
-int launch_plan_refresh(osm_plan* pl, const float* amax, const float* wmax, float alpha, cudaStream_t st) {
+int launch_plan_refresh(osm_plan* pl, const float* amax, const float* score, const float* wmax, float alpha,
+                        cudaStream_t st) {
     const int K = static_cast<int>(pl->K);
     int rc = check_cuda(cudaMemsetAsync(pl->d_bad, 0, sizeof(uint32_t), st), "plan_refresh flag");
     if (rc) return rc;
-    refresh_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(amax, wmax, static_cast<double>(alpha), K, pl->d_s_new,
-                                                          pl->d_bad);
+    refresh_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(amax, score, wmax, static_cast<double>(alpha), K,
+                                                          pl->d_s_new, pl->d_bad);
     if ((rc = check_cuda(cudaGetLastError(), "plan_refresh smooth launch"))) return rc;
-    RefreshParams p{amax, wmax, static_cast<double>(alpha), K, static_cast<int>(pl->k), static_cast<int>(pl->Kb),
+    RefreshParams p{amax, score, wmax, static_cast<double>(alpha), K, static_cast<int>(pl->k), static_cast<int>(pl->Kb),
                     static_cast<int>(pl->Kbp), pl->d_s_new, pl->d_bad, pl->d_s, pl->d_inv_s, pl->d_route,
                     pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status};
     const size_t smem = sizeof(uint32_t) * static_cast<size_t>(K < RF_SMEM_KEYS ? K : RF_SMEM_KEYS);

@@ -143,3 +143,46 @@ def test_refresh_with_non_finite_statistics_keeps_the_plan():
     plan.refresh(torch.from_numpy(amax).cuda(), torch.from_numpy(wbad).cuda(), 0.5)
     torch.cuda.synchronize()
     assert plan.status(clear=True) & osm.STATUS_NONFINITE
+
+
+@pytest.mark.parametrize("T,K,q", [(2048, 512, 0.999), (2048, 512, 0.99), (1000, 256, 0.5), (7, 64, 0.9),
+                                   (1, 32, 0.3), (513, 1024, 1.0)])
+def test_act_percentile_matches_oracle(T, K, q):
+    X = synth.acts_heavy_tailed(T, K, seed=T + K, frac=0.03)
+    X[: T // 3, ::5] = X[0, ::5]                       # many equal values in some columns
+    Xd = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    score = torch.empty(K, dtype=torch.float32, device="cuda")
+    osm.act_percentile(Xd, q, score)
+    want = oracle.act_percentile(X, oracle.percentile_rank(q, T))
+    assert np.array_equal(score.cpu().numpy(), want)
+    if q == 1.0:
+        assert np.array_equal(want, oracle.act_amax(X))
+
+
+def test_scored_refresh_matches_oracle():
+    T, K, k, alpha = 1024, 2048, 40, 0.55
+    X = synth.acts_heavy_tailed(T, K, seed=91, frac=0.02)
+    quiet = int(np.argmin(oracle.act_amax(X)))
+    X[3, quiet] = synth.to_bf16_bits(np.array([60.0], np.float32))[0]   # a one-token spike
+    W = synth.weights_gaussian(K, 128, 92, 0.04)
+    Xd = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    Wd = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+    amax = torch.zeros(K, dtype=torch.float32, device="cuda")
+    score = torch.empty(K, dtype=torch.float32, device="cuda")
+    wmax = torch.empty(K, dtype=torch.float32, device="cuda")
+    osm.act_amax_accumulate(Xd, amax)
+    osm.act_percentile(Xd, 0.99, score)
+    osm.weight_amax(Wd, wmax)
+    plan = osm.Plan(K, 128, k, np.ones(K, np.float32), np.arange(k, dtype=np.int32), osm.WSCALE_1x32)
+    plan.refresh_scored(amax, score, wmax, alpha)
+    s_g, _, O_g = plan.tables()
+    am_o, wm_o = oracle.act_amax(X), oracle.weight_amax(W)
+    sc_o = oracle.act_percentile(X, oracle.percentile_rank(0.99, T))
+    s_o, _, O_o = oracle.calibrate_scored(am_o, sc_o, wm_o, alpha, k)
+    assert np.array_equal(O_g, O_o)
+    assert _ulps(s_g, s_o).max() <= 1
+    assert quiet not in O_g                           # the spike does not decide the mask
+    assert quiet in oracle.calibrate(am_o, wm_o, alpha, k)[2]           # ... while the maximum would
+    # the host path on the same device statistics agrees
+    h = osm.calibrate_finalize_scored(amax.cpu().numpy(), score.cpu().numpy(), wmax.cpu().numpy(), alpha, k)
+    assert np.array_equal(h[2], O_g)

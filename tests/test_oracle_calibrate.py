@@ -177,3 +177,18 @@ def test_percentile_score_ignores_a_single_token_spike():
     O_pct = oracle.calibrate_scored(amax, score, wmax, 0.5, 2)[2]
     assert 10 in O_max and 20 in O_max
     assert 10 not in O_pct and 20 in O_pct
+
+
+def test_library_host_finalize_equals_the_oracle():
+    # osm_calibrate_finalize(_scored) is host code in libosm: no GPU needed.
+    import outlier_split_mixed_b200 as osm
+    rng = np.random.default_rng(3)
+    K, k = 777, 31
+    a = np.exp(rng.normal(0, 1, K)).astype(np.float32)
+    a[::50] = a[1]                                    # ties
+    sc = rng.permutation(a)
+    w = rng.uniform(0.01, 0.5, K).astype(np.float32)
+    for got, want in ((osm.calibrate_finalize(a, w, 0.6, k), oracle.calibrate(a, w, 0.6, k)),
+                      (osm.calibrate_finalize_scored(a, sc, w, 0.6, k), oracle.calibrate_scored(a, sc, w, 0.6, k))):
+        for x, y in zip(got, want):
+            assert np.array_equal(x, y)
