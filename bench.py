@@ -650,13 +650,47 @@ def run_refresh(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_search(args, cfg, rank, world, local_rank):
+    """Per-layer alpha / k search on a calibration batch: wall time per
+    candidate (host calibration and plan, device pack + quantize + GEMM +
+    error norms) over a 4 x 4 grid."""
+    import torch
+    from outlier_split_mixed_b200.search import search_alpha_k
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    T = min(cfg.M, 2048)
+    X = cfg.make_x(T)
+    Xd = torch.from_numpy(X.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd = torch.from_numpy(cfg.make_w().view(np.int16)).to(dev).view(torch.bfloat16)
+    alphas, ks = [0.4, 0.5, 0.6, 0.7], [0, 64, 128, 256]
+    search_alpha_k(Xd, Wd, alphas[:1], ks[:1], wmode=cfg.wmode)  # warm-up
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    r = search_alpha_k(Xd, Wd, alphas, ks, wmode=cfg.wmode)
+    torch.cuda.synchronize()
+    t = (time.perf_counter() - t0) / len(r.table)
+    if rank == 0:
+        line = {
+            "metric": "per-layer alpha/k search time per candidate (wall clock)",
+            "value": t * 1e3, "unit": "ms", "n_gpus": 1, "steps": len(r.table), "warmup": 1,
+            "ms_per_step": t * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in, mxfp4+bf16 path, fp64 error norms", "data": "synthetic",
+            "config": dict(workload_config(cfg), calibration_tokens=T, alphas=alphas, ks=ks),
+            "best": {"alpha": r.alpha, "k": r.k, "rel_err": r.rel_err},
+            "table": [{"alpha": a, "k": k, "rel_err": e} for a, k, e in r.table],
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn", "refresh"], default="up")
+    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn", "refresh", "search"], default="up")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -672,7 +706,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = workloads()[args.workload if args.workload != "refresh" else "up"]
+    cfg = workloads()[args.workload if args.workload not in ("refresh", "search") else "up"]
     if args.tokens or args.blocks:
         import dataclasses
         changes = {}
@@ -698,6 +732,8 @@ def main():
             return run_ffn(args, cfg, rank, world, local_rank)
         if args.workload == "refresh":
             return run_refresh(args, cfg, rank, world, local_rank)
+        if args.workload == "search":
+            return run_search(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:

@@ -238,6 +238,14 @@ OSM_API int osm_plan_refresh_scored(osm_plan* plan, const float* amax, const flo
  * host memory; any pointer may be NULL. Synchronous. */
 OSM_API int osm_plan_tables(const osm_plan* plan, float* s_host, float* inv_s_host, int32_t* O_host);
 
+/* ---- per-layer alpha / k search support -----------------------------------
+ * The paper suggests tuning alpha and k per layer; a search scores each
+ * candidate by the relative error of the layer's output against its
+ * unquantised product. out (device double[2], 8-byte aligned) receives
+ * sum (Y - Yref)^2 and sum Yref^2 over `count` FP32 values, accumulated in
+ * FP64 (the summation order varies between runs in the last bits). */
+OSM_API int osm_error_norms(const float* Y, const float* Yref, int64_t count, double* out, void* stream);
+
 /* ---- runtime activation path ----------------------------------------------
  * "activations are divided in-place by s, quantized ..., and routed through
  * either the W4A4 bulk path or a narrow FP16 outlier path" (implementation

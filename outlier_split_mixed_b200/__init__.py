@@ -46,6 +46,7 @@ _SIGNATURES = {
     "osm_plan_refresh": (_I, [_P, _P, _P, ctypes.c_float, _P]),
     "osm_plan_refresh_scored": (_I, [_P, _P, _P, _P, ctypes.c_float, _P]),
     "osm_act_percentile": (_I, [_P, _I64, _I64, ctypes.c_float, _P, _P]),
+    "osm_error_norms": (_I, [_P, _P, _I64, _P, _P]),
     "osm_calibrate_finalize_scored": (_I, [_P, _P, _P, _I64, ctypes.c_float, _I64, _P, _P, _P]),
     "osm_plan_tables": (_I, [_P, _P, _P, _P]),
     "osm_pack_weights": (_I, [_P, _P, _P, _P, _P, _P]),
@@ -246,6 +247,18 @@ def act_percentile(X, q: float, score, stream=None):
     import torch
     _check(lib().osm_act_percentile(_ptr(X, "X", _bf16_types()), T, K, float(q),
                                     _ptr(score, "score", (torch.float32,), K * 4), _stream(stream)))
+
+
+def error_norms(Y, Yref, stream=None):
+    """(sum (Y - Yref)^2, sum Yref^2) in FP64 on the device (osm_error_norms)."""
+    import torch
+    if Y.shape != Yref.shape:
+        raise ValueError("Y and Yref differ in shape")
+    out = torch.zeros(2, dtype=torch.float64, device=Y.device)
+    _check(lib().osm_error_norms(_ptr(Y, "Y", (torch.float32,)), _ptr(Yref, "Yref", (torch.float32,)), Y.numel(),
+                                 _ptr(out, "out", (torch.float64,)), _stream(stream)))
+    e, n = out.cpu().tolist()
+    return e, n
 
 
 def weight_amax(W, wmax, stream=None):

@@ -362,6 +362,15 @@ int osm_plan_tables(const osm_plan* p, float* s_host, float* inv_s_host, int32_t
     return check_cuda(e, "plan_tables: read");
 }
 
+int osm_error_norms(const float* Y, const float* Yref, int64_t count, double* out, void* stream) {
+    g_err[0] = 0;
+    OSM_REQUIRE(count >= 1, "error_norms: count must be >= 1");
+    OSM_REQUIRE(Y && Yref && out && (reinterpret_cast<uintptr_t>(out) & 7) == 0,
+                "error_norms: null or misaligned pointer");
+    OSM_TRY(check_device());
+    return launch_error_norms(Y, Yref, count, out, static_cast<cudaStream_t>(stream));
+}
+
 int osm_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* a_codes, uint8_t* a_scales,
                      uint16_t* a_hp, void* stream) {
     g_err[0] = 0;

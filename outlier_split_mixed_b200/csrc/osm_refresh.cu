@@ -250,3 +250,56 @@ int launch_plan_refresh(osm_plan* pl, const float* amax, const float* score, con
 }
 
 }  // namespace osm
+
+// ---------------------------------------------------------------------------
+// Error norms for the per-layer alpha / k search: out[0] += sum (y - r)^2,
+// out[1] += sum r^2 over `count` FP32 values, accumulated in FP64.
+
+namespace osm {
+namespace {
+
+__global__ void __launch_bounds__(256) error_norms_kernel(const float* __restrict__ y, const float* __restrict__ r,
+                                                          int64_t count, double* __restrict__ out) {
+    double e = 0.0, n = 0.0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+        const double d = static_cast<double>(y[i]) - static_cast<double>(r[i]);
+        e = fma(d, d, e);
+        n = fma(static_cast<double>(r[i]), static_cast<double>(r[i]), n);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+    }
+    __shared__ double part[2][8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        part[0][warp] = e;
+        part[1][warp] = n;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double se = 0.0, sn = 0.0;
+        for (int w = 0; w < 8; ++w) {
+            se += part[0][w];
+            sn += part[1][w];
+        }
+        atomicAdd(out, se);
+        atomicAdd(out + 1, sn);
+    }
+}
+
+}  // namespace
+
+int launch_error_norms(const float* y, const float* r, int64_t count, double* out, cudaStream_t st) {
+    int rc = check_cuda(cudaMemsetAsync(out, 0, 2 * sizeof(double), st), "error_norms clear");
+    if (rc) return rc;
+    int64_t blocks = (count + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    error_norms_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(y, r, count, out);
+    return check_cuda(cudaGetLastError(), "error_norms launch");
+}
+
+}  // namespace osm
