@@ -80,9 +80,13 @@ def _load():
             lib.oracle_act_percentile.argtypes = [P, I64, I64, I64, P]
             lib.oracle_smooth_act.argtypes = [P, I64, I64, P, P]
             lib.oracle_fold_weights.argtypes = [P, I64, I64, P, P]
-            lib.oracle_quantize_act.argtypes = [P, I64, I64, I64, P, P, P, P, P]
-            lib.oracle_pack_weights.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P, P, P]
-            lib.oracle_dual_gemm_rows.argtypes = [P, P, P, P, I64, P, P, P, I64, I64, I64, P, P, P]
+            lib.oracle_quantize_act_ex.argtypes = [P, I64, I64, I64, P, P, P, P, P, ctypes.c_int]
+            lib.oracle_pack_weights_ex.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P, P, P, ctypes.c_int]
+            lib.oracle_dual_gemm_rows_ex.argtypes = [P, P, P, P, I64, P, P, P, I64, I64, I64, P, P, P, ctypes.c_int]
+            lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+            lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+            lib.oracle_f16_to_f64.restype = ctypes.c_double
+            lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
             lib.oracle_gelu_tanh_f32.restype = ctypes.c_float
             lib.oracle_gelu_tanh_f32.argtypes = [ctypes.c_float]
             lib.oracle_gelu_exp_neg.restype = ctypes.c_float
@@ -241,8 +245,17 @@ def fold_weights(W: np.ndarray, s: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize_act(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray):
-    """Returns (codes [M][Kbp/2] u8, scales [M][Kbp/32] u8 logical, a_hp [M][kp] u16)."""
+def f32_to_f16(f: float) -> int:
+    return int(_load().oracle_f32_to_f16(float(np.float32(f))))
+
+
+def f16_to_f64(h: int) -> float:
+    return float(_load().oracle_f16_to_f64(int(h)))
+
+
+def quantize_act(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray, hp_fp16: bool = False):
+    """Returns (codes [M][Kbp/2] u8, scales [M][Kbp/32] u8 logical, a_hp [M][kp] u16);
+    hp_fp16: outlier slots in binary16 instead of BF16."""
     X = _c(X, np.uint16)
     inv_s = _c(inv_s, np.float32)
     O = _c(O, np.int32)
@@ -253,11 +266,12 @@ def quantize_act(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray):
     scales = np.zeros((M, Kbp // 32), np.uint8)
     a_hp = np.zeros((M, kpp), np.uint16)
     Op = O if k else np.zeros(1, np.int32)
-    _load().oracle_quantize_act(_p(X), M, K, k, _p(inv_s), _p(Op), _p(codes), _p(scales), _p(a_hp))
+    _load().oracle_quantize_act_ex(_p(X), M, K, k, _p(inv_s), _p(Op), _p(codes), _p(scales), _p(a_hp),
+                                   int(bool(hp_fp16)))
     return codes, scales, a_hp
 
 
-def pack_weights(W: np.ndarray, s: np.ndarray, O: np.ndarray, mode: int):
+def pack_weights(W: np.ndarray, s: np.ndarray, O: np.ndarray, mode: int, hp_fp16: bool = False):
     """Returns (codes [N][Kbp/2] u8, scales [N][Kbp/32] u8 logical, w_hp [N][kp] u16)."""
     W = _c(W, np.uint16)
     s = _c(s, np.float32)
@@ -269,7 +283,8 @@ def pack_weights(W: np.ndarray, s: np.ndarray, O: np.ndarray, mode: int):
     scales = np.zeros((N, Kbp // 32), np.uint8)
     w_hp = np.zeros((N, kpp), np.uint16)
     Op = O if k else np.zeros(1, np.int32)
-    _load().oracle_pack_weights(_p(W), K, N, k, _p(s), _p(Op), int(mode), _p(codes), _p(scales), _p(w_hp))
+    _load().oracle_pack_weights_ex(_p(W), K, N, k, _p(s), _p(Op), int(mode), _p(codes), _p(scales), _p(w_hp),
+                                   int(bool(hp_fp16)))
     return codes, scales, w_hp
 
 
@@ -281,7 +296,7 @@ def gelu_bf16(y: np.ndarray) -> np.ndarray:
     return out
 
 
-def dual_gemm_rows(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, bias=None):
+def dual_gemm_rows(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, bias=None, hp_fp16=False):
     """Eq. (5) for the given activation rows. Returns (y [r][N] f64, T [r][N] f64)."""
     a_codes = _c(a_codes, np.uint8)
     a_scales = _c(a_scales, np.uint8)
@@ -300,7 +315,7 @@ def dual_gemm_rows(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, bias=
     if bias is not None:
         bias = _c(bias, np.float32)
         bptr = _p(bias)
-    _load().oracle_dual_gemm_rows(_p(a_codes), _p(a_scales), _p(a_hp), _p(rows), rows.shape[0],
-                                  _p(w_codes), _p(w_scales), _p(w_hp), N, Kbp, kpp, bptr,
-                                  _p(y), _p(T))
+    _load().oracle_dual_gemm_rows_ex(_p(a_codes), _p(a_scales), _p(a_hp), _p(rows), rows.shape[0],
+                                     _p(w_codes), _p(w_scales), _p(w_hp), N, Kbp, kpp, bptr,
+                                     _p(y), _p(T), int(bool(hp_fp16)))
     return y, T

@@ -72,6 +72,51 @@ uint16_t oracle_f32_to_bf16(float f)
     return (uint16_t)(pick | (sign >> 16));
 }
 
+/* binary16 (IEEE half) -> FP64: sign, 5-bit exponent (bias 15), 10-bit
+ * significand, subnormals below 2^-14. */
+double oracle_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 31) v = m ? NAN : INFINITY;
+    else if (e == 0) v = ldexp((double)m, -24);
+    else v = ldexp((double)(m + 1024), e - 25);
+    return sign ? -v : v;
+}
+
+/*
+ * Round a binary32 value to the nearest binary16 value, ties to the even
+ * significand, written from the definition as for BF16: the truncated
+ * magnitude code and the next code up are the two neighbours, the nearer
+ * wins, a tie goes to the even code. Magnitudes from 65520 (halfway between
+ * the largest finite half, 65504, and 2^16) round to infinity.
+ */
+uint16_t oracle_f32_to_f16(float f)
+{
+    uint16_t sign = (f32_as_u32(f) >> 16) & 0x8000u;
+    double v = fabs((double)f);
+    if (isnan(f)) return (uint16_t)(sign | 0x7E00u);
+    if (v >= 65520.0) return (uint16_t)(sign | 0x7C00u);
+    uint16_t lo;
+    if (v < ldexp(1.0, -14)) {
+        lo = (uint16_t)floor(v / ldexp(1.0, -24));                /* subnormal grid */
+    } else {
+        int e;
+        frexp(v, &e);                                             /* v in [2^(e-1), 2^e) */
+        double q = ldexp(1.0, (e - 1) - 10);
+        uint16_t mant = (uint16_t)(floor(v / q) - 1024.0);
+        lo = (uint16_t)(((e - 1 + 15) << 10) | mant);
+    }
+    uint16_t hi = (uint16_t)(lo + 1);
+    double dlo = v - oracle_f16_to_f64(lo);
+    double dhi = oracle_f16_to_f64(hi) - v;   /* hi may be 0x7C00 = inf only for v >= 65504 + ... (excluded above) */
+    uint16_t pick;
+    if (dlo < dhi) pick = lo;
+    else if (dhi < dlo) pick = hi;
+    else pick = (lo & 1u) ? hi : lo;
+    return (uint16_t)(pick | sign);
+}
+
 /* Round an FP64 value to binary32 (C conversion is round-to-nearest-even). */
 float oracle_f64_to_f32(double v) { return (float)v; }
 
@@ -317,9 +362,11 @@ void oracle_fold_weights(const uint16_t* W, int64_t K, int64_t N, const float* s
  *   codes E2M1(x'/2^X_b), two per byte, low nibble = even position.
  * Outputs: codes [M][Kbp/2], scales (logical) [M][Kbp/32], a_hp [M][kp].
  */
-void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
-                         const float* inv_s, const int32_t* O,
-                         uint8_t* codes, uint8_t* scales, uint16_t* a_hp)
+/* hp_fp16 != 0: the outlier slots hold the same FP32 products x * inv_s
+ * rounded to binary16 instead of BF16 (the FP16 outlier branch). */
+void oracle_quantize_act_ex(const uint16_t* X, int64_t M, int64_t K, int64_t k,
+                            const float* inv_s, const int32_t* O,
+                            uint8_t* codes, uint8_t* scales, uint16_t* a_hp, int hp_fp16)
 {
     int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
     int64_t nb = Kbp / 32;
@@ -333,7 +380,11 @@ void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
             float p = oracle_bf16_to_f32(X[t * K + j]) * inv_s[j];
             row[j] = oracle_f32_to_bf16(p);
         }
-        for (int64_t i = 0; i < kp; ++i) a_hp[t * kp + i] = (i < k) ? row[O[i]] : 0;
+        for (int64_t i = 0; i < kp; ++i) {
+            if (i >= k) a_hp[t * kp + i] = 0;
+            else if (!hp_fp16) a_hp[t * kp + i] = row[O[i]];
+            else a_hp[t * kp + i] = oracle_f32_to_f16(oracle_bf16_to_f32(X[t * K + O[i]]) * inv_s[O[i]]);
+        }
         for (int64_t b = 0; b < nb; ++b) {
             int64_t p0 = 32 * b;
             int n_real = (int)(p0 >= Kb ? 0 : (Kb - p0 < 32 ? Kb - p0 : 32));
@@ -356,6 +407,13 @@ void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
     free(J);
 }
 
+void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
+                         const float* inv_s, const int32_t* O,
+                         uint8_t* codes, uint8_t* scales, uint16_t* a_hp)
+{
+    oracle_quantize_act_ex(X, M, K, k, inv_s, O, codes, scales, a_hp, 0);
+}
+
 /* ------------------------------------------------------------------ */
 /* Offline weight packing with block-wise scales                         */
 /* ------------------------------------------------------------------ */
@@ -373,9 +431,11 @@ void oracle_quantize_act(const uint16_t* X, int64_t M, int64_t K, int64_t k,
  *   elements (p < Kb, n < N) enter an amax; a block with no real element
  *   gets scale code 0.
  */
-void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
-                         const float* s, const int32_t* O, int mode,
-                         uint8_t* codes, uint8_t* scales, uint16_t* w_hp)
+/* hp_fp16 != 0: w_hp holds the folded outlier weights fp32(w) * s rounded
+ * to binary16 instead of BF16. */
+void oracle_pack_weights_ex(const uint16_t* W, int64_t K, int64_t N, int64_t k,
+                            const float* s, const int32_t* O, int mode,
+                            uint8_t* codes, uint8_t* scales, uint16_t* w_hp, int hp_fp16)
 {
     int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
     int64_t nb = Kbp / 32;
@@ -390,7 +450,11 @@ void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
             Wt[n * K + j] = oracle_f32_to_bf16(p);
         }
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t i = 0; i < kp; ++i) w_hp[n * kp + i] = (i < k) ? Wt[n * K + O[i]] : 0;
+        for (int64_t i = 0; i < kp; ++i) {
+            if (i >= k) w_hp[n * kp + i] = 0;
+            else if (!hp_fp16) w_hp[n * kp + i] = Wt[n * K + O[i]];
+            else w_hp[n * kp + i] = oracle_f32_to_f16(oracle_bf16_to_f32(W[(int64_t)O[i] * N + n]) * s[O[i]]);
+        }
 
     /* block amax of row n, block b (real elements only) */
     double* bam = (double*)calloc((size_t)(N * (nb > 0 ? nb : 1)), sizeof(double));
@@ -437,6 +501,13 @@ void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
     free(J);
 }
 
+void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
+                         const float* s, const int32_t* O, int mode,
+                         uint8_t* codes, uint8_t* scales, uint16_t* w_hp)
+{
+    oracle_pack_weights_ex(W, K, N, k, s, O, mode, codes, scales, w_hp, 0);
+}
+
 /* ------------------------------------------------------------------ */
 /* Eq. (5) / Eq. (3): the dual-branch product                            */
 /* ------------------------------------------------------------------ */
@@ -445,18 +516,18 @@ void oracle_pack_weights(const uint16_t* W, int64_t K, int64_t N, int64_t k,
  * For each requested activation row r (index rows[r] into the packed
  * activations) and every output channel n:
  *   y = sum_b 2^(Xa+Xw) sum_{p in b} e2m1(a) e2m1(w)     (bulk, W4A4)
- *     + sum_{i<kp} a_hp * w_hp                            (outliers, BF16)
+ *     + sum_{i<kp} a_hp * w_hp                            (outliers, BF16 or FP16)
  *     + bias[n]                                            (if bias != NULL)
  *   T = the same sum over absolute values of every term (no bias).
  * Every term is exact in FP64; the sum is accumulated in FP64 in the
  * order bulk blocks, then outlier slots.
  * Outputs y, T: [nrows][N].
  */
-void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
-                           const int64_t* rows, int64_t nrows,
-                           const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
-                           int64_t N, int64_t Kbp, int64_t kp, const float* bias,
-                           double* y, double* T)
+void oracle_dual_gemm_rows_ex(const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
+                              const int64_t* rows, int64_t nrows,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
+                              int64_t N, int64_t Kbp, int64_t kp, const float* bias,
+                              double* y, double* T, int hp_fp16)
 {
     int64_t nb = Kbp / 32;
     /* dequantise all weight rows once: value * 2^Xw, exact in FP64 */
@@ -480,7 +551,8 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
             int Xa = (int)a_scales[t * nb + p / 32] - 127;
             ad[p] = oracle_e2m1_decode(c) * ldexp(1.0, Xa);
         }
-        for (int64_t i = 0; i < kp; ++i) hd[i] = oracle_bf16_to_f64(a_hp[t * kp + i]);
+        for (int64_t i = 0; i < kp; ++i)
+            hd[i] = hp_fp16 ? oracle_f16_to_f64(a_hp[t * kp + i]) : oracle_bf16_to_f64(a_hp[t * kp + i]);
         for (int64_t n = 0; n < N; ++n) {
             double acc = 0.0, mag = 0.0;
             const double* wr = wd + n * Kbp;
@@ -490,7 +562,8 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
                 mag += fabs(term);
             }
             for (int64_t i = 0; i < kp; ++i) {
-                double term = hd[i] * oracle_bf16_to_f64(w_hp[n * kp + i]);
+                double wv = hp_fp16 ? oracle_f16_to_f64(w_hp[n * kp + i]) : oracle_bf16_to_f64(w_hp[n * kp + i]);
+                double term = hd[i] * wv;
                 acc += term;
                 mag += fabs(term);
             }
@@ -502,6 +575,15 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
         free(hd);
     }
     free(wd);
+}
+
+void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
+                           const int64_t* rows, int64_t nrows,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
+                           int64_t N, int64_t Kbp, int64_t kp, const float* bias,
+                           double* y, double* T)
+{
+    oracle_dual_gemm_rows_ex(a_codes, a_scales, a_hp, rows, nrows, w_codes, w_scales, w_hp, N, Kbp, kp, bias, y, T, 0);
 }
 
 /* ------------------------------------------------------------------ */

@@ -145,3 +145,26 @@ def test_gelu_exp_close_to_libm():
         want = math.exp(float(np.float32(x)))
         got = oracle.gelu_exp_neg(float(x))
         assert abs(got - want) <= 3e-7 * want + 1e-38, x
+
+
+# ---- binary16 (FP16 outlier branch) --------------------------------------
+
+def test_f16_rounding_matches_numpy_cast():
+    rng = np.random.default_rng(19)
+    # magnitudes across the whole half range, subnormals and overflow included
+    mag = np.ldexp(1.0 + rng.random(20000), rng.integers(-27, 17, 20000))
+    scaled = (mag * rng.choice([-1.0, 1.0], 20000)).astype(np.float32)
+    edge = np.array([65504.0, 65519.0, 65520.0, 65536.0, 2.0**-14, 2.0**-24, 2.0**-25, 1.5 * 2.0**-25,
+                     3 * 2.0**-26, 1.0 + 2.0**-11, 1.0 + 3 * 2.0**-11, -0.0, 0.0, -2.0**-25], np.float32)
+    for v in np.concatenate([scaled, edge]):
+        want = int(np.array([v], np.float32).astype(np.float16).view(np.uint16)[0])
+        assert oracle.f32_to_f16(float(v)) == want, float(v)
+
+
+def test_f16_decode_of_every_code():
+    codes = np.arange(65536, dtype=np.uint16)
+    want = codes.view(np.float16).astype(np.float64)
+    for c in range(0, 65536, 7):
+        got = oracle.f16_to_f64(c)
+        w = want[c]
+        assert (np.isnan(got) and np.isnan(w)) or got == w, c

@@ -294,3 +294,46 @@ def test_gelu_bf16_special_values():
         assert hi == oracle.f32_to_bf16(oracle.gelu_tanh_f32(yi))
         want = 0.5 * yi * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (yi + 0.044715 * yi ** 3)))
         assert abs(fi - want) <= 2.0 ** -8 * abs(want) + 1e-30, yi
+
+
+def test_fp16_outlier_branch_k_equals_K_is_a_plain_fp16_gemm():
+    # With every channel on the outlier branch in FP16, y is the FP64 sum of
+    # the FP16-rounded smoothed operands' products (a textbook GEMM).
+    M, K, N = 8, 64, 16
+    X = synth.acts_heavy_tailed(M, K, seed=91, frac=0.1)
+    W = synth.weights_gaussian(K, N, seed=92, sigma=0.1)
+    rng = np.random.default_rng(93)
+    s = np.exp(rng.uniform(-0.5, 0.5, K)).astype(np.float32)
+    inv_s = (np.float32(1.0) / s).astype(np.float32)
+    O = np.arange(K, dtype=np.int32)
+    ac, asc, ah = oracle.quantize_act(X, inv_s, O, hp_fp16=True)
+    wc, wsc, wh = oracle.pack_weights(W, s, O, 0, hp_fp16=True)
+    y, _ = oracle.dual_gemm_rows(ac, asc, ah, np.arange(M), wc, wsc, wh, hp_fp16=True)
+    xs = (synth.bf16_bits_to_f32(X) * inv_s[None, :]).astype(np.float32).astype(np.float16).astype(np.float64)
+    ws = (synth.bf16_bits_to_f32(W) * s[:, None]).astype(np.float32).astype(np.float16).astype(np.float64)
+    assert np.allclose(y, xs @ ws, rtol=1e-13, atol=0.0)
+    # bulk untouched by the outlier type
+    ac2, asc2, _ = oracle.quantize_act(X, inv_s, np.arange(4, dtype=np.int32), hp_fp16=True)
+    ac3, asc3, _ = oracle.quantize_act(X, inv_s, np.arange(4, dtype=np.int32), hp_fp16=False)
+    assert np.array_equal(ac2, ac3) and np.array_equal(asc2, asc3)
+
+
+def test_fp16_outlier_branch_is_closer_than_bf16():
+    # Same outlier set: the outlier contribution (y minus the same layer with
+    # the outlier slots zeroed) carries 3 more significand bits in FP16, so
+    # it is closer to the exact product of the smoothed, unrounded operands.
+    M, K, N, k = 64, 256, 32, 32
+    X = synth.acts_heavy_tailed(M, K, seed=95, frac=0.05)
+    W = synth.weights_gaussian(K, N, seed=96, sigma=0.05)
+    s, inv_s, O = oracle.calibrate(oracle.act_amax(X), oracle.weight_amax(W), 0.5, k)
+    xs = _f64(X)[:, O] * inv_s[O].astype(np.float64)
+    ws = _f64(W)[O, :] * s[O, None].astype(np.float64)
+    exact = xs @ ws
+    err = {}
+    for fp16 in (False, True):
+        ac, asc, ah = oracle.quantize_act(X, inv_s, O, hp_fp16=fp16)
+        wc, wsc, wh = oracle.pack_weights(W, s, O, 0, hp_fp16=fp16)
+        y, _ = oracle.dual_gemm_rows(ac, asc, ah, np.arange(M), wc, wsc, wh, hp_fp16=fp16)
+        y0, _ = oracle.dual_gemm_rows(ac, asc, np.zeros_like(ah), np.arange(M), wc, wsc, wh, hp_fp16=fp16)
+        err[fp16] = np.linalg.norm((y - y0) - exact)
+    assert err[True] < err[False] / 4
