@@ -269,7 +269,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     osm.act_amax_accumulate(Xd, amax)
     osm.weight_amax(Wd, wmax)
     s, inv_s, O = odist.calibrate_from_local_stats(amax, wmax, cfg.alpha, cfg.k)
-    plan = osm.Plan(K, N, cfg.k, s, O, cfg.wmode)
+    plan = osm.Plan(K, N, cfg.k, s, O, cfg.wmode, hp_fp16=args.hp_fp16)
     wc, wsc, wh = plan.alloc_packed(N, dev)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M, dev)
@@ -355,6 +355,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             "config": {"workload": cfg.name, "M_per_gpu": M, "K": K, "N": N, "k": cfg.k, "alpha": cfg.alpha,
                        "wscale": {0: "1x32", 1: "32x32", 2: "128x1"}[cfg.wmode],
                        "out": "bf16" if cfg.out_bf16 else "f32",
+                       "outlier_branch": "fp16" if args.hp_fp16 else "bf16",
                        "l2": "flushed between timed steps (256 MiB write, untimed)",
                        "parallelism": f"dp{world} (token shards, no data-path collective)"},
             "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
@@ -428,8 +429,8 @@ def run_ffn(args, cfg, rank, world, local_rank):
         s_d, _, O_d = odist.calibrate_from_local_stats(amax_d, wmax_d, cfg.alpha_down, cfg.k_down)
         full.close()
         del fa, fw, Hc
-        up = osm.Plan(D, F, cfg.k_up, s_u, O_u, cfg.wmode_up)
-        down = osm.Plan(F, D, cfg.k_down, s_d, O_d, cfg.wmode_down)
+        up = osm.Plan(D, F, cfg.k_up, s_u, O_u, cfg.wmode_up, hp_fp16=args.hp_fp16)
+        down = osm.Plan(F, D, cfg.k_down, s_d, O_d, cfg.wmode_down, hp_fp16=args.hp_fp16)
         wu = up.alloc_packed(F, dev)
         osm.pack_weights_for_next(up, down, Wu, *wu)
         wd = down.alloc_packed(D, dev)
@@ -537,7 +538,8 @@ def run_ffn(args, cfg, rank, world, local_rank):
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
             "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
-                           parallelism=f"dp{world} (token shards, no data-path collective)"),
+                           parallelism=f"dp{world} (token shards, no data-path collective)",
+                           outlier_branch="fp16" if args.hp_fp16 else "bf16"),
             "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
             "kernels": {
                 "dual_gemm_up_gelu_requant": {"ms": up_s * 1e3, "tflops": f_up / up_s / 1e12},
@@ -697,6 +699,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiler captures)")
     ap.add_argument("--blocks", type=int, default=0, help="override the number of FFN blocks (ffn workload)")
+    ap.add_argument("--hp-fp16", action="store_true", help="outlier branch in FP16 instead of BF16")
     ap.add_argument("--percentile", type=float, default=0.0,
                     help="refresh workload: score channels by this percentile of |x| (0: by the maximum)")
     args = ap.parse_args()

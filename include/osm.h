@@ -176,6 +176,17 @@ OSM_API int osm_plan_status(const osm_plan* plan, void* stream, uint32_t* status
  * usable. */
 OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
 
+/* Number format of the outlier (high-precision) branch. The paper's
+ * implementation paragraph names an FP16 outlier path; OSM_HP_BF16 is the
+ * default. With OSM_HP_FP16 the outlier slots of activations and weights
+ * hold the same FP32 products x * inv_s and w * s rounded once to binary16
+ * (ties to even; magnitudes of 65520 and above become infinite), and the
+ * branch runs as FP16 x FP16 -> FP32 MMAs; the bulk path is unchanged. Set
+ * it before packing: data packed under the other type must not be used. */
+#define OSM_HP_BF16 0
+#define OSM_HP_FP16 1
+OSM_API int osm_plan_set_outlier_dtype(osm_plan* plan, int dtype);
+
 /* Debug flags for failure-detection tests (no counterpart in the paper).
  * OSM_DEBUG_STARVE_QUANTIZE: osm_quantize_act expects 16 bytes more per row
  * group than its copies deliver, so every wait on a row group runs out after

@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libosm.so")
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
 STATUS_TIMEOUT = 1
+HP_BF16, HP_FP16 = 0, 1
 STATUS_NONFINITE = 2
 DEBUG_STARVE_QUANTIZE = 1
 WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
@@ -43,6 +44,7 @@ _SIGNATURES = {
     "osm_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _I]),
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
     "osm_plan_set_debug": (_I, [_P, ctypes.c_uint32]),
+    "osm_plan_set_outlier_dtype": (_I, [_P, _I]),
     "osm_plan_refresh": (_I, [_P, _P, _P, ctypes.c_float, _P]),
     "osm_plan_refresh_scored": (_I, [_P, _P, _P, _P, ctypes.c_float, _P]),
     "osm_act_percentile": (_I, [_P, _I64, _I64, ctypes.c_float, _P, _P]),
@@ -145,7 +147,8 @@ class Plan:
     """An osm_plan: K, N, k, the smoothing vector s, the outlier set O and
     the weight block-scale mode, with its device tables."""
 
-    def __init__(self, K: int, N: int, k: int, s: np.ndarray, O: np.ndarray, wscale_mode: int = WSCALE_1x32):
+    def __init__(self, K: int, N: int, k: int, s: np.ndarray, O: np.ndarray, wscale_mode: int = WSCALE_1x32,
+                 hp_fp16: bool = False):
         s = np.ascontiguousarray(s, dtype=np.float32)
         O = np.ascontiguousarray(O, dtype=np.int32)
         if s.shape != (K,) or O.shape != (k,):
@@ -158,6 +161,9 @@ class Plan:
         d = [ctypes.c_int64() for _ in range(6)]
         _check(lib().osm_plan_dims(self._h, *[ctypes.byref(x) for x in d]))
         self.K, self.N, self.k, self.Kb, self.Kbp, self.kp = (int(x.value) for x in d)
+        self.hp_fp16 = bool(hp_fp16)
+        if hp_fp16:
+            _check(lib().osm_plan_set_outlier_dtype(self._h, HP_FP16))
 
     @property
     def handle(self):

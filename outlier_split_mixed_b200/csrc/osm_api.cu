@@ -180,6 +180,7 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
     p->Kbp = round_up(K - k, 128);
     p->kp = round_up(k, 64);
     p->wmode = wscale_mode;
+    p->hp_fp16 = 0;
     p->wait_limit_ns = 2000000000ull;
     p->debug_flags = 0;
 
@@ -290,6 +291,14 @@ int osm_plan_set_wait_limit(osm_plan* p, uint64_t ns) {
     OSM_REQUIRE(p, "plan_set_wait_limit: plan is NULL");
     OSM_REQUIRE(ns >= 1000ull, "plan_set_wait_limit: limit below 1 us");
     p->wait_limit_ns = ns;
+    return OSM_OK;
+}
+
+int osm_plan_set_outlier_dtype(osm_plan* p, int dtype) {
+    g_err[0] = 0;
+    OSM_REQUIRE(p, "plan_set_outlier_dtype: plan is NULL");
+    OSM_REQUIRE(dtype == OSM_HP_BF16 || dtype == OSM_HP_FP16, "plan_set_outlier_dtype: unknown type %d", dtype);
+    p->hp_fp16 = dtype == OSM_HP_FP16;
     return OSM_OK;
 }
 

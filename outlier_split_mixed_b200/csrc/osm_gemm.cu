@@ -94,9 +94,11 @@ static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budg
 // (bit 23), M>>4 @24; scale-factor byte ids at bits 29-30 (A) and 4-5 (B).
 constexpr uint32_t IDESC_MXF4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
                                 ((uint32_t)((2 * BM) >> 4) << 24);
-// kind::f16: FP32 accumulate (bit 4), A/B BF16 (1 @7, 1 @10), K-major.
+// kind::f16: FP32 accumulate (bit 4), A/B BF16 (1 @7, 1 @10), K-major;
+// IDESC_F16: the same with A and B binary16 (type 0 in both fields).
 constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                 ((uint32_t)((2 * BM) >> 4) << 24);
+constexpr uint32_t IDESC_F16 = IDESC_BF16 & ~((1u << 7) | (1u << 10));
 
 struct __align__(1024) Smem {
     uint8_t a[STAGES][A_TILE];
@@ -130,12 +132,14 @@ struct GemmParams {
     int num_m, num_n;
     int n_row_tiles; // ceil(N / 128): scale-atom rows of W
     int epi;
+    uint32_t idesc_hp;        // instruction descriptor of the outlier K-steps (BF16 or FP16 operands)
     // OSM_EPI_GELU_REQUANT: the next layer's packed activations
     uint8_t* next_codes;      // [M][nKbp/2]
     uint8_t* next_scales;     // layout, rows padded to 128
     uint16_t* next_hp;        // [M][nkp]
     const float* inv_s_ord;   // next's inv_s in its [J | O] channel order (= this layer's column order)
     int nKb, nKbp, nk, nkp;   // next's bulk / outlier widths
+    int next_hp_fp16;         // next's outlier slots in binary16
     int64_t m_pad;            // M rounded up to 128 (rows of next_scales)
 };
 
@@ -290,7 +294,24 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
         }
     }
     if (c0 + 32 > p.nKb) {
-        // outlier part: columns max(c0, nKb) .. c0+31 -> slots c - nKb
+        // outlier part: columns max(c0, nKb) .. c0+31 -> slots c - nKb; for an
+        // FP16 outlier branch of the next layer the same products
+        // bf16(GELU(acc)) * inv_s, rounded to binary16 instead
+        if (p.next_hp_fp16) {
+            const float4* iv = reinterpret_cast<const float4*>(p.inv_s_ord + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 sv = __ldg(iv + i);
+                const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+                float pr[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    pr[j] = __fmul_rn(mx::bf16_bits_to_f32(mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])))),
+                                      s4[j]);
+                hw[2 * i] = mx::f16x2_bits(pr[0], pr[1]);
+                hw[2 * i + 1] = mx::f16x2_bits(pr[2], pr[3]);
+            }
+        }
         uint16_t* hp = p.next_hp + row * p.nkp;
         if (c0 >= p.nKb && ((c0 - p.nKb) & 7) == 0) {
             uint4* dst = reinterpret_cast<uint4*>(hp + (c0 - p.nKb));
@@ -427,7 +448,7 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool lead
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         ptx::mma_bf16_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
-                                           IDESC_BF16, accumulate);
+                                           p.idesc_hp, accumulate);
                         accumulate = 1;
                     }
                 }
@@ -647,10 +668,11 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
             return rc;
     }
     if (pl->kp > 0) {
-        if ((rc = make_map(&p.tm_ah, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_hp, pl->kp, M, pl->kp * 2, 64, BM, SW,
+        const CUtensorMapDataType hpt = pl->hp_fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        if ((rc = make_map(&p.tm_ah, hpt, a_hp, pl->kp, M, pl->kp * 2, 64, BM, SW,
                            "a_hp")))
             return rc;
-        if ((rc = make_map(&p.tm_bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_hp, pl->kp, pl->N, pl->kp * 2, 64, BN / 2,
+        if ((rc = make_map(&p.tm_bh, hpt, w_hp, pl->kp, pl->N, pl->kp * 2, 64, BN / 2,
                            SW, "w_hp")))
             return rc;
     }
@@ -667,6 +689,7 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     p.num_n = static_cast<int>(ceil_div(pl->N, BN));
     p.n_row_tiles = static_cast<int>(ceil_div(pl->N, 128));
     p.epi = epi;
+    p.idesc_hp = pl->hp_fp16 ? IDESC_F16 : IDESC_BF16;
     if (epi == OSM_EPI_GELU_REQUANT) {
         p.next_codes = next_codes;
         p.next_scales = next_scales;
@@ -677,6 +700,7 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
         p.nk = static_cast<int>(next->k);
         p.nkp = static_cast<int>(next->kp);
         p.m_pad = round_up(M, 128);
+        p.next_hp_fp16 = next->hp_fp16;
     }
 
     void (*kernel)(GemmParams) = nullptr;

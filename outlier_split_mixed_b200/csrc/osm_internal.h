@@ -11,6 +11,7 @@ struct osm_plan {
     int device;
     int64_t K, N, k, Kb, Kbp, kp;
     int wmode;
+    int hp_fp16;         // outlier branch in binary16 (OSM_HP_FP16) instead of BF16
     // device tables, owned by the plan
     float* d_s;          // [K]  smoothing vector s (Eq. (2))
     float* d_inv_s;      // [K]  1.0f / s

@@ -26,6 +26,14 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     return d;
 }
 
+// Two FP32 values -> binary16 pair (RNE each, one cvt.rn.f16x2.f32): lo in
+// bits 0-15, hi in bits 16-31.
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // max(|a|, |b|) of each BF16 half of two packed words; the sign bits of the
 // result are the XOR of the inputs' signs (mask them off before use).
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {

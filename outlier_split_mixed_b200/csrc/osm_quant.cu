@@ -61,6 +61,21 @@ __device__ __forceinline__ uint32_t smooth2(uint32_t w, float2 s) {
     return mx::bf16x2_bits(v.x, v.y);
 }
 
+// As smooth2 with the halves selected by `f16mask` (0xFFFF per half) rounded
+// to binary16 instead of BF16: the outlier slots of an FP16 outlier branch.
+__device__ __forceinline__ uint32_t smooth2_mixed(uint32_t w, float2 s, uint32_t f16mask) {
+    const float2 v = __fmul2_rn(make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)), s);
+    const uint32_t b = mx::bf16x2_bits(v.x, v.y);
+    const uint32_t h = mx::f16x2_bits(v.x, v.y);
+    return (h & f16mask) | (b & ~f16mask);
+}
+
+// Mask for smooth2_mixed: the halves whose routed offset is an outlier slot
+// (offsets from `slot0` on) when the outlier branch is FP16.
+__device__ __forceinline__ uint32_t slot_mask(int2 dv, int slot0) {
+    return (dv.x >= slot0 ? 0x0000FFFFu : 0u) | (dv.y >= slot0 ? 0xFFFF0000u : 0u);
+}
+
 // ------------------------------------------------------------ calibration
 
 constexpr int AMAX_ROWS = 32;
@@ -203,7 +218,7 @@ constexpr int PK_THREADS = 256;
 // Load rows src_row(r) of W (r < nrows; a negative row is zero), columns
 // n0 .. n0+127 (packed order: W column col_order[n] when col_order is set),
 // as w' = bf16(fp32(w) * s[row]) into tile[r][0..63] (BF16 pairs).
-template <typename RowOf>
+template <bool F16, typename RowOf>
 __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0, int nrows, RowOf src_row,
                                                  uint32_t (*tile)[64]) {
     for (int t = threadIdx.x; t < nrows * 16; t += PK_THREADS) {
@@ -223,7 +238,9 @@ __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0
                 for (int i = 0; i < 8; ++i) e[i] = p.W[j * p.N + __ldg(p.col_order + n + i)];
                 w = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
             }
-            v = make_uint4(smooth2(w.x, s2), smooth2(w.y, s2), smooth2(w.z, s2), smooth2(w.w, s2));
+            const uint32_t m = F16 ? 0xFFFFFFFFu : 0u;
+            v = make_uint4(smooth2_mixed(w.x, s2, m), smooth2_mixed(w.y, s2, m), smooth2_mixed(w.z, s2, m),
+                           smooth2_mixed(w.w, s2, m));
         }
         *reinterpret_cast<uint4*>(&tile[r][4 * c]) = v;
     }
@@ -243,7 +260,8 @@ __global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams 
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
     const int64_t p0 = static_cast<int64_t>(blockIdx.y) * 128;
     const int64_t katoms = p.Kbp / 128;
-    load_folded_rows(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; }, tile);
+    load_folded_rows<false>(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; },
+                            tile);
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,14 +325,17 @@ __global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams 
 }
 
 // Outlier channels: CTA = 64 outlier slots x 128 packed output channels;
-// w_hp[n][i] = bf16(fp32(w[O_i][n]) * s[O_i]) for i < k, 0 for k <= i < kp.
+// w_hp[n][i] = bf16(fp32(w[O_i][n]) * s[O_i]) (binary16 for an FP16 outlier
+// branch) for i < k, 0 for k <= i < kp.
 // Thread (n, 8-slot group) gathers its eight values down the tile and writes
 // them as one 16-byte store.
+template <bool F16>
 __global__ void __launch_bounds__(PK_THREADS) pack_hp_tiled_kernel(PackParams p) {
     __shared__ __align__(16) uint32_t tile[64][64];
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
     const int64_t i0 = static_cast<int64_t>(blockIdx.y) * 64;
-    load_folded_rows(p, n0, 64, [&](int r) -> int64_t { return i0 + r < p.k ? __ldg(p.O + i0 + r) : -1; }, tile);
+    load_folded_rows<F16>(p, n0, 64, [&](int r) -> int64_t { return i0 + r < p.k ? __ldg(p.O + i0 + r) : -1; },
+                          tile);
     __syncthreads();
     const uint16_t* t16 = reinterpret_cast<const uint16_t*>(&tile[0][0]);
     for (int t = threadIdx.x; t < 128 * 8; t += PK_THREADS) {
@@ -342,6 +363,7 @@ struct QuantParams {
     uint32_t* status;        // OSM_STATUS_* bits
     uint64_t wait_limit_ns;  // bound of every wait on an incoming row group
     uint32_t extra_tx;       // bytes expected beyond each group's copy (0; 16 when starved for a test)
+    int hp_fp16;             // outlier slots in binary16 instead of BF16
 };
 
 constexpr int QA_THREADS = 256;
@@ -364,7 +386,7 @@ __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * Q
 //           amax by packed u16 max, E8M0 exponent, sixteen E2M1x2
 //           conversions, one 128-bit code store and one scale byte;
 //  phase 3: the outlier slots go out as 128-bit stores.
-template <int R>
+template <int R, bool HPF>
 __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p) {
     extern __shared__ __align__(16) uint8_t sbuf[];
     const int nb = p.Kbp >> 5;
@@ -414,7 +436,8 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
             if (c < npairs) {
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const uint32_t h = smooth2(w[u][r], sv[u]);
+                    const uint32_t h = HPF ? smooth2_mixed(w[u][r], sv[u], slot_mask(dv[u], nb * QA_BLOCK_BYTES))
+                                           : smooth2(w[u][r], sv[u]);
                     *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].x) = static_cast<uint16_t>(h);
                     *reinterpret_cast<uint16_t*>(sbuf + r * stride + dv[u].y) = static_cast<uint16_t>(h >> 16);
                 }
@@ -547,7 +570,7 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 //  are encoded (encode_staged).
 // Every wait on a slot is bounded; a wait that runs out sets
 // OSM_STATUS_TIMEOUT, and the CTA lets its copies land before it returns.
-template <int R, int S, int NT, int TR>
+template <int R, int S, int NT, int TR, bool HPF>
 __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int nb = p.Kbp >> 5;
@@ -602,6 +625,7 @@ __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams 
     // the shared addresses of their routed slots (row 0) in registers
     float2 tsv[TR > 0 ? TR : 1];
     uint2 tad[TR > 0 ? TR : 1];
+    uint32_t tmask[TR > 0 ? TR : 1];  // FP16 outlier branch: halves that are outlier slots
     if constexpr (TR > 0) {
 #pragma unroll
         for (int j = 0; j < TR; ++j) {
@@ -609,6 +633,7 @@ __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams 
             tsv[j] = c < npairs ? __ldg(is2 + c) : make_float2(0.f, 0.f);
             const int2 dv = c < npairs ? __ldg(rt2 + c) : make_int2(0, 0);
             tad[j] = make_uint2(sbuf_u32 + dv.x, sbuf_u32 + dv.y);
+            tmask[j] = HPF ? slot_mask(dv, nb * QA_BLOCK_BYTES) : 0u;
         }
     }
     int issued = min(S, mine);
@@ -637,7 +662,8 @@ __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams 
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         if (r < rows) {
-                            const uint32_t h = smooth2(ptx::ld_shared_u32(src + r * row_bytes + j * NT * 4), tsv[j]);
+                            const uint32_t x = ptx::ld_shared_u32(src + r * row_bytes + j * NT * 4);
+                            const uint32_t h = HPF ? smooth2_mixed(x, tsv[j], tmask[j]) : smooth2(x, tsv[j]);
                             ptx::st_shared_u16(tad[j].x + r * stride, h);
                             ptx::st_shared_u16(tad[j].y + r * stride, h >> 16);
                         }
@@ -651,7 +677,9 @@ __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams 
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     if (r < rows) {
-                        const uint32_t h = smooth2(ptx::ld_shared_u32(src + r * row_bytes + (c - tid) * 4), sv);
+                        const uint32_t x = ptx::ld_shared_u32(src + r * row_bytes + (c - tid) * 4);
+                        const uint32_t h = HPF ? smooth2_mixed(x, sv, slot_mask(dv, nb * QA_BLOCK_BYTES))
+                                               : smooth2(x, sv);
                         ptx::st_shared_u16(sbuf_u32 + r * stride + dv.x, h);
                         ptx::st_shared_u16(sbuf_u32 + r * stride + dv.y, h >> 16);
                     }
@@ -705,7 +733,8 @@ int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* co
     }
     if (pl->kp > 0) {
         dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 128), static_cast<unsigned>(pl->kp / 64));
-        pack_hp_tiled_kernel<<<grid, PK_THREADS, 0, st>>>(p);
+        if (pl->hp_fp16) pack_hp_tiled_kernel<true><<<grid, PK_THREADS, 0, st>>>(p);
+        else pack_hp_tiled_kernel<false><<<grid, PK_THREADS, 0, st>>>(p);
         return check_cuda(cudaGetLastError(), "pack_hp launch");
     }
     return OSM_OK;
@@ -757,7 +786,7 @@ static int prepare_kernel(const void* kern, int threads, size_t smem, int* per_s
 
 template <int R>
 static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
-    auto kern = quantize_act_kernel<R>;
+    auto kern = p.hp_fp16 ? quantize_act_kernel<R, true> : quantize_act_kernel<R, false>;
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), QA_THREADS, smem, nullptr, nullptr);
     if (rc) return rc;
     const int64_t grid = ceil_div(p.M, R);
@@ -768,7 +797,7 @@ static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
 template <int R, int S, int NT, int TR>
 static int launch_stream(const QuantParams& p, int stride, cudaStream_t st) {
     const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
-    auto kern = quantize_act_stream_kernel<R, S, NT, TR>;
+    auto kern = p.hp_fp16 ? quantize_act_stream_kernel<R, S, NT, TR, true> : quantize_act_stream_kernel<R, S, NT, TR, false>;
     int per_sm = 0, sms = 0;
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
     if (rc) return rc;
@@ -785,7 +814,7 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
     QuantParams p{X, pl->d_inv_s, pl->d_route, static_cast<int>(M), static_cast<int>(pl->K),
                   static_cast<int>(pl->k), static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp),
                   static_cast<int>(pl->kp), codes, scales, hp, pl->d_status, pl->wait_limit_ns,
-                  (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u};
+                  (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u, pl->hp_fp16};
     const int stride = qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp));
     // streaming form: two CTAs of at most 110 KB per SM
     const size_t two_per_sm = 110 * 1024;

@@ -35,7 +35,8 @@ def gpu_calibrate(X: np.ndarray, W: np.ndarray, alpha: float, k: int, batches: i
     return Xd, Wd, s, inv_s, O, amax, wmax
 
 
-def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_sO=None, rows=None):
+def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_sO=None, rows=None,
+              hp_fp16=False):
     """Full CUDA path. Returns a dict of host arrays (rows of the activation
     outputs and of Y restricted to `rows` when given)."""
     M, K = X.shape
@@ -43,7 +44,7 @@ def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_
     Xd, Wd, s, inv_s, O, amax, wmax = gpu_calibrate(X, W, alpha, k, batches)
     if plan_sO is not None:
         s, O = plan_sO
-    plan = osm.Plan(K, N, k, s, O, mode)
+    plan = osm.Plan(K, N, k, s, O, mode, hp_fp16=hp_fp16)
     wc, wsc, wh = plan.alloc_packed(N)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M)
@@ -68,13 +69,13 @@ def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_
     return out
 
 
-def oracle_layer(X, W, alpha, k, mode, rows=None, bias=None):
+def oracle_layer(X, W, alpha, k, mode, rows=None, bias=None, hp_fp16=False):
     amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
     s, inv_s, O = oracle.calibrate(amax, wmax, alpha, k)
-    wc, wsc, wh = oracle.pack_weights(W, s, O, mode)
+    wc, wsc, wh = oracle.pack_weights(W, s, O, mode, hp_fp16=hp_fp16)
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
-    ac, asc, ah = oracle.quantize_act(X[rows], inv_s, O)
-    y, T = oracle.dual_gemm_rows(ac, asc, ah, np.arange(len(rows)), wc, wsc, wh, bias)
+    ac, asc, ah = oracle.quantize_act(X[rows], inv_s, O, hp_fp16=hp_fp16)
+    y, T = oracle.dual_gemm_rows(ac, asc, ah, np.arange(len(rows)), wc, wsc, wh, bias, hp_fp16=hp_fp16)
     return dict(amax=amax, wmax=wmax, s=s, inv_s=inv_s, O=O, w_codes=wc, w_scales=wsc, w_hp=wh,
                 a_codes=ac, a_scales=asc, a_hp=ah, y=y, T=T, rows=rows)
 

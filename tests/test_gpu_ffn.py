@@ -85,13 +85,14 @@ def test_fused_requant_is_bitexact_with_exact_accumulators():
     assert_bitexact("next outlier slots", to_np_u16(nh).reshape(M, nxt.kp), nh_o)
 
 
-@pytest.mark.parametrize("shape", [(512, 1024, 1536, 32, 48), (130, 512, 1024, 0, 64), (256, 512, 768, 64, 0)],
-                         ids=["partial_bulk_block", "up_k0", "next_k0"])
+@pytest.mark.parametrize("shape", [(512, 1024, 1536, 32, 48, False), (130, 512, 1024, 0, 64, False),
+                                   (256, 512, 768, 64, 0, False), (512, 1024, 1536, 32, 48, True)],
+                         ids=["partial_bulk_block", "up_k0", "next_k0", "next_fp16_outliers"])
 def test_fused_requant_equals_gelu_bf16_then_quantize(shape):
     # Realistic data: the fused epilogue must equal the unfused pipeline
     # (GELU_BF16 epilogue, then quantize_act of the next layer) bit for bit,
     # since both see the same FP32 accumulators.
-    M, K, N, k, kn = shape
+    M, K, N, k, kn, next_fp16 = shape
     X = synth.acts_heavy_tailed(M, K, seed=600 + K, frac=0.02)
     W = synth.weights_gaussian(K, N, seed=601 + K, sigma=0.04)
     Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
@@ -105,7 +106,7 @@ def test_fused_requant_equals_gelu_bf16_then_quantize(shape):
     osm.dual_gemm(up, ac, asc, ah, M, wc, wsc, wh, H, epi=osm.EPI_GELU_BF16)
     Wn = synth.weights_gaussian(N, 256, seed=602 + K, sigma=0.02)
     sn, _, On, _, _ = osm.calibrate([H], to_dev_bf16(Wn), 0.5, kn)
-    nxt = osm.Plan(N, 256, kn, sn, On, osm.WSCALE_TILE32x32)
+    nxt = osm.Plan(N, 256, kn, sn, On, osm.WSCALE_TILE32x32, hp_fp16=next_fp16)
     c1, s1, h1 = nxt.alloc_packed(M)
     osm.quantize_act(nxt, H, c1, s1, h1)
     wc2, wsc2, wh2 = up.alloc_packed(N)

@@ -59,6 +59,23 @@ def test_layer_parity_small(case):
     assert_y_close(g["Y"], o["y"], o["T"], bf16=(epi == osm.EPI_BF16))
 
 
+FP16_CASES = [c for c in SMALL if c[0] in ("tiny_cfg", "ragged_tile32", "odd_atoms_strip", "kK_pure_bf16",
+                                             "bf16_out_bias", "long_k_wraps_ring", "wide_k_staged")]
+
+
+@pytest.mark.parametrize("case", FP16_CASES, ids=[c[0] + "_fp16" for c in FP16_CASES])
+def test_layer_parity_fp16_outlier_branch(case):
+    # The FP16 outlier branch: outlier slots rounded to binary16, FP16 MMAs.
+    name, M, K, N, alpha, k, mode, epi, use_bias, x_kind = case
+    seed = 1000 + sum(map(ord, name))
+    X, W = _inputs(M, K, N, x_kind, seed)
+    bias = (np.random.default_rng(seed).standard_normal(N).astype(np.float32) * 0.1) if use_bias else None
+    g = gpu_layer(X, W, alpha, k, mode, epi=epi, bias=bias, hp_fp16=True)
+    o = oracle_layer(X, W, alpha, k, mode, bias=bias, hp_fp16=True)
+    compare_layer(g, o)
+    assert_y_close(g["Y"], o["y"], o["T"], bf16=(epi == osm.EPI_BF16))
+
+
 def test_tiny_config_exact_shapes():
     cfg = synth.TINY
     X, W = cfg.make_x(), cfg.make_w()
