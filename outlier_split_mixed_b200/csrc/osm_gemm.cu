@@ -200,23 +200,23 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
     for (int j = 0; j < 16; ++j) {
         const int64_t col = col0 + 8 * j + cq;
         if (col >= p.N) break;
-        float a0 = __uint_as_float(r[4 * j]), a1 = __uint_as_float(r[4 * j + 1]);
-        float b0 = __uint_as_float(r[4 * j + 2]), b1 = __uint_as_float(r[4 * j + 3]);
+        float2 a = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
+        float2 b = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
         if (p.bias) {
             const float2 bb = __ldg(reinterpret_cast<const float2*>(p.bias + col));
-            a0 += bb.x; a1 += bb.y; b0 += bb.x; b1 += bb.y;
+            a = __fadd2_rn(a, bb);
+            b = __fadd2_rn(b, bb);
         }
         if constexpr (EPI == OSM_EPI_GELU_BF16) {
-            a0 = mx::gelu_tanh(a0); a1 = mx::gelu_tanh(a1);
-            b0 = mx::gelu_tanh(b0); b1 = mx::gelu_tanh(b1);
+            a = mx::gelu_tanh2(a);
+            b = mx::gelu_tanh2(b);
         }
         if constexpr (EPI == OSM_EPI_F32) {
-            if (ra < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + ra * p.N + col) = make_float2(a0, a1);
-            if (rb < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + rb * p.N + col) = make_float2(b0, b1);
+            if (ra < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + ra * p.N + col) = a;
+            if (rb < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + rb * p.N + col) = b;
         } else {
-            const __nv_bfloat162 ha = __floats2bfloat162_rn(a0, a1), hb = __floats2bfloat162_rn(b0, b1);
-            if (ra < p.M) *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(p.Y) + ra * p.N + col) = ha;
-            if (rb < p.M) *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(p.Y) + rb * p.N + col) = hb;
+            if (ra < p.M) *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.Y) + ra * p.N + col) = mx::bf16x2_bits(a.x, a.y);
+            if (rb < p.M) *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.Y) + rb * p.N + col) = mx::bf16x2_bits(b.x, b.y);
         }
     }
 }
@@ -251,20 +251,33 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
         }
         return;
     }
-    uint32_t hw[16];  // x' as BF16 pairs, element 2i in the low half of word i
+    // x' = round(bf16(GELU(acc)) * inv_s) as pairs, element 2i in the low
+    // half of word i: BF16 for the bulk columns; for an FP16 outlier branch
+    // of the next layer, binary16 in the columns from nKb on (the same
+    // product, rounded to the other format)
+    const bool f16_tail = p.next_hp_fp16 && c0 + 32 > p.nKb;  // uniform across the warp
+    const int d = static_cast<int>(c0 - p.nKb);
+    uint32_t hw[16];
     const float4* iv = reinterpret_cast<const float4*>(p.inv_s_ord + c0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float4 sv = __ldg(iv + i);
-        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
-        uint32_t xs[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t hb = mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])));
-            xs[j] = mx::f32_to_bf16_bits(__fmul_rn(mx::bf16_bits_to_f32(hb), s4[j]));
+        const float2 g0 = mx::gelu_tanh2(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])));
+        const float2 g1 = mx::gelu_tanh2(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+        const uint32_t h0 = mx::bf16x2_bits(g0.x, g0.y), h1 = mx::bf16x2_bits(g1.x, g1.y);
+        const float2 x0 = __fmul2_rn(make_float2(__uint_as_float(h0 << 16), __uint_as_float(h0 & 0xFFFF0000u)),
+                                     make_float2(sv.x, sv.y));
+        const float2 x1 = __fmul2_rn(make_float2(__uint_as_float(h1 << 16), __uint_as_float(h1 & 0xFFFF0000u)),
+                                     make_float2(sv.z, sv.w));
+        hw[2 * i] = mx::bf16x2_bits(x0.x, x0.y);
+        hw[2 * i + 1] = mx::bf16x2_bits(x1.x, x1.y);
+        if (f16_tail) {
+            const int o = d + 4 * i;  // column of element 4i, relative to nKb
+            const uint32_t m0 = (o >= 0 ? 0x0000FFFFu : 0u) | (o + 1 >= 0 ? 0xFFFF0000u : 0u);
+            const uint32_t m1 = (o + 2 >= 0 ? 0x0000FFFFu : 0u) | (o + 3 >= 0 ? 0xFFFF0000u : 0u);
+            hw[2 * i] = (hw[2 * i] & ~m0) | (mx::f16x2_bits(x0.x, x0.y) & m0);
+            hw[2 * i + 1] = (hw[2 * i + 1] & ~m1) | (mx::f16x2_bits(x1.x, x1.y) & m1);
         }
-        hw[2 * i] = xs[0] | (xs[1] << 16);
-        hw[2 * i + 1] = xs[2] | (xs[3] << 16);
     }
     if (c0 < p.nKb) {
         const int nreal = static_cast<int>(p.nKb - c0 < 32 ? p.nKb - c0 : 32);
@@ -294,24 +307,7 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
         }
     }
     if (c0 + 32 > p.nKb) {
-        // outlier part: columns max(c0, nKb) .. c0+31 -> slots c - nKb; for an
-        // FP16 outlier branch of the next layer the same products
-        // bf16(GELU(acc)) * inv_s, rounded to binary16 instead
-        if (p.next_hp_fp16) {
-            const float4* iv = reinterpret_cast<const float4*>(p.inv_s_ord + c0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 sv = __ldg(iv + i);
-                const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
-                float pr[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    pr[j] = __fmul_rn(mx::bf16_bits_to_f32(mx::f32_to_bf16_bits(mx::gelu_tanh(__uint_as_float(r[4 * i + j])))),
-                                      s4[j]);
-                hw[2 * i] = mx::f16x2_bits(pr[0], pr[1]);
-                hw[2 * i + 1] = mx::f16x2_bits(pr[2], pr[3]);
-            }
-        }
+        // outlier part: columns max(c0, nKb) .. c0+31 -> slots c - nKb
         uint16_t* hp = p.next_hp + row * p.nkp;
         if (c0 >= p.nKb && ((c0 - p.nKb) & 7) == 0) {
             uint4* dst = reinterpret_cast<uint4*>(hp + (c0 - p.nKb));

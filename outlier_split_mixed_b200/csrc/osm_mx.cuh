@@ -109,6 +109,14 @@ __device__ __forceinline__ uint32_t encode8_words(uint32_t w0, uint32_t w1, uint
     return out;
 }
 
+// The GELU below works on two values at once with the packed FP32
+// instructions of sm_100 (fma / mul / add .rn.f32x2): each lane of a packed
+// operation is one IEEE operation rounded to nearest even, so every element
+// goes through exactly the operations of the scalar definition, in the same
+// order, at half the instruction count. Negated operands are written as
+// negated constants (x (-c) = (-x) c exactly).
+__device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
+
 // exp(a) for a <= 0 in FP32: a clamped to -100, Cody-Waite reduction
 // a = n ln2 + r with ln2 split into a 12-bit high part and a low remainder,
 // the degree-7 Taylor polynomial of exp(r) in Horner form with fused
@@ -118,33 +126,34 @@ __device__ __forceinline__ uint32_t encode8_words(uint32_t w0, uint32_t w1, uint
 // and the factor 2^n is built from bits (an exponent field clamped at 0
 // gives the factor 0). Every operation is an explicitly rounded intrinsic so
 // that no contraction or reassociation changes the result.
-__device__ __forceinline__ float gelu_exp_neg(float a) {
-    const float ac = fmaxf(a, -100.0f);
-    const float t = __fmaf_rn(ac, 0x1.715476p+0f, 0x1.8p+23f);
-    const float n = __fsub_rn(t, 0x1.8p+23f);
-    float r = __fmaf_rn(-n, 0x1.62e4p-1f, ac);
-    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);
-    float p = 0x1.a01a02p-13f;
-    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
-    p = __fmaf_rn(p, r, 0x1.111112p-7f);
-    p = __fmaf_rn(p, r, 0x1.555556p-5f);
-    p = __fmaf_rn(p, r, 0x1.555556p-3f);
-    p = __fmaf_rn(p, r, 0.5f);
-    p = __fmaf_rn(p, r, 1.0f);
-    p = __fmaf_rn(p, r, 1.0f);
+__device__ __forceinline__ float2 gelu_exp_neg2(float2 a) {
+    const float2 ac = make_float2(fmaxf(a.x, -100.0f), fmaxf(a.y, -100.0f));
+    const float2 t = __ffma2_rn(ac, splat2(0x1.715476p+0f), splat2(0x1.8p+23f));
+    const float2 n = __fadd2_rn(t, splat2(-0x1.8p+23f));
+    float2 r = __ffma2_rn(n, splat2(-0x1.62e4p-1f), ac);
+    r = __ffma2_rn(n, splat2(-0x1.7f7d1cp-20f), r);
+    float2 q = __ffma2_rn(splat2(0x1.a01a02p-13f), r, splat2(0x1.6c16c2p-10f));
+    q = __ffma2_rn(q, r, splat2(0x1.111112p-7f));
+    q = __ffma2_rn(q, r, splat2(0x1.555556p-5f));
+    q = __ffma2_rn(q, r, splat2(0x1.555556p-3f));
+    q = __ffma2_rn(q, r, splat2(0.5f));
+    q = __ffma2_rn(q, r, splat2(1.0f));
+    q = __ffma2_rn(q, r, splat2(1.0f));
     // t = 1.5*2^23 + n with n in [-145, 0]: its bit pattern is that of 1.5*2^23 plus n
-    const int e = max(static_cast<int>(__float_as_uint(t) - 0x4B400000u) + 127, 0);
-    return __fmul_rn(p, __uint_as_float(static_cast<uint32_t>(e) << 23));
+    const int ex = max(static_cast<int>(__float_as_uint(t.x) - 0x4B400000u) + 127, 0);
+    const int ey = max(static_cast<int>(__float_as_uint(t.y) - 0x4B400000u) + 127, 0);
+    return __fmul2_rn(q, make_float2(__uint_as_float(static_cast<uint32_t>(ex) << 23),
+                                     __uint_as_float(static_cast<uint32_t>(ey) << 23)));
 }
 
-// 1/d for d in [1, 2]: linear seed 24/17 - (8/17) d, then three Newton
-// steps y <- y + y (1 - d y) as two fused multiply-adds each.
-__device__ __forceinline__ float gelu_recip(float d) {
-    float y = __fmaf_rn(-0x1.e1e1e2p-2f, d, 0x1.69696ap+0f);
+// 1/d for d in [1, 2], given nd = -d: linear seed 24/17 - (8/17) d, then
+// three Newton steps y <- y + y (1 - d y) as two fused multiply-adds each.
+__device__ __forceinline__ float2 gelu_recip2_neg(float2 nd) {
+    float2 y = __ffma2_rn(splat2(0x1.e1e1e2p-2f), nd, splat2(0x1.69696ap+0f));
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
-        const float e = __fmaf_rn(-d, y, 1.0f);
-        y = __fmaf_rn(y, e, y);
+        const float2 e = __ffma2_rn(nd, y, splat2(1.0f));
+        y = __ffma2_rn(y, e, y);
     }
     return y;
 }
@@ -152,18 +161,18 @@ __device__ __forceinline__ float gelu_recip(float d) {
 // GELU_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), for
 // finite x, through 0.5 (1 + tanh(u)) = sigma(2u): with E = exp(-2|u|),
 // x sigma(2u) = x/(1+E) for u >= 0 and x E/(1+E) for u < 0; u has the sign
-// of x and 0 <= E <= 1, so the numerator is max(x, x E). Operations in this
-// order: x2 = x x; k = fma(C1, x2, 1); u = (C0 x) k; E; y = recip(1 + E);
-// max(x, x E) y. No division, no branch.
-__device__ __forceinline__ float gelu_tanh(float x) {
-    const float C0 = 0x1.988454p-1f;  // sqrt(2/pi)
-    const float C1 = 0x1.6e4e26p-5f;  // 0.044715
-    const float x2 = __fmul_rn(x, x);
-    const float k = __fmaf_rn(C1, x2, 1.0f);
-    const float u = __fmul_rn(__fmul_rn(C0, x), k);
-    const float E = gelu_exp_neg(__fmul_rn(-2.0f, fabsf(u)));
-    const float y = gelu_recip(__fadd_rn(1.0f, E));
-    return __fmul_rn(fmaxf(x, __fmul_rn(x, E)), y);
+// of x and 0 <= E <= 1, so the numerator is max(x, x E). Operations per
+// element in this order: x2 = x x; k = fma(C1, x2, 1); u = (C0 x) k; E; y =
+// recip(1 + E) (1 + E formed as -(1 + E) = fma(E, -1, -1), the same rounding
+// with the sign flipped); max(x, x E) y. No division, no branch.
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+    const float2 x2 = __fmul2_rn(x, x);
+    const float2 k = __ffma2_rn(splat2(0x1.6e4e26p-5f), x2, splat2(1.0f));    // C1 = 0.044715
+    const float2 u = __fmul2_rn(__fmul2_rn(splat2(0x1.988454p-1f), x), k);   // C0 = sqrt(2/pi)
+    const float2 E = gelu_exp_neg2(__fmul2_rn(make_float2(fabsf(u.x), fabsf(u.y)), splat2(-2.0f)));
+    const float2 y = gelu_recip2_neg(__ffma2_rn(E, splat2(-1.0f), splat2(-1.0f)));
+    const float2 xE = __fmul2_rn(x, E);
+    return __fmul2_rn(make_float2(fmaxf(x.x, xE.x), fmaxf(x.y, xE.y)), y);
 }
 
 // Byte offset of E8M0 scale (row r, 32-block b) in the tcgen05 block-scale
