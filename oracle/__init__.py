@@ -15,8 +15,10 @@ Pinned functions (see tests/test_oracle_*.py): BF16 rounding, E2M1 codec,
 MX scale exponent, calibration (Eq. (2), Eq. (4), the tail-aware percentile
 score), smoothing/folding
 (Eq. (1)), quantize_act, pack_weights (all three block-scale modes),
-dual_gemm_rows (Eq. (5)). The FP32 tanh-form GELU is pinned only to libm
-within an error bound ("parity unpinned" for its exact bits).
+dual_gemm_rows (Eq. (5)), and the NVFP4 forms (E4M3 codec, block scale,
+element multiplier, per-tensor exponent, quantize_act_nv, pack_weights_nv,
+dual_gemm_rows_nv). The FP32 tanh-form GELU is pinned only to libm within an
+error bound ("parity unpinned" for its exact bits).
 """
 from __future__ import annotations
 
@@ -94,6 +96,21 @@ def _load():
             lib.oracle_gelu_recip.restype = ctypes.c_float
             lib.oracle_gelu_recip.argtypes = [ctypes.c_float]
             lib.oracle_gelu_bf16_rows.argtypes = [P, I64, P]
+            lib.oracle_e4m3_decode.restype = ctypes.c_double
+            lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_encode_satfinite.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode_satfinite.argtypes = [ctypes.c_float]
+            lib.oracle_nvfp4_tensor_exponent.restype = ctypes.c_int
+            lib.oracle_nvfp4_tensor_exponent.argtypes = [ctypes.c_double]
+            lib.oracle_nvfp4_scale.restype = ctypes.c_uint8
+            lib.oracle_nvfp4_scale.argtypes = [ctypes.c_double, ctypes.c_int]
+            lib.oracle_nvfp4_recip.restype = ctypes.c_float
+            lib.oracle_nvfp4_recip.argtypes = [ctypes.c_uint8, ctypes.c_int]
+            lib.oracle_nvfp4_plan_exponents.argtypes = [P, P, P, P, P, I64, I64, P, P]
+            lib.oracle_quantize_act_nv.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P, P, P]
+            lib.oracle_pack_weights_nv.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P, P, P]
+            lib.oracle_dual_gemm_rows_nv.argtypes = [P, P, P, P, I64, P, P, P, I64, I64, I64, ctypes.c_int,
+                                                     ctypes.c_int, P, P, P]
             _lib = lib
     return _lib
 
@@ -318,4 +335,94 @@ def dual_gemm_rows(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, bias=
     _load().oracle_dual_gemm_rows_ex(_p(a_codes), _p(a_scales), _p(a_hp), _p(rows), rows.shape[0],
                                      _p(w_codes), _p(w_scales), _p(w_hp), N, Kbp, kpp, bptr,
                                      _p(y), _p(T), int(bool(hp_fp16)))
+    return y, T
+
+
+# ---- NVFP4 ---------------------------------------------------------------
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(f: float) -> int:
+    """Nearest E4M3 code (ties to even), saturating at 448."""
+    return int(_load().oracle_e4m3_encode_satfinite(float(np.float32(f))))
+
+
+def nvfp4_tensor_exponent(amax: float) -> int:
+    return int(_load().oracle_nvfp4_tensor_exponent(float(amax)))
+
+
+def nvfp4_scale(amax: float, g: int) -> int:
+    return int(_load().oracle_nvfp4_scale(float(amax), int(g)))
+
+
+def nvfp4_recip(S: int, g: int) -> float:
+    return float(_load().oracle_nvfp4_recip(int(S), int(g)))
+
+
+def nvfp4_plan_exponents(amax, wmax, s, inv_s, O):
+    """(g_act, g_w) of a plan from its calibration statistics."""
+    amax, wmax = _c(amax, np.float32), _c(wmax, np.float32)
+    s, inv_s = _c(s, np.float32), _c(inv_s, np.float32)
+    O = _c(O, np.int32)
+    K, k = amax.shape[0], O.shape[0]
+    ga, gw = ctypes.c_int(0), ctypes.c_int(0)
+    Op = O if k else np.zeros(1, np.int32)
+    _load().oracle_nvfp4_plan_exponents(_p(amax), _p(wmax), _p(s), _p(inv_s), _p(Op), K, k,
+                                        ctypes.byref(ga), ctypes.byref(gw))
+    return ga.value, gw.value
+
+
+def quantize_act_nv(X: np.ndarray, inv_s: np.ndarray, O: np.ndarray, g_act: int):
+    """NVFP4 activations: (codes [M][Kbp/2], scales [M][Kbp/16] logical UE4M3, a_hp [M][kp])."""
+    X = _c(X, np.uint16)
+    inv_s = _c(inv_s, np.float32)
+    O = _c(O, np.int32)
+    M, K = X.shape
+    k = O.shape[0]
+    Kbp, kpp = kbp(K, k), kp(k)
+    codes = np.zeros((M, Kbp // 2), np.uint8)
+    scales = np.zeros((M, Kbp // 16), np.uint8)
+    a_hp = np.zeros((M, kpp), np.uint16)
+    Op = O if k else np.zeros(1, np.int32)
+    _load().oracle_quantize_act_nv(_p(X), M, K, k, _p(inv_s), _p(Op), int(g_act), _p(codes), _p(scales), _p(a_hp))
+    return codes, scales, a_hp
+
+
+def pack_weights_nv(W: np.ndarray, s: np.ndarray, O: np.ndarray, g_w: int):
+    """NVFP4 weights: (codes [N][Kbp/2], scales [N][Kbp/16] logical UE4M3, w_hp [N][kp])."""
+    W = _c(W, np.uint16)
+    s = _c(s, np.float32)
+    O = _c(O, np.int32)
+    K, N = W.shape
+    k = O.shape[0]
+    Kbp, kpp = kbp(K, k), kp(k)
+    codes = np.zeros((N, Kbp // 2), np.uint8)
+    scales = np.zeros((N, Kbp // 16), np.uint8)
+    w_hp = np.zeros((N, kpp), np.uint16)
+    Op = O if k else np.zeros(1, np.int32)
+    _load().oracle_pack_weights_nv(_p(W), K, N, k, _p(s), _p(Op), int(g_w), _p(codes), _p(scales), _p(w_hp))
+    return codes, scales, w_hp
+
+
+def dual_gemm_rows_nv(a_codes, a_scales, a_hp, rows, w_codes, w_scales, w_hp, g_act, g_w, bias=None):
+    """Eq. (5) with NVFP4 operands. Returns (y [r][N] f64, T [r][N] f64)."""
+    a_codes, a_scales, a_hp = _c(a_codes, np.uint8), _c(a_scales, np.uint8), _c(a_hp, np.uint16)
+    w_codes, w_scales, w_hp = _c(w_codes, np.uint8), _c(w_scales, np.uint8), _c(w_hp, np.uint16)
+    rows = _c(rows, np.int64)
+    N = w_codes.shape[0]
+    Kbp = w_codes.shape[1] * 2
+    kpp = w_hp.shape[1]
+    assert a_codes.shape[1] * 2 == Kbp and a_hp.shape[1] == kpp
+    assert a_scales.shape[1] == Kbp // 16 and w_scales.shape[1] == Kbp // 16
+    y = np.empty((rows.shape[0], N), np.float64)
+    T = np.empty((rows.shape[0], N), np.float64)
+    bptr = None
+    if bias is not None:
+        bias = _c(bias, np.float32)
+        bptr = _p(bias)
+    _load().oracle_dual_gemm_rows_nv(_p(a_codes), _p(a_scales), _p(a_hp), _p(rows), rows.shape[0],
+                                     _p(w_codes), _p(w_scales), _p(w_hp), N, Kbp, kpp, int(g_act), int(g_w),
+                                     bptr, _p(y), _p(T))
     return y, T

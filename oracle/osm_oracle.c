@@ -24,6 +24,9 @@
  *     positions hold code 0 / BF16 zero, and a 32-block with no real
  *     element gets scale code 0.
  *
+ * NVFP4 (a second 4-bit block format on the same dual product) has its
+ * own section at the end of the file.
+ *
  * Parity pins: see tests/test_oracle_*.py. Every function below is pinned
  * except the tanh-form GELU, which is pinned only against libm's tanh
  * within a stated error bound.
@@ -670,4 +673,254 @@ float oracle_gelu_tanh_f32(float x)
 void oracle_gelu_bf16_rows(const double* y, int64_t n, uint16_t* h)
 {
     for (int64_t i = 0; i < n; ++i) h[i] = oracle_f32_to_bf16(oracle_gelu_tanh_f32((float)y[i]));
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4: E2M1 elements, one UE4M3 scale per 16, a per-tensor 2^g      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The pages ask for other 4-bit block formats on the same dual product
+ * (Sec. "Implementation" of "W4A4 Quantization for Inference on
+ * Wan2.2-I2V-A14B" names block formats as the thing to explore). NVFP4
+ * as read here:
+ *   - elements E2M1 (the same codec as MXFP4), blocks of 16 consecutive
+ *     compacted bulk positions;
+ *   - one scale per block in unsigned FP8 E4M3 (bias 7, 3 mantissa bits,
+ *     largest finite 448, no infinities);
+ *   - one power-of-two factor 2^g per tensor, g the smallest integer in
+ *     [-100, 100] with tensor amax <= 6 * 448 * 2^g (g = 0 for amax 0), so
+ *     that the largest block scale fits E4M3;
+ *   - block scale S = E4M3_RNE_satfinite(fp32(amax_b * k)), k = fp32(1/6) * 2^-g;
+ *   - element code = E2M1_RNE_sat(fp32(x * R)), R = fp32(1 / (S * 2^g))
+ *     (R = 0 when S = 0: the block encodes as signed zeros);
+ *   - decoded element = e2m1 * S * 2^g;
+ *   - the BF16 outlier branch shares the accumulator, so its stored
+ *     operands carry 2^-g: a_hp = bf16(fp32(x' * 2^-g_a)) and
+ *     w_hp = bf16(fp32(w' * 2^-g_w)), and the product is multiplied by
+ *     2^(g_a + g_w) after accumulation.
+ */
+
+/* E4M3 code -> value (sign, 4-bit exponent bias 7, 3-bit mantissa;
+ * exponent field 0 is subnormal 2^-6 * m/8; S.1111.111 is NaN). */
+double oracle_e4m3_decode(uint8_t code)
+{
+    int sign = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) v = NAN;
+    else if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(8.0 + m, e - 10);
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 value to f, ties to the even code (mantissa LSB 0),
+ * magnitudes above 448 (and infinities) saturate to 448, NaN -> 0x7F.
+ * Written as a search over all 127 finite non-negative codes. */
+uint8_t oracle_e4m3_encode_satfinite(float f)
+{
+    if (isnan(f)) return 0x7Fu;
+    uint8_t sign = signbit(f) ? 0x80u : 0u;
+    double a = fabs((double)f);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);
+    int best = 0;
+    double bestd = a;
+    for (int c = 1; c < 127; ++c) {
+        double d = fabs(a - oracle_e4m3_decode((uint8_t)c));
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* Smallest g in [-100, 100] with amax <= 2688 * 2^g (2688 = 6 * 448); 0 for
+ * amax 0. amax must be finite and non-negative. */
+int oracle_nvfp4_tensor_exponent(double amax)
+{
+    if (!(amax > 0.0)) return 0;
+    int g = -100;
+    while (g < 100 && amax > ldexp(2688.0, g)) ++g;
+    return g;
+}
+
+/* fp32(1/6) * 2^-g, exact (a power-of-two scaling of a normal number). */
+static float nvfp4_k(int g) { return (float)ldexp((double)(float)(1.0 / 6.0), -g); }
+
+/* Block scale code for a block maximum amax (a BF16 value). */
+uint8_t oracle_nvfp4_scale(double amax, int g)
+{
+    float sc = (float)(amax * (double)nvfp4_k(g));   /* exact product, one rounding to FP32 */
+    return oracle_e4m3_encode_satfinite(sc);
+}
+
+/* Element multiplier R = fp32(1 / (S * 2^g)) for scale code S, 0 for S = 0. */
+float oracle_nvfp4_recip(uint8_t S, int g)
+{
+    double D = oracle_e4m3_decode(S) * ldexp(1.0, g);
+    if (!(D > 0.0)) return 0.0f;
+    return (float)(1.0 / D);
+}
+
+/* Encode n BF16 values with scale code S (multiplier R). */
+static void nv_encode_values(const uint16_t* v16, int n, uint8_t S, int g, uint8_t* codes)
+{
+    float R = oracle_nvfp4_recip(S, g);
+    for (int i = 0; i < n; ++i) {
+        double v = oracle_bf16_to_f64(v16[i]);
+        float q = (float)(v * (double)R);             /* exact product, one rounding */
+        codes[i] = oracle_e2m1_encode((double)q, (v16[i] & 0x8000u) != 0);
+    }
+}
+
+/* bf16(fp32(h * 2^-g)) for a BF16 value h. */
+static uint16_t nv_hp_scaled(uint16_t h, int g)
+{
+    return oracle_f32_to_bf16((float)ldexp(oracle_bf16_to_f64(h), -g));
+}
+
+/*
+ * Per-tensor exponents of a plan from its calibration: the activations'
+ * tensor amax is max over bulk channels of bf16(fp32(amax_j * inv_s_j))
+ * (the largest smoothed calibration value: both roundings are monotone),
+ * the weights' is max over bulk channels of bf16(fp32(wmax_j * s_j)).
+ */
+void oracle_nvfp4_plan_exponents(const float* amax, const float* wmax, const float* s, const float* inv_s,
+                                 const int32_t* O, int64_t K, int64_t k, int* g_act, int* g_w)
+{
+    char* is_out = (char*)calloc((size_t)(K > 0 ? K : 1), 1);
+    for (int64_t i = 0; i < k; ++i) is_out[O[i]] = 1;
+    double am = 0.0, wm = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+        if (is_out[j]) continue;
+        double a = fabs(oracle_bf16_to_f64(oracle_f32_to_bf16(amax[j] * inv_s[j])));
+        double w = fabs(oracle_bf16_to_f64(oracle_f32_to_bf16(wmax[j] * s[j])));
+        if (a > am) am = a;
+        if (w > wm) wm = w;
+    }
+    free(is_out);
+    *g_act = oracle_nvfp4_tensor_exponent(am);
+    *g_w = oracle_nvfp4_tensor_exponent(wm);
+}
+
+/* One row of bulk values (BF16, compacted, Kb real of Kbp) -> codes
+ * [Kbp/2] and logical scales [Kbp/16]. */
+static void nv_encode_row(const uint16_t* bulk, int64_t Kb, int64_t Kbp, int g, uint8_t* codes, uint8_t* scales)
+{
+    uint8_t c4[16];
+    for (int64_t b = 0; b < Kbp / 16; ++b) {
+        int64_t p0 = 16 * b;
+        int n_real = (int)(p0 >= Kb ? 0 : (Kb - p0 < 16 ? Kb - p0 : 16));
+        double amax = 0.0;
+        for (int i = 0; i < n_real; ++i) {
+            double a = fabs(oracle_bf16_to_f64(bulk[p0 + i]));
+            if (a > amax) amax = a;
+        }
+        uint8_t S = n_real ? oracle_nvfp4_scale(amax, g) : 0;
+        scales[b] = S;
+        memset(c4, 0, sizeof c4);
+        nv_encode_values(bulk + p0, n_real, S, g, c4);
+        for (int i = 0; i < 8; ++i) codes[p0 / 2 + i] = (uint8_t)(c4[2 * i] | (c4[2 * i + 1] << 4));
+    }
+}
+
+/* quantize_act in NVFP4: as the MXFP4 form, with 16-blocks, UE4M3 scales
+ * (logical [M][Kbp/16]) and the outlier slots scaled by 2^-g_act. */
+void oracle_quantize_act_nv(const uint16_t* X, int64_t M, int64_t K, int64_t k, const float* inv_s,
+                            const int32_t* O, int g_act, uint8_t* codes, uint8_t* scales, uint16_t* a_hp)
+{
+    int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
+    int32_t* J = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K > 0 ? K : 1));
+    int64_t Kb = build_J(O, K, k, J);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t) {
+        uint16_t* row = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(K > 0 ? K : 1));
+        uint16_t* bulk = (uint16_t*)calloc((size_t)(Kbp > 0 ? Kbp : 1), sizeof(uint16_t));
+        for (int64_t j = 0; j < K; ++j) {
+            float p = oracle_bf16_to_f32(X[t * K + j]) * inv_s[j];
+            row[j] = oracle_f32_to_bf16(p);
+        }
+        for (int64_t i = 0; i < kp; ++i) a_hp[t * kp + i] = i < k ? nv_hp_scaled(row[O[i]], g_act) : 0;
+        for (int64_t p = 0; p < Kb; ++p) bulk[p] = row[J[p]];
+        nv_encode_row(bulk, Kb, Kbp, g_act, codes + t * (Kbp / 2), scales + t * (Kbp / 16));
+        free(bulk);
+        free(row);
+    }
+    free(J);
+}
+
+/* pack_weights in NVFP4: folded weights w', 16-blocks along the compacted
+ * bulk index of each output channel, w_hp scaled by 2^-g_w. */
+void oracle_pack_weights_nv(const uint16_t* W, int64_t K, int64_t N, int64_t k, const float* s,
+                            const int32_t* O, int g_w, uint8_t* codes, uint8_t* scales, uint16_t* w_hp)
+{
+    int64_t Kbp = oracle_kbp(K, k), kp = oracle_kp(k);
+    int32_t* J = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K > 0 ? K : 1));
+    int64_t Kb = build_J(O, K, k, J);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        uint16_t* bulk = (uint16_t*)calloc((size_t)(Kbp > 0 ? Kbp : 1), sizeof(uint16_t));
+        for (int64_t i = 0; i < kp; ++i) {
+            if (i >= k) { w_hp[n * kp + i] = 0; continue; }
+            float p = oracle_bf16_to_f32(W[(int64_t)O[i] * N + n]) * s[O[i]];
+            w_hp[n * kp + i] = nv_hp_scaled(oracle_f32_to_bf16(p), g_w);
+        }
+        for (int64_t p = 0; p < Kb; ++p) {
+            float v = oracle_bf16_to_f32(W[(int64_t)J[p] * N + n]) * s[J[p]];
+            bulk[p] = oracle_f32_to_bf16(v);
+        }
+        nv_encode_row(bulk, Kb, Kbp, g_w, codes + n * (Kbp / 2), scales + n * (Kbp / 16));
+        free(bulk);
+    }
+    free(J);
+}
+
+/* Eq. (5) with NVFP4 operands: y = 2^(g_a + g_w) * (sum_b Sa Sw sum e2m1 e2m1
+ * + sum a_hp w_hp) (+ bias); T the same over absolute values of every term
+ * (times 2^(g_a + g_w)). Every term is exact in FP64. */
+void oracle_dual_gemm_rows_nv(const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
+                              const int64_t* rows, int64_t nrows,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
+                              int64_t N, int64_t Kbp, int64_t kp, int g_act, int g_w, const float* bias,
+                              double* y, double* T)
+{
+    int64_t nb = Kbp / 16;
+    double f = ldexp(1.0, g_act + g_w);
+    double* wd = (double*)malloc(sizeof(double) * (size_t)(N * (Kbp > 0 ? Kbp : 1)));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t p = 0; p < Kbp; ++p) {
+            uint8_t byte = w_codes[n * (Kbp / 2) + p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15u);
+            wd[n * Kbp + p] = oracle_e2m1_decode(c) * oracle_e4m3_decode(w_scales[n * nb + p / 16]);
+        }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows[r];
+        double* ad = (double*)malloc(sizeof(double) * (size_t)(Kbp > 0 ? Kbp : 1));
+        for (int64_t p = 0; p < Kbp; ++p) {
+            uint8_t byte = a_codes[t * (Kbp / 2) + p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15u);
+            ad[p] = oracle_e2m1_decode(c) * oracle_e4m3_decode(a_scales[t * nb + p / 16]);
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t p = 0; p < Kbp; ++p) {
+                double term = ad[p] * wd[n * Kbp + p];
+                acc += term;
+                mag += fabs(term);
+            }
+            for (int64_t i = 0; i < kp; ++i) {
+                double term = oracle_bf16_to_f64(a_hp[t * kp + i]) * oracle_bf16_to_f64(w_hp[n * kp + i]);
+                acc += term;
+                mag += fabs(term);
+            }
+            acc *= f;
+            if (bias) acc += (double)bias[n];
+            y[r * N + n] = acc;
+            T[r * N + n] = mag * f;
+        }
+        free(ad);
+    }
+    free(wd);
 }
