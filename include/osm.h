@@ -157,7 +157,8 @@ OSM_API int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host
 OSM_API int osm_plan_destroy(osm_plan* plan);
 
 /* Bytes of the packed buffers for `rows` rows (activations: rows = M;
- * weights: rows = N). scales_bytes includes the padding to 128 rows. */
+ * weights: rows = N). scales_bytes includes the padding to 128 rows
+ * (Kbp/32 bytes per row for MXFP4, Kbp/16 for NVFP4). */
 OSM_API int osm_plan_sizes(const osm_plan* plan, int64_t rows, size_t* codes_bytes, size_t* scales_bytes,
                    size_t* hp_bytes);
 
@@ -186,6 +187,50 @@ OSM_API int osm_plan_set_wait_limit(osm_plan* plan, uint64_t ns);
 #define OSM_HP_BF16 0
 #define OSM_HP_FP16 1
 OSM_API int osm_plan_set_outlier_dtype(osm_plan* plan, int dtype);
+
+/* ---- second 4-bit block format: NVFP4 --------------------------------------
+ * The implementation paragraph of "W4A4 Quantization for Inference on
+ * Wan2.2-I2V-A14B" leaves the block format of the W4A4 bulk path open to
+ * exploration. OSM_FMT_MXFP4 (default) is the OCP MXFP4 path described
+ * above. OSM_FMT_NVFP4 runs the same dual product with:
+ *   - E2M1 elements in blocks of 16 consecutive compacted bulk positions;
+ *   - one unsigned E4M3 scale per block (bias 7, 3 mantissa bits, largest
+ *     448), laid out like the E8M0 scales (128 x 4 atoms: four 16-blocks
+ *     per atom row), so a scales buffer holds Kbp/16 bytes per padded row;
+ *   - one power-of-two factor per tensor, 2^g_act for activations and 2^g_w
+ *     for weights (see osm_nvfp4_tensor_exponent);
+ *   - block scale S = E4M3_RNE_satfinite(fp32(amax_b * k)), k = fp32(1/6) *
+ *     2^-g; element code = E2M1_RNE_sat(fp32(x * R)), R = fp32(1 / (S * 2^g))
+ *     (R = 0 for S = 0, the block then encodes as signed zeros); the decoded
+ *     element is e2m1 * S * 2^g;
+ *   - the BF16 outlier branch shares the accumulator, so its stored operands
+ *     carry the inverse factors: a_hp = bf16(fp32(x' * 2^-g_act)), w_hp =
+ *     bf16(fp32(w' * 2^-g_w)); the epilogue multiplies the accumulator by
+ *     2^(g_act + g_w) (exact) before the bias.
+ * Requirements: the plan's weight scale mode is OSM_WSCALE_1x32 (read as one
+ * scale per 16-block of each output channel), its outlier branch BF16, and
+ * -100 <= g <= 100 with |g_act + g_w| <= 126. OSM_EPI_GELU_REQUANT needs
+ * both plans in MXFP4. Set the
+ * format before packing or quantising; data packed under the other format
+ * must not be used. */
+#define OSM_FMT_MXFP4 0
+#define OSM_FMT_NVFP4 1
+OSM_API int osm_plan_set_format(osm_plan* plan, int format, int g_act, int g_w);
+
+/* Host-only: the per-tensor exponent for a tensor maximum amax (finite,
+ * >= 0): the smallest g in [-100, 100] with amax <= 6 * 448 * 2^g, so that
+ * the largest block scale fits E4M3; 0 for amax == 0. */
+OSM_API int osm_nvfp4_tensor_exponent(float amax, int* g);
+
+/* Host-only: g_act and g_w of a plan from its calibration statistics (the
+ * inputs of osm_calibrate_finalize and its outputs s, inv_s, O): the
+ * activations' tensor maximum is max over bulk channels of
+ * bf16(fp32(amax_j * inv_s_j)) -- the largest smoothed calibration value --
+ * and the weights' max over bulk channels of bf16(fp32(wmax_j * s_j)).
+ * Activations beyond the calibration range saturate (scale 448, element 6). */
+OSM_API int osm_nvfp4_plan_exponents(const float* amax_host, const float* wmax_host, const float* s_host,
+                                     const float* inv_s_host, const int32_t* O_host, int64_t K, int64_t k,
+                                     int* g_act, int* g_w);
 
 /* Debug flags for failure-detection tests (no counterpart in the paper).
  * OSM_DEBUG_STARVE_QUANTIZE: osm_quantize_act expects 16 bytes more per row
@@ -341,7 +386,8 @@ OSM_API int osm_linear_noalloc(const osm_plan* plan, const uint16_t* X, int64_t 
 /* ---- helpers ------------------------------------------------------------ */
 
 /* Host-only: un-swizzle a scales buffer (layout above) of `rows` rows and
- * `nblocks` = Kbp/32 blocks into a row-major [rows][nblocks] host array. */
+ * `nblocks` blocks (Kbp/32 for MXFP4, Kbp/16 for NVFP4) into a row-major
+ * [rows][nblocks] host array. */
 OSM_API int osm_scales_to_logical(const uint8_t* swizzled_host, int64_t rows, int64_t nblocks,
                           uint8_t* logical_host);
 

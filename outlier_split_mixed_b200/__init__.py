@@ -26,6 +26,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_NOMEM = 1, 2, 3, 4, 5, 6
 STATUS_TIMEOUT = 1
 HP_BF16, HP_FP16 = 0, 1
+FMT_MXFP4, FMT_NVFP4 = 0, 1
 STATUS_NONFINITE = 2
 DEBUG_STARVE_QUANTIZE = 1
 WSCALE_1x32, WSCALE_TILE32x32, WSCALE_STRIP128x1 = 0, 1, 2
@@ -45,6 +46,9 @@ _SIGNATURES = {
     "osm_plan_set_wait_limit": (_I, [_P, _U64]),
     "osm_plan_set_debug": (_I, [_P, ctypes.c_uint32]),
     "osm_plan_set_outlier_dtype": (_I, [_P, _I]),
+    "osm_plan_set_format": (_I, [_P, _I, _I, _I]),
+    "osm_nvfp4_tensor_exponent": (_I, [ctypes.c_float, ctypes.POINTER(_I)]),
+    "osm_nvfp4_plan_exponents": (_I, [_P, _P, _P, _P, _P, _I64, _I64, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "osm_plan_refresh": (_I, [_P, _P, _P, ctypes.c_float, _P]),
     "osm_plan_refresh_scored": (_I, [_P, _P, _P, _P, ctypes.c_float, _P]),
     "osm_act_percentile": (_I, [_P, _I64, _I64, ctypes.c_float, _P, _P]),
@@ -145,10 +149,12 @@ def _u8_types():
 
 class Plan:
     """An osm_plan: K, N, k, the smoothing vector s, the outlier set O and
-    the weight block-scale mode, with its device tables."""
+    the weight block-scale mode, with its device tables; optionally the FP16
+    outlier branch (hp_fp16) or the NVFP4 bulk format (fmt = FMT_NVFP4 with
+    the per-tensor exponents g_act, g_w)."""
 
     def __init__(self, K: int, N: int, k: int, s: np.ndarray, O: np.ndarray, wscale_mode: int = WSCALE_1x32,
-                 hp_fp16: bool = False):
+                 hp_fp16: bool = False, fmt: int = FMT_MXFP4, g_act: int = 0, g_w: int = 0):
         s = np.ascontiguousarray(s, dtype=np.float32)
         O = np.ascontiguousarray(O, dtype=np.int32)
         if s.shape != (K,) or O.shape != (k,):
@@ -164,6 +170,20 @@ class Plan:
         self.hp_fp16 = bool(hp_fp16)
         if hp_fp16:
             _check(lib().osm_plan_set_outlier_dtype(self._h, HP_FP16))
+        self.fmt, self.g_act, self.g_w = FMT_MXFP4, 0, 0
+        if fmt != FMT_MXFP4:
+            self.set_format(fmt, g_act, g_w)
+
+    def set_format(self, fmt: int, g_act: int = 0, g_w: int = 0):
+        """osm_plan_set_format: the 4-bit block format of the bulk branch."""
+        _check(lib().osm_plan_set_format(self._h, int(fmt), int(g_act), int(g_w)))
+        self.fmt = int(fmt)
+        self.g_act, self.g_w = (int(g_act), int(g_w)) if fmt == FMT_NVFP4 else (0, 0)
+
+    @property
+    def nblocks(self) -> int:
+        """Scale blocks per row: Kbp/32 (MXFP4) or Kbp/16 (NVFP4)."""
+        return self.Kbp // (16 if self.fmt == FMT_NVFP4 else 32)
 
     @property
     def handle(self):
@@ -286,6 +306,27 @@ def calibrate_finalize(amax_host: np.ndarray, wmax_host: np.ndarray, alpha: floa
     _check(lib().osm_calibrate_finalize(_host_ptr(amax_host), _host_ptr(wmax_host), K, float(alpha), int(k),
                                         _host_ptr(s), _host_ptr(inv_s), _host_ptr(O)))
     return s, inv_s, O[:k].copy()
+
+
+def nvfp4_tensor_exponent(amax: float) -> int:
+    """osm_nvfp4_tensor_exponent: smallest g in [-100, 100] with amax <= 6 * 448 * 2^g."""
+    g = ctypes.c_int()
+    _check(lib().osm_nvfp4_tensor_exponent(float(amax), ctypes.byref(g)))
+    return int(g.value)
+
+
+def nvfp4_plan_exponents(amax_host, wmax_host, s, inv_s, O):
+    """osm_nvfp4_plan_exponents: (g_act, g_w) from the calibration statistics."""
+    a = np.ascontiguousarray(amax_host, dtype=np.float32)
+    w = np.ascontiguousarray(wmax_host, dtype=np.float32)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    inv_s = np.ascontiguousarray(inv_s, dtype=np.float32)
+    O = np.ascontiguousarray(O, dtype=np.int32)
+    ga, gw = ctypes.c_int(), ctypes.c_int()
+    _check(lib().osm_nvfp4_plan_exponents(_host_ptr(a), _host_ptr(w), _host_ptr(s), _host_ptr(inv_s),
+                                          _host_ptr(O) if O.size else None, a.shape[0], O.shape[0],
+                                          ctypes.byref(ga), ctypes.byref(gw)))
+    return int(ga.value), int(gw.value)
 
 
 def calibrate_finalize_scored(amax_host: np.ndarray, score_host: np.ndarray, wmax_host: np.ndarray, alpha: float,

@@ -39,6 +39,9 @@ int check_cuda(cudaError_t e, const char* what) {
     return fail(OSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+float pow2f(int g) { return std::ldexp(1.0f, g); }
+float nvfp4_k(int g) { return std::ldexp(1.0f / 6.0f, -g); }
+
 // The kernels are built for sm_100a only.
 static int check_device() {
     int dev = 0;
@@ -181,6 +184,9 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
     p->kp = round_up(k, 64);
     p->wmode = wscale_mode;
     p->hp_fp16 = 0;
+    p->fmt = OSM_FMT_MXFP4;
+    p->g_act = 0;
+    p->g_w = 0;
     p->wait_limit_ns = 2000000000ull;
     p->debug_flags = 0;
 
@@ -257,7 +263,7 @@ int osm_plan_sizes(const osm_plan* p, int64_t rows, size_t* codes_bytes, size_t*
     OSM_REQUIRE(p, "plan_sizes: plan is NULL");
     OSM_REQUIRE(rows >= 0, "plan_sizes: rows < 0");
     if (codes_bytes) *codes_bytes = static_cast<size_t>(rows * (p->Kbp / 2));
-    if (scales_bytes) *scales_bytes = static_cast<size_t>(osm::scales_bytes(rows, p->Kbp));
+    if (scales_bytes) *scales_bytes = static_cast<size_t>(osm::scales_bytes(rows, p->Kbp, p->fmt));
     if (hp_bytes) *hp_bytes = static_cast<size_t>(rows * p->kp * 2);
     return OSM_OK;
 }
@@ -298,8 +304,74 @@ int osm_plan_set_outlier_dtype(osm_plan* p, int dtype) {
     g_err[0] = 0;
     OSM_REQUIRE(p, "plan_set_outlier_dtype: plan is NULL");
     OSM_REQUIRE(dtype == OSM_HP_BF16 || dtype == OSM_HP_FP16, "plan_set_outlier_dtype: unknown type %d", dtype);
+    OSM_REQUIRE(dtype == OSM_HP_BF16 || p->fmt == OSM_FMT_MXFP4,
+                "plan_set_outlier_dtype: an NVFP4 plan keeps a BF16 outlier branch");
     p->hp_fp16 = dtype == OSM_HP_FP16;
     return OSM_OK;
+}
+
+int osm_plan_set_format(osm_plan* p, int format, int g_act, int g_w) {
+    g_err[0] = 0;
+    OSM_REQUIRE(p, "plan_set_format: plan is NULL");
+    OSM_REQUIRE(format == OSM_FMT_MXFP4 || format == OSM_FMT_NVFP4, "plan_set_format: unknown format %d", format);
+    if (format == OSM_FMT_NVFP4) {
+        OSM_REQUIRE(g_act >= -100 && g_act <= 100 && g_w >= -100 && g_w <= 100 && std::abs(g_act + g_w) <= 126,
+                    "plan_set_format: exponents must lie in [-100, 100], |g_act + g_w| <= 126 (%d, %d)", g_act, g_w);
+        OSM_REQUIRE(p->wmode == OSM_WSCALE_1x32, "plan_set_format: NVFP4 needs the OSM_WSCALE_1x32 weight mode");
+        OSM_REQUIRE(!p->hp_fp16, "plan_set_format: NVFP4 needs the BF16 outlier branch");
+    }
+    p->fmt = format;
+    p->g_act = format == OSM_FMT_NVFP4 ? g_act : 0;
+    p->g_w = format == OSM_FMT_NVFP4 ? g_w : 0;
+    return OSM_OK;
+}
+
+int osm_nvfp4_tensor_exponent(float amax, int* g) {
+    g_err[0] = 0;
+    OSM_REQUIRE(g, "nvfp4_tensor_exponent: g is NULL");
+    OSM_REQUIRE(std::isfinite(amax) && amax >= 0.0f, "nvfp4_tensor_exponent: amax must be finite and >= 0");
+    int e = 0;
+    if (amax > 0.0f) {
+        e = -100;
+        while (e < 100 && static_cast<double>(amax) > std::ldexp(2688.0, e)) ++e;
+    }
+    *g = e;
+    return OSM_OK;
+}
+
+// bf16(fp32 v), round to nearest even (v finite)
+static float bf16_round_host(float v) {
+    uint32_t u;
+    std::memcpy(&u, &v, 4);
+    const uint32_t lsb = (u >> 16) & 1u;
+    u = (u + 0x7FFFu + lsb) & 0xFFFF0000u;
+    float r;
+    std::memcpy(&r, &u, 4);
+    return r;
+}
+
+int osm_nvfp4_plan_exponents(const float* amax, const float* wmax, const float* s, const float* inv_s,
+                             const int32_t* O, int64_t K, int64_t k, int* g_act, int* g_w) {
+    g_err[0] = 0;
+    OSM_REQUIRE(amax && wmax && s && inv_s && g_act && g_w, "nvfp4_plan_exponents: null pointer");
+    OSM_REQUIRE(K > 0 && k >= 0 && k <= K && (k == 0 || O), "nvfp4_plan_exponents: bad K / k / O");
+    std::vector<char> out(static_cast<size_t>(K), 0);
+    for (int64_t i = 0; i < k; ++i) {
+        OSM_REQUIRE(O[i] >= 0 && O[i] < K, "nvfp4_plan_exponents: O[%lld] out of range", (long long)i);
+        out[O[i]] = 1;
+    }
+    float am = 0.0f, wm = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+        if (out[j]) continue;
+        const float a = std::fabs(bf16_round_host(amax[j] * inv_s[j]));
+        const float w = std::fabs(bf16_round_host(wmax[j] * s[j]));
+        OSM_REQUIRE(std::isfinite(a) && std::isfinite(w), "nvfp4_plan_exponents: statistic %lld not finite",
+                    (long long)j);
+        am = std::max(am, a);
+        wm = std::max(wm, w);
+    }
+    OSM_TRY(osm_nvfp4_tensor_exponent(am, g_act));
+    return osm_nvfp4_tensor_exponent(wm, g_w);
 }
 
 int osm_plan_set_debug(osm_plan* p, uint32_t flags) {
@@ -406,6 +478,8 @@ int osm_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_sc
         OSM_REQUIRE(next->K == p->N, "dual_gemm: next->K (%lld) must equal plan->N (%lld)", (long long)next->K,
                     (long long)p->N);
         OSM_REQUIRE(!Y && !bias, "dual_gemm: GELU_REQUANT writes next_* only; Y and bias must be NULL");
+        OSM_REQUIRE(p->fmt == OSM_FMT_MXFP4 && next->fmt == OSM_FMT_MXFP4,
+                    "dual_gemm: GELU_REQUANT needs MXFP4 plans");
         OSM_REQUIRE(next->Kbp == 0 || (next_codes && aligned16(next_codes) && next_scales && aligned16(next_scales)),
                     "dual_gemm: next_codes / next_scales null or misaligned");
         OSM_REQUIRE(next->kp == 0 || (next_hp && aligned16(next_hp)), "dual_gemm: next_hp null or misaligned");

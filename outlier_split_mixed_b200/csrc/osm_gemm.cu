@@ -54,11 +54,8 @@ namespace {
 
 constexpr int BM = 128;                 // accumulator rows per CTA (TMEM lanes); pair tile M = 256
 constexpr int BN = 256;                 // output columns per tile; each CTA loads BN/2 rows of B
-constexpr int STAGES = 6;
 constexpr int A_TILE = BM * 128;        // one K-step of A: 128 rows x 128 bytes
 constexpr int B_TILE = (BN / 2) * 128;  // one K-step of this CTA's half of B
-constexpr int SFA_TILE = 2 * 512;       // two 128x4 scale atoms (K = 256)
-constexpr int SFB_TILE = 2 * 2 * 512;   // two 128-row tiles x two atoms (all 256 B rows)
 constexpr int NUM_EPI_WARPS = 8;        // two per TMEM lane quadrant, 128 columns each
 constexpr int CTRL_WG = 2;              // warpgroup of the producer (warp 8) and MMA issuer (warp 9)
 constexpr int PRODUCER_WARP = 4 * CTRL_WG;
@@ -82,11 +79,26 @@ static_assert(LAUNCH_REGS * 3 <= 512 && CTRL_REGS % 8 == 0 && EPI_REGS % 8 == 0,
 __host__ __device__ constexpr bool uses_register_split(int epi) { return epi == OSM_EPI_GELU_REQUANT; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;       // scale factors live after the accumulator
-constexpr uint32_t SF_STAGE_COLS = 24;  // 8 columns for A, 16 for B per ring slot
 constexpr int GROUP_M = 8;              // raster: 8 M-tiles sweep the N-tiles together
 constexpr uint16_t PAIR_MASK = 0x3;
 
-static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+// Ring shape per 4-bit format. A slot carries one K-step of 256 FP4 values;
+// its scales are 128 x 4 atoms of 512 bytes: two atoms per 128-row tile for
+// MXFP4 (8 E8M0 scales per row), four for NVFP4 (16 E4M3 scales). Each atom
+// is copied to four tensor-memory columns (A) or eight (B: two 128-row
+// tiles). NVFP4's larger slots leave room for five in shared and tensor
+// memory, MXFP4's for six.
+template <bool NV>
+struct Fmt {
+    static constexpr int STAGES = NV ? 5 : 6;
+    static constexpr int APS = NV ? 4 : 2;                // scale atoms per K-step and 128-row tile
+    static constexpr int SFA_TILE = APS * 512;
+    static constexpr int SFB_HALF = APS * 512;            // one 128-row tile of B
+    static constexpr int SFB_TILE = 2 * SFB_HALF;
+    static constexpr uint32_t SF_STAGE_COLS = 12 * APS;   // 4 columns per atom for A, 8 for B
+};
+static_assert(SF_COL0 + Fmt<false>::STAGES * Fmt<false>::SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+static_assert(SF_COL0 + Fmt<true>::STAGES * Fmt<true>::SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
 
 // Instruction descriptors (tcgen05 instruction-descriptor format), M = 256
 // over the CTA pair, N = 256.
@@ -94,17 +106,22 @@ static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budg
 // (bit 23), M>>4 @24; scale-factor byte ids at bits 29-30 (A) and 4-5 (B).
 constexpr uint32_t IDESC_MXF4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
                                 ((uint32_t)((2 * BM) >> 4) << 24);
+// kind::mxf4nvf4 with UE4M3 scales (bit 23 clear), four scales per row and
+// MMA: scale-factor byte ids 0.
+constexpr uint32_t IDESC_NVF4 = IDESC_MXF4 & ~(1u << 23);
 // kind::f16: FP32 accumulate (bit 4), A/B BF16 (1 @7, 1 @10), K-major;
 // IDESC_F16: the same with A and B binary16 (type 0 in both fields).
 constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                 ((uint32_t)((2 * BM) >> 4) << 24);
 constexpr uint32_t IDESC_F16 = IDESC_BF16 & ~((1u << 7) | (1u << 10));
 
+template <bool NV>
 struct __align__(1024) Smem {
+    static constexpr int STAGES = Fmt<NV>::STAGES;
     uint8_t a[STAGES][A_TILE];
     uint8_t b[STAGES][B_TILE];
-    uint8_t sfa[STAGES][SFA_TILE];
-    uint8_t sfb[STAGES][SFB_TILE];
+    uint8_t sfa[STAGES][Fmt<NV>::SFA_TILE];
+    uint8_t sfb[STAGES][Fmt<NV>::SFB_TILE];
     uint64_t full[STAGES];   // leader: all copies of both CTAs for the slot have landed
     uint64_t empty[STAGES];  // both: the MMAs reading the slot have completed
     uint64_t acc_full;       // both: the tile's accumulator is complete
@@ -126,13 +143,14 @@ struct GemmParams {
     uint32_t* status;
     uint64_t wait_limit_ns;
     int64_t M, N;
-    int katoms;      // Kbp / 128
-    int n_fp4;       // K-steps of the bulk branch: ceil(katoms / 2)
+    int katoms;      // scale atoms per 128-row tile: Kbp / 128 (MXFP4), Kbp / 64 (NVFP4)
+    int n_fp4;       // K-steps of the bulk branch: ceil(Kbp / 256)
     int n_hp;        // K-steps of the outlier branch: kp / 64
     int num_m, num_n;
     int n_row_tiles; // ceil(N / 128): scale-atom rows of W
     int epi;
     uint32_t idesc_hp;        // instruction descriptor of the outlier K-steps (BF16 or FP16 operands)
+    float out_scale;          // NVFP4: 2^(g_act + g_w), applied to the accumulator before the bias
     // OSM_EPI_GELU_REQUANT: the next layer's packed activations
     uint8_t* next_codes;      // [M][nKbp/2]
     uint8_t* next_scales;     // layout, rows padded to 128
@@ -153,7 +171,8 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
     n_blk = local / gm;
 }
 
-__device__ __forceinline__ void raise_abort(Smem& S, uint32_t* status) {
+template <class SM>
+__device__ __forceinline__ void raise_abort(SM& S, uint32_t* status) {
     S.abort_flag = 1;
     atomicOr(status, OSM_STATUS_TIMEOUT);
 }
@@ -192,7 +211,7 @@ __device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r)
 // store instruction of the warp writes eight full 32-byte sectors (one per
 // row), FP32 as 8-byte pairs or BF16 as 4-byte pairs. Rows >= M and
 // columns >= N (N % 32 == 0, so whole 8-column blocks) are skipped.
-template <int EPI>
+template <int EPI, bool NV>
 __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, int64_t col0, int lane, const uint32_t* r) {
     const int64_t ra = row0 + (lane >> 2), rb = ra + 8;
     const int cq = 2 * (lane & 3);
@@ -202,6 +221,10 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
         if (col >= p.N) break;
         float2 a = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
         float2 b = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        if constexpr (NV) {
+            a = __fmul2_rn(a, make_float2(p.out_scale, p.out_scale));
+            b = __fmul2_rn(b, make_float2(p.out_scale, p.out_scale));
+        }
         if (p.bias) {
             const float2 bb = __ldg(reinterpret_cast<const float2*>(p.bias + col));
             a = __fadd2_rn(a, bb);
@@ -336,7 +359,8 @@ __device__ __forceinline__ void shift_down(uint32_t (&r)[N]) {
 }
 
 // TMA producer, one elected thread in each CTA of the pair.
-__device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint32_t rank, bool leader, int pair,
+template <bool NV>
+__device__ __forceinline__ void producer_role(const GemmParams& p, Smem<NV>& S, uint32_t rank, bool leader, int pair,
                                               int npairs, int tiles, int ksteps, const volatile int* abort,
                                               const volatile int* never, uint64_t drain_ns) {
     if (ptx::elect_one()) {
@@ -360,7 +384,8 @@ __device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint
                 }
                 const uint32_t fb = ptx::mapa(ptx::smem_u32(&S.full[stage]), 0);  // leader's barrier
                 if (ks < p.n_fp4) {
-                    const int natoms = min(2, p.katoms - 2 * ks);
+                    constexpr int APS = Fmt<NV>::APS;
+                    const int natoms = min(APS, p.katoms - APS * ks);
                     if (leader)
                         ptx::mbar_arrive_expect_tx(ptx::smem_u32(&S.full[stage]),
                                                    2u * (A_TILE + B_TILE + natoms * 512u * (1u + nbt)));
@@ -368,10 +393,10 @@ __device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint
                     ptx::tma_load_2d_pair(ptx::smem_u32(S.b[stage]), &p.tm_b, ks * 128, brow, fb);
                     for (int a = 0; a < natoms; ++a) {
                         ptx::tma_load_2d_pair(ptx::smem_u32(S.sfa[stage]) + 512 * a, &p.tm_sa, 0,
-                                              (sfa_tile * p.katoms + 2 * ks + a) * 4, fb);
+                                              (sfa_tile * p.katoms + APS * ks + a) * 4, fb);
                         for (int h = 0; h < nbt; ++h)
-                            ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + 1024 * h + 512 * a, &p.tm_sb, 0,
-                                                  ((2 * n_blk + h) * p.katoms + 2 * ks + a) * 4, fb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(S.sfb[stage]) + Fmt<NV>::SFB_HALF * h + 512 * a,
+                                                  &p.tm_sb, 0, ((2 * n_blk + h) * p.katoms + APS * ks + a) * 4, fb);
                     }
                 } else {
                     const int kh = ks - p.n_fp4;
@@ -382,7 +407,7 @@ __device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint
                 }
                 last_stage = stage;
                 last_phase = phase;
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == Fmt<NV>::STAGES) { stage = 0; phase ^= 1u; }
             }
         }
         if (!ok) raise_abort(S, p.status);
@@ -398,7 +423,8 @@ __device__ __forceinline__ void producer_role(const GemmParams& p, Smem& S, uint
 }
 
 // MMA issuer, one elected thread of the leader CTA.
-__device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool leader, int pair, int npairs, int tiles,
+template <bool NV>
+__device__ __forceinline__ void mma_role(const GemmParams& p, Smem<NV>& S, bool leader, int pair, int npairs, int tiles,
                                          int ksteps, const volatile int* abort, const volatile int* never,
                                          uint64_t drain_ns, uint32_t tmem) {
     if (leader && ptx::elect_one()) {
@@ -423,22 +449,32 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool lead
                 const uint32_t a_base = ptx::smem_u32(S.a[stage]);
                 const uint32_t b_base = ptx::smem_u32(S.b[stage]);
                 if (ks < p.n_fp4) {
-                    const int natoms = min(2, p.katoms - 2 * ks);
-                    const uint32_t sfa_col = tmem + SF_COL0 + stage * SF_STAGE_COLS;
-                    const uint32_t sfb_col = sfa_col + 8;
+                    constexpr int APS = Fmt<NV>::APS;
+                    const int natoms = min(APS, p.katoms - APS * ks);
+                    const uint32_t sfa_col = tmem + SF_COL0 + stage * Fmt<NV>::SF_STAGE_COLS;
+                    const uint32_t sfb_col = sfa_col + 4 * APS;
                     const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
                     const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
                     for (int a = 0; a < natoms; ++a) {
                         ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
                         ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
-                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + 1024 + 512 * a));
+                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + Fmt<NV>::SFB_HALF + 512 * a));
                     }
-                    for (int kk = 0; kk < 2 * natoms; ++kk) {
-                        const uint32_t sf_id = (uint32_t)(kk & 1) * 2u;  // bytes 0-1 or 2-3 of the atom
-                        const uint32_t idesc = IDESC_MXF4 | (sf_id << 29) | (sf_id << 4);
-                        ptx::mma_mxf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32), idesc,
-                                           sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
-                        accumulate = 1;
+                    if constexpr (NV) {
+                        // one atom (four 16-blocks per row) per MMA of K = 64
+                        for (int kk = 0; kk < natoms; ++kk) {
+                            ptx::mma_nvf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                                               IDESC_NVF4, sfa_col + 4 * kk, sfb_col + 8 * kk, accumulate);
+                            accumulate = 1;
+                        }
+                    } else {
+                        for (int kk = 0; kk < 2 * natoms; ++kk) {
+                            const uint32_t sf_id = (uint32_t)(kk & 1) * 2u;  // bytes 0-1 or 2-3 of the atom
+                            const uint32_t idesc = IDESC_MXF4 | (sf_id << 29) | (sf_id << 4);
+                            ptx::mma_mxf4_pair(acc, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                                               idesc, sfa_col + 4 * (kk >> 1), sfb_col + 8 * (kk >> 1), accumulate);
+                            accumulate = 1;
+                        }
                     }
                 } else {
 #pragma unroll
@@ -449,7 +485,7 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool lead
                     }
                 }
                 ptx::tc_commit_pair_mc(ptx::smem_u32(&S.empty[stage]), PAIR_MASK);
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == Fmt<NV>::STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             ptx::tc_commit_pair_mc(ptx::smem_u32(&S.acc_full), PAIR_MASK);
@@ -464,8 +500,8 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem& S, bool lead
 
 // Epilogue, warps 0..7 of both CTAs: drain the accumulator, release
 // it to the MMA issuer, then convert and store.
-template <int EPI>
-__device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int warp, int lane, uint32_t rank,
+template <int EPI, bool NV>
+__device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem<NV>& S, int warp, int lane, uint32_t rank,
                                               int pair, int npairs, int tiles, const volatile int* abort,
                                               uint32_t tmem) {
     const int q = warp & 3;                   // TMEM lanes 32q..32q+31 are reachable from this warp
@@ -488,6 +524,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int 
         const int64_t y0 = (int64_t)m_blk * 2 * BM + (int64_t)rank * BM + q * 32;
         const int64_t x0 = (int64_t)n_blk * BN + half * 128;
         if constexpr (EPI == OSM_EPI_GELU_REQUANT) {
+            static_assert(!NV, "the fused requantisation takes MXFP4 operands");
             // lane = row, 32 consecutive columns per load: whole MX blocks per lane
             uint32_t r[128];
             ptx::tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
@@ -510,7 +547,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem& S, int 
             if (x0 < p.N) {
 #pragma unroll 1
                 for (int sl = 0; sl < 2; ++sl) {
-                    store_slab<EPI>(p, y0 + 16 * sl, x0, lane, r);
+                    store_slab<EPI, NV>(p, y0 + 16 * sl, x0, lane, r);
                     shift_down<64>(r);
                 }
             }
@@ -533,11 +570,11 @@ __device__ __forceinline__ void teardown(int warp, uint32_t tmem) {
     }
 }
 
-template <int EPI>
+template <int EPI, bool NV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     dual_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<NV>& S = *reinterpret_cast<Smem<NV>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = ptx::cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
@@ -553,7 +590,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint64_t drain_ns = p.wait_limit_ns > 200000000ull ? p.wait_limit_ns : 200000000ull;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < Fmt<NV>::STAGES; ++s) {
             ptx::mbar_init(ptx::smem_u32(&S.full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&S.empty[s]), 1);
         }
@@ -592,7 +629,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         teardown(warp, tmem);
     } else {
         if constexpr (uses_register_split(EPI)) ptx::setmaxnreg_inc<EPI_REGS>();
-        epilogue_role<EPI>(p, S, warp, lane, rank, pair, npairs, tiles, abort, tmem);
+        epilogue_role<EPI, NV>(p, S, warp, lane, rank, pair, npairs, tiles, abort, tmem);
         teardown(warp, tmem);
     }
 }
@@ -634,13 +671,14 @@ struct LaunchInfo {
 
 }  // namespace
 
-size_t dual_gemm_smem_bytes() { return sizeof(Smem) + 1024; }
 
 int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
                      int64_t M, const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
                      const float* bias, int epi, void* Y, const osm_plan* next, uint8_t* next_codes,
                      uint8_t* next_scales, uint16_t* next_hp, cudaStream_t st) {
-    static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
+    static_assert(sizeof(Smem<false>) + 1024 <= 232448 && sizeof(Smem<true>) + 1024 <= 232448,
+                  "shared memory budget");
+    const bool nv = pl->fmt == OSM_FMT_NVFP4;
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
     int rc;
@@ -654,8 +692,8 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
             return rc;
         // scale atoms are contiguous 512-byte runs: view them as 128-byte rows so
         // that one atom is four wide TMA requests rather than 32 narrow ones
-        const uint64_t sa_rows = static_cast<uint64_t>(scales_bytes(M, pl->Kbp)) / 128;
-        const uint64_t sb_rows = static_cast<uint64_t>(scales_bytes(pl->N, pl->Kbp)) / 128;
+        const uint64_t sa_rows = static_cast<uint64_t>(scales_bytes(M, pl->Kbp, pl->fmt)) / 128;
+        const uint64_t sb_rows = static_cast<uint64_t>(scales_bytes(pl->N, pl->Kbp, pl->fmt)) / 128;
         if ((rc = make_map(&p.tm_sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 128, sa_rows, 128, 128, 4, NOSW,
                            "a_scales")))
             return rc;
@@ -678,14 +716,15 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     p.wait_limit_ns = pl->wait_limit_ns;
     p.M = M;
     p.N = pl->N;
-    p.katoms = static_cast<int>(pl->Kbp / 128);
-    p.n_fp4 = (p.katoms + 1) / 2;
+    p.katoms = static_cast<int>(pl->Kbp / (4 * block_elems(pl->fmt)));
+    p.n_fp4 = static_cast<int>(ceil_div(pl->Kbp, 256));
     p.n_hp = static_cast<int>(pl->kp / 64);
     p.num_m = static_cast<int>(ceil_div(M, 2 * BM));
     p.num_n = static_cast<int>(ceil_div(pl->N, BN));
     p.n_row_tiles = static_cast<int>(ceil_div(pl->N, 128));
     p.epi = epi;
     p.idesc_hp = pl->hp_fp16 ? IDESC_F16 : IDESC_BF16;
+    p.out_scale = nv ? pow2f(pl->g_act + pl->g_w) : 1.0f;
     if (epi == OSM_EPI_GELU_REQUANT) {
         p.next_codes = next_codes;
         p.next_scales = next_scales;
@@ -701,21 +740,30 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
 
     void (*kernel)(GemmParams) = nullptr;
     switch (epi) {
-        case OSM_EPI_F32: kernel = dual_gemm_kernel<OSM_EPI_F32>; break;
-        case OSM_EPI_BF16: kernel = dual_gemm_kernel<OSM_EPI_BF16>; break;
-        case OSM_EPI_GELU_REQUANT: kernel = dual_gemm_kernel<OSM_EPI_GELU_REQUANT>; break;
-        case OSM_EPI_GELU_BF16: kernel = dual_gemm_kernel<OSM_EPI_GELU_BF16>; break;
+        case OSM_EPI_F32:
+            kernel = nv ? dual_gemm_kernel<OSM_EPI_F32, true> : dual_gemm_kernel<OSM_EPI_F32, false>;
+            break;
+        case OSM_EPI_BF16:
+            kernel = nv ? dual_gemm_kernel<OSM_EPI_BF16, true> : dual_gemm_kernel<OSM_EPI_BF16, false>;
+            break;
+        case OSM_EPI_GELU_REQUANT:
+            if (nv) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: GELU_REQUANT takes MXFP4 operands");
+            kernel = dual_gemm_kernel<OSM_EPI_GELU_REQUANT, false>;
+            break;
+        case OSM_EPI_GELU_BF16:
+            kernel = nv ? dual_gemm_kernel<OSM_EPI_GELU_BF16, true> : dual_gemm_kernel<OSM_EPI_GELU_BF16, false>;
+            break;
         default: return fail(OSM_ERR_INVALID_ARG, "dual_gemm: epilogue %d", epi);
     }
 
     // co-resident clusters of two CTAs, queried once per device and epilogue
-    static LaunchInfo info[64][4];
+    static LaunchInfo info[64][8];
     static std::mutex mu;
     int dev = 0;
     if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
     if (dev < 0 || dev >= 64) return fail(OSM_ERR_UNSUPPORTED, "device index %d", dev);
-    const size_t smem = sizeof(Smem) + 1024;
-    LaunchInfo& li = info[dev][epi];
+    const size_t smem = (nv ? sizeof(Smem<true>) : sizeof(Smem<false>)) + 1024;
+    LaunchInfo& li = info[dev][2 * epi + (nv ? 1 : 0)];
     {
         std::lock_guard<std::mutex> lk(mu);
         if (!li.ready) {

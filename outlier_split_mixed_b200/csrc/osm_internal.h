@@ -12,6 +12,8 @@ struct osm_plan {
     int64_t K, N, k, Kb, Kbp, kp;
     int wmode;
     int hp_fp16;         // outlier branch in binary16 (OSM_HP_FP16) instead of BF16
+    int fmt;             // OSM_FMT_MXFP4 or OSM_FMT_NVFP4
+    int g_act, g_w;      // NVFP4 per-tensor exponents (activations, weights)
     // device tables, owned by the plan
     float* d_s;          // [K]  smoothing vector s (Eq. (2))
     float* d_inv_s;      // [K]  1.0f / s
@@ -45,10 +47,17 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Elements per scale block: 32 (MXFP4) or 16 (NVFP4).
+inline int64_t block_elems(int fmt) { return fmt == OSM_FMT_NVFP4 ? 16 : 32; }
+
 // Bytes of one scales buffer for `rows` rows of a plan.
-inline int64_t scales_bytes(int64_t rows, int64_t Kbp) {
-    return round_up(rows, 128) * (Kbp / 32);
+inline int64_t scales_bytes(int64_t rows, int64_t Kbp, int fmt) {
+    return round_up(rows, 128) * (Kbp / block_elems(fmt));
 }
+
+// fp32(1/6) * 2^-g and 2^g as floats (exact for |g| <= 100).
+float nvfp4_k(int g);
+float pow2f(int g);
 
 // launchers (return OSM_OK or an error code; arguments already validated)
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st);

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstdint>
 
@@ -32,6 +33,46 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
     uint32_t d;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
+}
+
+// Two FP32 values -> two E4M3 codes (RNE, saturating at +-448): lo in bits
+// 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// Two E4M3 codes (lo in bits 0-7) -> their values (exact: E4M3 is a subset
+// of binary16).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t codes) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(codes)));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// NVFP4 block scales of two blocks from their maxima (BF16 bit patterns,
+// sign clear): S = E4M3_RNE_satfinite(fp32(amax * k)) with k = fp32(1/6) *
+// 2^-g, and each block's element multiplier R = fp32(1 / (S * 2^g)), 0 when
+// S is 0. Returns the two codes (lo in bits 0-7).
+__device__ __forceinline__ uint32_t nv_block_scales(uint32_t amax_lo, uint32_t amax_hi, float k, float p2g,
+                                                    float* r_lo, float* r_hi) {
+    const uint32_t s2 = e4m3x2_bits(__fmul_rn(bf16_bits_to_f32(amax_lo), k), __fmul_rn(bf16_bits_to_f32(amax_hi), k));
+    const float2 d = e4m3x2_to_f32(s2);
+    *r_lo = (s2 & 0xFFu) ? __frcp_rn(__fmul_rn(d.x, p2g)) : 0.0f;
+    *r_hi = (s2 & 0xFF00u) ? __frcp_rn(__fmul_rn(d.y, p2g)) : 0.0f;
+    return s2;
+}
+
+// Eight BF16 values (4 packed words) times a power of two, each rounded
+// back to BF16 (exact unless the product leaves the normal range).
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float f) {
+    const float2 f2 = make_float2(f, f);
+    auto one = [&](uint32_t w) {
+        const float2 x = __fmul2_rn(make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)), f2);
+        return bf16x2_bits(x.x, x.y);
+    };
+    return make_uint4(one(v.x), one(v.y), one(v.z), one(v.w));
 }
 
 // max(|a|, |b|) of each BF16 half of two packed words; the sign bits of the

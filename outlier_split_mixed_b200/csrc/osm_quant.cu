@@ -23,12 +23,7 @@ namespace {
 
 // ------------------------------------------------------------ helpers
 
-using mx::bf16_bits_to_f32;
-using mx::exp2_neg;
-using mx::f32_to_bf16_bits;
 using mx::sf_offset;
-
-__device__ __forceinline__ int mx_exponent(float amax) { return mx::exponent(amax); }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;
@@ -37,8 +32,6 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
                  : "l"(p));
     return v;
 }
-
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
 __device__ __forceinline__ uint32_t ldg_nc_u32(const uint32_t* p) {
     uint32_t v;
@@ -206,6 +199,11 @@ struct PackParams {
     uint8_t* codes;     // [N][Kbp/2]
     uint8_t* scales;    // layout, rows padded to 128
     uint16_t* hp;       // [N][kp]
+    int katoms;         // scale atoms per 128-row tile: Kbp/128 (MXFP4) or Kbp/64 (NVFP4)
+    int nv;             // NVFP4 encoding
+    float nv_k;         // NVFP4: fp32(1/6) * 2^-g_w
+    float nv_p2g;       // NVFP4: 2^g_w
+    float hp_scale;     // NVFP4: 2^-g_w on the outlier rows
 };
 
 // Tiled forms of the two packing kernels: a CTA gathers whole W rows (input
@@ -252,14 +250,16 @@ __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0
 // down the block, so one packed abs-max chain gives both channels' block
 // maxima. 1x32: the block maximum; 32x32: the maximum over 32 channels (16
 // lanes); 128x1: the maximum over the strip's four blocks (four warps, via
-// shared memory). Codes and scales as in pack_bulk_kernel.
+// shared memory). NV: the 32 positions are two NVFP4 16-blocks, each with
+// its own E4M3 scale and element multiplier.
+template <bool NV>
 __global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams p) {
     __shared__ __align__(16) uint32_t tile[128][64];
     __shared__ uint32_t red[4][64];
-    __shared__ uint32_t sxs[4][64];  // exponent codes, (lo | hi << 8) per quarter and pair
+    __shared__ uint32_t sxs[4][64];  // scale codes per quarter and pair: MX (n | n+1 << 8), NV (n: 2 bytes | n+1: 2 bytes)
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
     const int64_t p0 = static_cast<int64_t>(blockIdx.y) * 128;
-    const int64_t katoms = p.Kbp / 128;
+    const int64_t katoms = p.katoms;
     load_folded_rows<false>(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; },
                             tile);
     __syncthreads();
@@ -271,6 +271,51 @@ __global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams 
 #pragma unroll
     for (int i = 0; i < 32; ++i) wv[i] = tile[32 * q + i][c];
     using mx::bf16x2_absmax;
+    const int64_t n = n0 + 2 * c;
+    if constexpr (NV) {
+        uint32_t ma = wv[0], mb = wv[16];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) {
+            ma = bf16x2_absmax(ma, wv[i]);
+            mb = bf16x2_absmax(mb, wv[16 + i]);
+        }
+        float r0a, r0b, r1a, r1b;  // multipliers of channel n (blocks 2q, 2q+1) and n + 1
+        const uint32_t s0 = mx::nv_block_scales(ma & 0x7FFFu, mb & 0x7FFFu, p.nv_k, p.nv_p2g, &r0a, &r0b);
+        const uint32_t s1 =
+            mx::nv_block_scales((ma >> 16) & 0x7FFFu, (mb >> 16) & 0x7FFFu, p.nv_k, p.nv_p2g, &r1a, &r1b);
+        if (n < p.N) {
+            uint32_t lo[16], hi[16];
+#pragma unroll
+            for (int k2 = 0; k2 < 16; ++k2) {
+                lo[k2] = __byte_perm(wv[2 * k2], wv[2 * k2 + 1], 0x5410);
+                hi[k2] = __byte_perm(wv[2 * k2], wv[2 * k2 + 1], 0x7632);
+            }
+            const uint4 clo = make_uint4(mx::encode8_words(lo[0], lo[1], lo[2], lo[3], r0a),
+                                         mx::encode8_words(lo[4], lo[5], lo[6], lo[7], r0a),
+                                         mx::encode8_words(lo[8], lo[9], lo[10], lo[11], r0b),
+                                         mx::encode8_words(lo[12], lo[13], lo[14], lo[15], r0b));
+            const uint4 chi = make_uint4(mx::encode8_words(hi[0], hi[1], hi[2], hi[3], r1a),
+                                         mx::encode8_words(hi[4], hi[5], hi[6], hi[7], r1a),
+                                         mx::encode8_words(hi[8], hi[9], hi[10], hi[11], r1b),
+                                         mx::encode8_words(hi[12], hi[13], hi[14], hi[15], r1b));
+            *reinterpret_cast<uint4*>(p.codes + n * (p.Kbp / 2) + p0 / 2 + 16 * q) = clo;
+            *reinterpret_cast<uint4*>(p.codes + (n + 1) * (p.Kbp / 2) + p0 / 2 + 16 * q) = chi;
+        }
+        sxs[q][c] = (s0 & 0xFFFFu) | (s1 << 16);
+        __syncthreads();
+        if (warp < 2) {  // a channel's eight scale bytes of the strip: one word in each of two atoms
+            uint32_t w0lo = (sxs[0][c] & 0xFFFFu) | (sxs[1][c] << 16), w1lo = (sxs[2][c] & 0xFFFFu) | (sxs[3][c] << 16);
+            uint32_t w0hi = (sxs[0][c] >> 16) | (sxs[1][c] & 0xFFFF0000u), w1hi = (sxs[2][c] >> 16) | (sxs[3][c] & 0xFFFF0000u);
+            if (n >= p.N) w0lo = w1lo = 0;
+            if (n + 1 >= p.N) w0hi = w1hi = 0;
+            const int64_t b0 = static_cast<int64_t>(blockIdx.y) * 8;
+            *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, b0, katoms)) = w0lo;
+            *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, b0 + 4, katoms)) = w1lo;
+            *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n + 1, b0, katoms)) = w0hi;
+            *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n + 1, b0 + 4, katoms)) = w1hi;
+        }
+        return;
+    }
     uint32_t m = wv[0];
 #pragma unroll
     for (int i = 1; i < 32; ++i) m = bf16x2_absmax(m, wv[i]);
@@ -288,7 +333,6 @@ __global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams 
     float inv_lo, inv_hi;
     const int X_lo = mx::bf16_block_exponent(m & 0x7FFFu, &inv_lo);
     const int X_hi = mx::bf16_block_exponent((m >> 16) & 0x7FFFu, &inv_hi);
-    const int64_t n = n0 + 2 * c;
     if (n < p.N) {
         uint32_t lo[16], hi[16];
 #pragma unroll
@@ -345,8 +389,9 @@ __global__ void __launch_bounds__(PK_THREADS) pack_hp_tiled_kernel(PackParams p)
         uint32_t e[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) e[i] = t16[(8 * g + i) * 128 + nl];
-        *reinterpret_cast<uint4*>(p.hp + n * p.kp + i0 + 8 * g) =
-            make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+        uint4 v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+        if (p.nv) v = mx::scale_bf16x8(v, p.hp_scale);  // NVFP4: w_hp = bf16(fp32(w') * 2^-g_w)
+        *reinterpret_cast<uint4*>(p.hp + n * p.kp + i0 + 8 * g) = v;
     }
 }
 
@@ -364,7 +409,14 @@ struct QuantParams {
     uint64_t wait_limit_ns;  // bound of every wait on an incoming row group
     uint32_t extra_tx;       // bytes expected beyond each group's copy (0; 16 when starved for a test)
     int hp_fp16;             // outlier slots in binary16 instead of BF16
+    int katoms;              // scale atoms per 128-row tile: Kbp/128 (MXFP4) or Kbp/64 (NVFP4)
+    float nv_k;              // NVFP4: fp32(1/6) * 2^-g_act
+    float nv_p2g;            // NVFP4: 2^g_act
+    float hp_scale;          // NVFP4: 2^-g_act on the outlier slots
 };
+
+// Encodings of quantize_act: MXFP4 with BF16 or FP16 outlier slots, NVFP4.
+enum QaMode { QA_MX = 0, QA_MX_F16 = 1, QA_NV = 2 };
 
 constexpr int QA_THREADS = 256;
 constexpr int STREAM_NT = 512;  // threads of the streaming form
@@ -386,8 +438,13 @@ __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * Q
 //           amax by packed u16 max, E8M0 exponent, sixteen E2M1x2
 //           conversions, one 128-bit code store and one scale byte;
 //  phase 3: the outlier slots go out as 128-bit stores.
-template <int R, bool HPF>
+template <int MODE>
+__device__ __forceinline__ void encode_staged(const QuantParams& p, uint32_t sbuf, int stride, int row0, int nrows);
+__device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p);
+
+template <int R, int MODE>
 __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p) {
+    constexpr bool HPF = MODE == QA_MX_F16;
     extern __shared__ __align__(16) uint8_t sbuf[];
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
@@ -446,68 +503,24 @@ __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p)
     }
     __syncthreads();
 
-    // phase 2
-    const int katoms = p.Kbp >> 7;
-    const float inv_nb = 1.0f / static_cast<float>(nb);
-    for (int wi = tid; wi < R * nb; wi += QA_THREADS) {
-        // r = wi / nb (exact: wi < 2^20 and the quotient is below 8)
-        int r = static_cast<int>((static_cast<float>(wi) + 0.5f) * inv_nb);
-        r -= (r * nb > wi);
-        r += ((r + 1) * nb <= wi);
-        const int b = wi - r * nb;
-        const int t = row0 + r;
-        if (t >= p.M) continue;
-        const uint8_t* src = sbuf + r * stride + b * QA_BLOCK_BYTES;
-        const uint4 q0 = lds128(src), q1 = lds128(src + 16), q2 = lds128(src + 32), q3 = lds128(src + 48);
-        uint32_t m = vmax_u16x2(vmax_u16x2(q0.x & 0x7FFF7FFFu, q0.y & 0x7FFF7FFFu),
-                                vmax_u16x2(q0.z & 0x7FFF7FFFu, q0.w & 0x7FFF7FFFu));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q1.x & 0x7FFF7FFFu, q1.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q1.z & 0x7FFF7FFFu, q1.w & 0x7FFF7FFFu)));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q2.x & 0x7FFF7FFFu, q2.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q2.z & 0x7FFF7FFFu, q2.w & 0x7FFF7FFFu)));
-        m = vmax_u16x2(m, vmax_u16x2(vmax_u16x2(q3.x & 0x7FFF7FFFu, q3.y & 0x7FFF7FFFu),
-                                     vmax_u16x2(q3.z & 0x7FFF7FFFu, q3.w & 0x7FFF7FFFu)));
-        const uint32_t amax = max(m & 0xFFFFu, m >> 16);
-        const int X = mx_exponent(bf16_bits_to_f32(amax));
-        const float inv = exp2_neg(X);
-        const uint4 out = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv), encode8_words(q2, inv),
-                                     encode8_words(q3, inv));
-        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16) = out;
-        p.scales[sf_offset(t, b, katoms)] = static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
-    }
-
-    // phase 3: outlier slots
-    const int hv = p.kp >> 3;
-    for (int i = tid; i < R * hv; i += QA_THREADS) {
-        const int r = i / hv, c = i - r * hv;
-        const int t = row0 + r;
-        if (t < p.M)
-            *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(t) * p.kp + c * 8) =
-                lds128(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
-    }
-
-    // scale bytes of the padding rows [M, round_up(M,128)) are zero
-    if (row0 <= p.M - 1 && p.M - 1 < row0 + R && (p.M & 127) != 0) {
-        const int tile = (p.M - 1) >> 7;
-        const int rem = p.M & 127;
-        const int nwords = (128 - rem) * katoms;
-        for (int i = tid; i < nwords; i += QA_THREADS) {
-            const int a = i / (128 - rem), rr = rem + (i - a * (128 - rem));
-            *reinterpret_cast<uint32_t*>(p.scales + sf_offset(tile * 128 + rr, a * 4, katoms)) = 0u;
-        }
-    }
+    // phases 2 and 3
+    encode_staged<MODE>(p, ptx::smem_u32(sbuf), stride, row0, min(R, p.M - row0));
+    if (row0 <= p.M - 1 && p.M - 1 < row0 + R) zero_padding_scale_rows(p);
 }
 
 
 // Encode the staged rows [0, nrows) of a routed buffer: one thread per
 // (row, 32-block) -- four 128-bit shared loads, amax by packed u16 max, the
-// E8M0 exponent, sixteen E2M1x2 conversions, one 16-byte code store and one
-// scale byte -- then the outlier slots as 16-byte copies. Rows are
-// row0 + r of the output.
+// block scale(s), sixteen E2M1x2 conversions, one 16-byte code store and the
+// scale byte(s) -- then the outlier slots as 16-byte copies. MXFP4: one E8M0
+// exponent per 32-block. NVFP4: the 32-block is two 16-blocks, each with its
+// E4M3 scale and element multiplier; the outlier slots are scaled by
+// 2^-g_act. Rows are row0 + r of the output.
+template <int MODE>
 __device__ __forceinline__ void encode_staged(const QuantParams& p, uint32_t sbuf, int stride, int row0,
                                               int nrows) {
     const int nb = p.Kbp >> 5;
-    const int katoms = p.Kbp >> 7;
+    const int katoms = p.katoms;
     const int tid = threadIdx.x;
     const float inv_nb = 1.0f / static_cast<float>(nb);
     for (int wi = tid; wi < nrows * nb; wi += blockDim.x) {
@@ -521,31 +534,43 @@ __device__ __forceinline__ void encode_staged(const QuantParams& p, uint32_t sbu
         const uint4 q0 = ptx::ld_shared_v4(src), q1 = ptx::ld_shared_v4(src + 16), q2 = ptx::ld_shared_v4(src + 32),
                     q3 = ptx::ld_shared_v4(src + 48);
         using mx::bf16x2_absmax;
-        const uint32_t m = bf16x2_absmax(
-            bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q0.x, q0.y), bf16x2_absmax(q0.z, q0.w)),
-                          bf16x2_absmax(bf16x2_absmax(q1.x, q1.y), bf16x2_absmax(q1.z, q1.w))),
-            bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q2.x, q2.y), bf16x2_absmax(q2.z, q2.w)),
-                          bf16x2_absmax(bf16x2_absmax(q3.x, q3.y), bf16x2_absmax(q3.z, q3.w))));
-        const uint32_t amax = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
-        float inv;
-        const int X = mx::bf16_block_exponent(amax, &inv);
-        const uint4 out = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv), encode8_words(q2, inv),
-                                     encode8_words(q3, inv));
-        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16) = out;
-        p.scales[sf_offset(t, b, katoms)] = static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
+        const uint32_t m01 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q0.x, q0.y), bf16x2_absmax(q0.z, q0.w)),
+                                           bf16x2_absmax(bf16x2_absmax(q1.x, q1.y), bf16x2_absmax(q1.z, q1.w)));
+        const uint32_t m23 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(q2.x, q2.y), bf16x2_absmax(q2.z, q2.w)),
+                                           bf16x2_absmax(bf16x2_absmax(q3.x, q3.y), bf16x2_absmax(q3.z, q3.w)));
+        uint8_t* codes = p.codes + static_cast<size_t>(t) * (p.Kbp >> 1) + b * 16;
+        if constexpr (MODE == QA_NV) {
+            float r_lo, r_hi;
+            const uint32_t s2 = mx::nv_block_scales(max(m01 & 0x7FFFu, (m01 >> 16) & 0x7FFFu),
+                                                    max(m23 & 0x7FFFu, (m23 >> 16) & 0x7FFFu), p.nv_k, p.nv_p2g,
+                                                    &r_lo, &r_hi);
+            *reinterpret_cast<uint4*>(codes) = make_uint4(encode8_words(q0, r_lo), encode8_words(q1, r_lo),
+                                                          encode8_words(q2, r_hi), encode8_words(q3, r_hi));
+            // 16-blocks 2b and 2b + 1: adjacent bytes of one atom row
+            *reinterpret_cast<uint16_t*>(p.scales + sf_offset(t, 2 * b, katoms)) = static_cast<uint16_t>(s2);
+        } else {
+            const uint32_t m = bf16x2_absmax(m01, m23);
+            const uint32_t amax = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
+            float inv;
+            const int X = mx::bf16_block_exponent(amax, &inv);
+            *reinterpret_cast<uint4*>(codes) = make_uint4(encode8_words(q0, inv), encode8_words(q1, inv),
+                                                          encode8_words(q2, inv), encode8_words(q3, inv));
+            p.scales[sf_offset(t, b, katoms)] = static_cast<uint8_t>(b * 32 < p.Kb ? X + 127 : 0);
+        }
     }
     const int hv = p.kp >> 3;
     for (int i = tid; i < nrows * hv; i += blockDim.x) {
         const int r = i / hv, c = i - r * hv;
-        *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(row0 + r) * p.kp + c * 8) =
-            ptx::ld_shared_v4(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
+        uint4 v = ptx::ld_shared_v4(sbuf + r * stride + nb * QA_BLOCK_BYTES + c * 16);
+        if constexpr (MODE == QA_NV) v = mx::scale_bf16x8(v, p.hp_scale);
+        *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(row0 + r) * p.kp + c * 8) = v;
     }
 }
 
 // Scale bytes of the padding rows [M, round_up(M, 128)) are zero; done by
 // the CTA that handles row M - 1.
 __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
-    const int katoms = p.Kbp >> 7;
+    const int katoms = p.katoms;
     const int tile = (p.M - 1) >> 7;
     const int rem = p.M & 127;
     if (rem == 0) return;
@@ -570,8 +595,9 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 //  are encoded (encode_staged).
 // Every wait on a slot is bounded; a wait that runs out sets
 // OSM_STATUS_TIMEOUT, and the CTA lets its copies land before it returns.
-template <int R, int S, int NT, int TR, bool HPF>
+template <int R, int S, int NT, int TR, int MODE>
 __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams p) {
+    constexpr bool HPF = MODE == QA_MX_F16;
     extern __shared__ __align__(128) uint8_t smem[];
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
@@ -688,7 +714,7 @@ __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams 
         }
         __syncthreads();  // raw slot consumed, staged rows complete
         if (tid == 0 && issued < mine) issue(issued++);
-        encode_staged(p, sbuf_u32, stride, g * R, rows);
+        encode_staged<MODE>(p, sbuf_u32, stride, g * R, rows);
         if (g * R <= p.M - 1 && p.M - 1 < g * R + rows) zero_padding_scale_rows(p);
         __syncthreads();  // staged rows free for the next group
     }
@@ -723,11 +749,14 @@ int launch_weight_amax(const uint16_t* W, int64_t K, int64_t N, float* wmax, cud
 
 int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* col_order, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st) {
+    const bool nv = pl->fmt == OSM_FMT_NVFP4;
     PackParams p{W, col_order, pl->d_s, pl->d_J, pl->d_O, pl->K, pl->N, pl->k, pl->Kb, pl->Kbp, pl->kp,
-                 pl->wmode, codes, scales, hp};
+                 pl->wmode, codes, scales, hp, static_cast<int>(pl->Kbp / (4 * block_elems(pl->fmt))), nv ? 1 : 0,
+                 nvfp4_k(pl->g_w), pow2f(pl->g_w), pow2f(-pl->g_w)};
     if (pl->Kbp > 0) {
         dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 128), static_cast<unsigned>(pl->Kbp / 128));
-        pack_bulk_tiled_kernel<<<grid, PK_THREADS, 0, st>>>(p);
+        if (nv) pack_bulk_tiled_kernel<true><<<grid, PK_THREADS, 0, st>>>(p);
+        else pack_bulk_tiled_kernel<false><<<grid, PK_THREADS, 0, st>>>(p);
         int rc = check_cuda(cudaGetLastError(), "pack_bulk launch");
         if (rc) return rc;
     }
@@ -785,8 +814,9 @@ static int prepare_kernel(const void* kern, int threads, size_t smem, int* per_s
 }
 
 template <int R>
-static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
-    auto kern = p.hp_fp16 ? quantize_act_kernel<R, true> : quantize_act_kernel<R, false>;
+static int launch_qa(const QuantParams& p, int mode, size_t smem, cudaStream_t st) {
+    auto kern = mode == QA_NV ? quantize_act_kernel<R, QA_NV>
+                              : (mode == QA_MX_F16 ? quantize_act_kernel<R, QA_MX_F16> : quantize_act_kernel<R, QA_MX>);
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), QA_THREADS, smem, nullptr, nullptr);
     if (rc) return rc;
     const int64_t grid = ceil_div(p.M, R);
@@ -795,9 +825,11 @@ static int launch_qa(const QuantParams& p, size_t smem, cudaStream_t st) {
 }
 
 template <int R, int S, int NT, int TR>
-static int launch_stream(const QuantParams& p, int stride, cudaStream_t st) {
+static int launch_stream(const QuantParams& p, int mode, int stride, cudaStream_t st) {
     const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
-    auto kern = p.hp_fp16 ? quantize_act_stream_kernel<R, S, NT, TR, true> : quantize_act_stream_kernel<R, S, NT, TR, false>;
+    auto kern = mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV>
+                              : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16>
+                                                   : quantize_act_stream_kernel<R, S, NT, TR, QA_MX>);
     int per_sm = 0, sms = 0;
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
     if (rc) return rc;
@@ -814,24 +846,27 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
     QuantParams p{X, pl->d_inv_s, pl->d_route, static_cast<int>(M), static_cast<int>(pl->K),
                   static_cast<int>(pl->k), static_cast<int>(pl->Kb), static_cast<int>(pl->Kbp),
                   static_cast<int>(pl->kp), codes, scales, hp, pl->d_status, pl->wait_limit_ns,
-                  (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u, pl->hp_fp16};
+                  (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u, pl->hp_fp16,
+                  static_cast<int>(pl->Kbp / (4 * block_elems(pl->fmt))), nvfp4_k(pl->g_act), pow2f(pl->g_act),
+                  pow2f(-pl->g_act)};
+    const int mode = pl->fmt == OSM_FMT_NVFP4 ? QA_NV : (pl->hp_fp16 ? QA_MX_F16 : QA_MX);
     const int stride = qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp));
     // streaming form: two CTAs of at most 110 KB per SM
     const size_t two_per_sm = 110 * 1024;
     const int npairs = p.K / 2;
     if (stream_smem_bytes<2, 3>(p.K, stride) <= two_per_sm) {
-        if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, stride, st);
-        return launch_stream<2, 3, STREAM_NT, 0>(p, stride, st);
+        if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, mode, stride, st);
+        return launch_stream<2, 3, STREAM_NT, 0>(p, mode, stride, st);
     }
-    if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3, STREAM_NT, 0>(p, stride, st);
-    if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2, STREAM_NT, 0>(p, stride, st);
+    if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3, STREAM_NT, 0>(p, mode, stride, st);
+    if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2, STREAM_NT, 0>(p, mode, stride, st);
     // very wide rows: the staged, phase-serial form
     const size_t row_bytes = static_cast<size_t>(stride);
     const size_t budget = 72 * 1024;
-    if (row_bytes * 8 <= budget) return launch_qa<8>(p, row_bytes * 8, st);
-    if (row_bytes * 4 <= budget) return launch_qa<4>(p, row_bytes * 4, st);
-    if (row_bytes * 2 <= budget) return launch_qa<2>(p, row_bytes * 2, st);
-    if (row_bytes <= 200 * 1024) return launch_qa<1>(p, row_bytes, st);
+    if (row_bytes * 8 <= budget) return launch_qa<8>(p, mode, row_bytes * 8, st);
+    if (row_bytes * 4 <= budget) return launch_qa<4>(p, mode, row_bytes * 4, st);
+    if (row_bytes * 2 <= budget) return launch_qa<2>(p, mode, row_bytes * 2, st);
+    if (row_bytes <= 200 * 1024) return launch_qa<1>(p, mode, row_bytes, st);
     return fail(OSM_ERR_UNSUPPORTED, "quantize_act: K too large for one staged row");
 }
 

@@ -36,7 +36,7 @@ def gpu_calibrate(X: np.ndarray, W: np.ndarray, alpha: float, k: int, batches: i
 
 
 def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_sO=None, rows=None,
-              hp_fp16=False):
+              hp_fp16=False, nv=False):
     """Full CUDA path. Returns a dict of host arrays (rows of the activation
     outputs and of Y restricted to `rows` when given)."""
     M, K = X.shape
@@ -44,7 +44,11 @@ def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_
     Xd, Wd, s, inv_s, O, amax, wmax = gpu_calibrate(X, W, alpha, k, batches)
     if plan_sO is not None:
         s, O = plan_sO
-    plan = osm.Plan(K, N, k, s, O, mode, hp_fp16=hp_fp16)
+    g_act = g_w = 0
+    if nv:
+        g_act, g_w = osm.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+    plan = osm.Plan(K, N, k, s, O, mode, hp_fp16=hp_fp16, fmt=osm.FMT_NVFP4 if nv else osm.FMT_MXFP4,
+                    g_act=g_act, g_w=g_w)
     wc, wsc, wh = plan.alloc_packed(N)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M)
@@ -54,10 +58,10 @@ def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_
     osm.dual_gemm(plan, ac, asc, ah, M, wc, wsc, wh, Y, bias=bd, epi=epi)
     torch.cuda.synchronize()
     status = plan.status()
-    nb = plan.Kbp // 32
+    nb = plan.nblocks
     sel = slice(None) if rows is None else torch.from_numpy(np.asarray(rows)).cuda()
     out = dict(
-        s=s, inv_s=inv_s, O=O, amax=amax, wmax=wmax, status=status, plan=plan, M=M,
+        s=s, inv_s=inv_s, O=O, amax=amax, wmax=wmax, status=status, plan=plan, M=M, g=(g_act, g_w),
         w_codes=wc.cpu().numpy().reshape(N, plan.Kbp // 2),
         w_scales=unswizzle(wsc.cpu().numpy(), N, nb),
         w_hp=to_np_u16(wh).reshape(N, plan.kp),
@@ -69,15 +73,22 @@ def gpu_layer(X, W, alpha, k, mode, epi=osm.EPI_F32, bias=None, batches=1, plan_
     return out
 
 
-def oracle_layer(X, W, alpha, k, mode, rows=None, bias=None, hp_fp16=False):
+def oracle_layer(X, W, alpha, k, mode, rows=None, bias=None, hp_fp16=False, nv=False):
     amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
     s, inv_s, O = oracle.calibrate(amax, wmax, alpha, k)
-    wc, wsc, wh = oracle.pack_weights(W, s, O, mode, hp_fp16=hp_fp16)
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
-    ac, asc, ah = oracle.quantize_act(X[rows], inv_s, O, hp_fp16=hp_fp16)
-    y, T = oracle.dual_gemm_rows(ac, asc, ah, np.arange(len(rows)), wc, wsc, wh, bias, hp_fp16=hp_fp16)
+    g = None
+    if nv:
+        g = oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+        wc, wsc, wh = oracle.pack_weights_nv(W, s, O, g[1])
+        ac, asc, ah = oracle.quantize_act_nv(X[rows], inv_s, O, g[0])
+        y, T = oracle.dual_gemm_rows_nv(ac, asc, ah, np.arange(len(rows)), wc, wsc, wh, g[0], g[1], bias)
+    else:
+        wc, wsc, wh = oracle.pack_weights(W, s, O, mode, hp_fp16=hp_fp16)
+        ac, asc, ah = oracle.quantize_act(X[rows], inv_s, O, hp_fp16=hp_fp16)
+        y, T = oracle.dual_gemm_rows(ac, asc, ah, np.arange(len(rows)), wc, wsc, wh, bias, hp_fp16=hp_fp16)
     return dict(amax=amax, wmax=wmax, s=s, inv_s=inv_s, O=O, w_codes=wc, w_scales=wsc, w_hp=wh,
-                a_codes=ac, a_scales=asc, a_hp=ah, y=y, T=T, rows=rows)
+                a_codes=ac, a_scales=asc, a_hp=ah, y=y, T=T, rows=rows, g=g)
 
 
 def bits(a):
@@ -117,6 +128,8 @@ def compare_layer(g, o, rows=None, check_weights_rows=None):
     assert_bitexact("s", g["s"], o["s"])
     assert_bitexact("inv_s", g["inv_s"], o["inv_s"])
     assert_bitexact("O", g["O"], o["O"])
+    if o.get("g") is not None:
+        assert tuple(g["g"]) == tuple(o["g"]), ("NVFP4 tensor exponents", g["g"], o["g"])
     N = o["w_codes"].shape[0]
     wr = np.arange(N) if check_weights_rows is None else check_weights_rows
     assert_bitexact("w_codes", g["w_codes"][wr], o["w_codes"][wr])

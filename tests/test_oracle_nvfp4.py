@@ -246,3 +246,19 @@ def test_dual_gemm_nv_all_outliers_is_the_bf16_product():
     xs = synth.bf16_bits_to_f32(oracle.smooth_act(X, inv_s)).astype(np.float64)
     ws = synth.bf16_bits_to_f32(oracle.fold_weights(W, s)).astype(np.float64)
     np.testing.assert_allclose(y, xs @ ws, rtol=1e-12, atol=1e-12)
+
+
+def test_library_host_exponents_equal_the_oracle():
+    # osm_nvfp4_tensor_exponent / osm_nvfp4_plan_exponents are host code in
+    # libosm: no GPU needed.
+    import outlier_split_mixed_b200 as osm
+    rng = np.random.default_rng(17)
+    for a in np.concatenate([np.exp(rng.uniform(-50, 50, 200)), [0.0, 2688.0, 2689.0]]).astype(np.float32):
+        assert osm.nvfp4_tensor_exponent(float(a)) == oracle.nvfp4_tensor_exponent(float(a))
+    for seed, k in ((1, 0), (2, 17), (3, 200)):
+        M, K, N = 96, 512, 64
+        X = synth.acts_heavy_tailed(M, K, seed, frac=0.03)
+        W = synth.weights_gaussian(K, N, seed + 50, 0.05)
+        amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
+        s, inv_s, O = oracle.calibrate(amax, wmax, 0.6, k)
+        assert osm.nvfp4_plan_exponents(amax, wmax, s, inv_s, O) == oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
