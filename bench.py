@@ -76,6 +76,13 @@ def workload_config(cfg):
     return {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "k": cfg.k, "alpha": cfg.alpha}
 
 
+def fmt_config(args, cfg):
+    """The 4-bit format and weight-scale mode a layer workload runs with."""
+    if getattr(args, "nvfp4", False):
+        return {"format": "nvfp4", "wscale": "1x16"}
+    return {"format": "mxfp4", "wscale": WSCALE_NAMES[cfg.wmode]} if hasattr(cfg, "wmode") else {"format": "mxfp4"}
+
+
 def blended_peak(peaks, parts):
     """Tensor-pipe peak for a mix of FP4 and BF16 MMAs: parts is a list of
     (fp4_flops, bf16_flops); FP4 runs at the measured BF16 burst x 4 (the
@@ -147,10 +154,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_sample_throughput(cfg, rows_per_step: int, steps: int, warmup: int):
-    """Time the CPU oracle (quantize_act + dual-branch product) on
-    `rows_per_step` tokens of the workload per step. Weights are packed
-    offline, outside the timed region, as on the GPU path."""
+def oracle_sample_throughput(cfg, rows_per_step: int, steps: int, warmup: int, nv: bool = False):
+    """Time the CPU oracle (quantize_act + dual-branch product, MXFP4 or
+    NVFP4) on `rows_per_step` tokens of the workload per step. Weights are
+    packed offline, outside the timed region, as on the GPU path."""
     import oracle
     from outlier_split_mixed_b200 import synth
     M_s = rows_per_step * (steps + warmup)
@@ -158,14 +165,22 @@ def oracle_sample_throughput(cfg, rows_per_step: int, steps: int, warmup: int):
     W = cfg.make_w()
     amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
     s, inv_s, O = oracle.calibrate(amax, wmax, cfg.alpha, cfg.k)
-    wc, wsc, wh = oracle.pack_weights(W, s, O, cfg.wmode)
+    if nv:
+        ga, gw = oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+        wc, wsc, wh = oracle.pack_weights_nv(W, s, O, gw)
+    else:
+        wc, wsc, wh = oracle.pack_weights(W, s, O, cfg.wmode)
     times = []
     for i in range(steps + warmup):
         lo = (i * rows_per_step) % max(1, X.shape[0] - rows_per_step)
         xr = X[lo:lo + rows_per_step]
         t0 = time.perf_counter()
-        ac, asc, ah = oracle.quantize_act(xr, inv_s, O)
-        oracle.dual_gemm_rows(ac, asc, ah, np.arange(rows_per_step), wc, wsc, wh)
+        if nv:
+            ac, asc, ah = oracle.quantize_act_nv(xr, inv_s, O, ga)
+            oracle.dual_gemm_rows_nv(ac, asc, ah, np.arange(rows_per_step), wc, wsc, wh, ga, gw)
+        else:
+            ac, asc, ah = oracle.quantize_act(xr, inv_s, O)
+            oracle.dual_gemm_rows(ac, asc, ah, np.arange(rows_per_step), wc, wsc, wh)
         t1 = time.perf_counter()
         if i >= warmup:
             times.append(t1 - t0)
@@ -226,14 +241,14 @@ def run_reference(args, cfg, rank, world):
     if is_ffn:
         tflops, t, cores = oracle_ffn_throughput(cfg, rows, args.steps, args.warmup)
     else:
-        tflops, t, cores = oracle_sample_throughput(cfg, rows, args.steps, args.warmup)
+        tflops, t, cores = oracle_sample_throughput(cfg, rows, args.steps, args.warmup, nv=args.nvfp4)
     line = {
         "impl": "reference",
         "metric": METRIC,
         "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": dict(workload_config(cfg), sample_rows_per_step=rows),
+        "config": dict(workload_config(cfg), sample_rows_per_step=rows, **fmt_config(args, cfg)),
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows} of {cfg.M} tokens per step, weights packed offline"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -269,7 +284,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     osm.act_amax_accumulate(Xd, amax)
     osm.weight_amax(Wd, wmax)
     s, inv_s, O = odist.calibrate_from_local_stats(amax, wmax, cfg.alpha, cfg.k)
-    plan = osm.Plan(K, N, cfg.k, s, O, cfg.wmode, hp_fp16=args.hp_fp16)
+    plan = osm.Plan(K, N, cfg.k, s, O, osm.WSCALE_1x32 if args.nvfp4 else cfg.wmode, hp_fp16=args.hp_fp16)
+    if args.nvfp4:
+        amax_all = odist.allreduce_max_(amax.clone())
+        plan.set_format(osm.FMT_NVFP4, *osm.nvfp4_plan_exponents(amax_all.cpu().numpy(), wmax.cpu().numpy(), s,
+                                                                 inv_s, O))
     wc, wsc, wh = plan.alloc_packed(N, dev)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M, dev)
@@ -351,9 +370,10 @@ def run_ours(args, cfg, rank, world, local_rank):
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
+            "dtype": ("nvfp4(e2m1,ue4m3 per 16,2^g per tensor)" if args.nvfp4 else "mxfp4(e2m1,e8m0)")
+                     + "+bf16, fp32 accumulate", "data": "synthetic",
             "config": {"workload": cfg.name, "M_per_gpu": M, "K": K, "N": N, "k": cfg.k, "alpha": cfg.alpha,
-                       "wscale": {0: "1x32", 1: "32x32", 2: "128x1"}[cfg.wmode],
+                       **fmt_config(args, cfg), "g": [plan.g_act, plan.g_w] if args.nvfp4 else None,
                        "out": "bf16" if cfg.out_bf16 else "f32",
                        "outlier_branch": "fp16" if args.hp_fp16 else "bf16",
                        "l2": "flushed between timed steps (256 MiB write, untimed)",
@@ -377,7 +397,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            tf, t, cores = oracle_sample_throughput(cfg, args.cpu_rows, 2, 1)
+            tf, t, cores = oracle_sample_throughput(cfg, args.cpu_rows, 2, 1, nv=args.nvfp4)
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                     "sample": f"{args.cpu_rows} of {M} tokens per step (2 steps), weights "
                                               f"packed offline"}
@@ -700,11 +720,15 @@ def main():
                     help="override the workload's token count (small cases for profiler captures)")
     ap.add_argument("--blocks", type=int, default=0, help="override the number of FFN blocks (ffn workload)")
     ap.add_argument("--hp-fp16", action="store_true", help="outlier branch in FP16 instead of BF16")
+    ap.add_argument("--nvfp4", action="store_true",
+                    help="layer workloads: NVFP4 bulk format (16-blocks, UE4M3 scales) instead of MXFP4")
     ap.add_argument("--percentile", type=float, default=0.0,
                     help="refresh workload: score channels by this percentile of |x| (0: by the maximum)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.nvfp4 and (args.workload in ("ffn", "refresh", "search") or args.hp_fp16):
+        ap.error("--nvfp4 applies to the layer workloads (up, down, long, tiny) with the BF16 outlier branch")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
