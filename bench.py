@@ -61,10 +61,16 @@ METRIC = "dual-branch W4A4 GEMM effective TFLOP/s (+act quantize)"
 
 WSCALE_NAMES = {0: "1x32", 1: "32x32", 2: "128x1"}
 
+# streams that consecutive end-to-end steps rotate over (copies of one step
+# overlap the kernels of another)
+E2E_STREAMS = 3
+
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one dual_gemm
-# launch, from one ncu capture of the current kernel on the workload; a
-# workload without a capture of the current kernel reports null.
-DUAL_GEMM_TRAFFIC = {"wan_ffn_up_4096x5120x13824": 92.180992e6 + 179.756544e6}
+# launch, from one ncu capture of the current kernel on the workload, per
+# (workload, bulk format); a workload without a capture of the current
+# kernel reports null.
+DUAL_GEMM_TRAFFIC = {("wan_ffn_up_4096x5120x13824", "mxfp4"): 92.17e6 + 178.10e6,
+                     ("wan_ffn_up_4096x5120x13824", "nvfp4"): 97.07e6 + 178.99e6}
 
 
 def workload_config(cfg):
@@ -330,20 +336,29 @@ def run_ours(args, cfg, rank, world, local_rank):
         dist.all_reduce(loc, op=dist.ReduceOp.MAX)
     step_s, gemm_s, quant_s = (float(x) for x in loc.cpu())
 
-    # end-to-end through the host entry point: pinned X in, Y out
+    # end-to-end through the host entry point: pinned X in, Y out, every
+    # step. Consecutive steps rotate over E2E_STREAMS streams (each with its
+    # own workspace and host Y), so one step's copy in, another's kernels
+    # and a third's copy out overlap, as a serving loop would run them.
     Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Yh = torch.empty((M, N), dtype=Y.dtype).pin_memory()
-    ws = torch.empty(osm.linear_workspace_size(plan, M, epi), dtype=torch.uint8, device=dev)
-    e2e_steps = max(3, min(20, n))
-    for _ in range(2):
-        osm.linear_host(plan, Xh, M, wc, wsc, wh, Yh, ws, epi=epi)
+    streams = [torch.cuda.Stream(device=dev) for _ in range(E2E_STREAMS)]
+    Yhs = [torch.empty((M, N), dtype=Y.dtype).pin_memory() for _ in streams]
+    wss = [torch.empty(osm.linear_workspace_size(plan, M, epi), dtype=torch.uint8, device=dev) for _ in streams]
+    e2e_steps = max(3 * E2E_STREAMS, min(24, n))
+    for j in range(E2E_STREAMS):
+        osm.linear_host(plan, Xh, M, wc, wsc, wh, Yhs[j], wss[j], epi=epi, stream=streams[j])
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    for _ in range(e2e_steps):
-        osm.linear_host(plan, Xh, M, wc, wsc, wh, Yh, ws, epi=epi)
+    for st in streams:
+        st.wait_event(e0)
+    for i in range(e2e_steps):
+        j = i % E2E_STREAMS
+        osm.linear_host(plan, Xh, M, wc, wsc, wh, Yhs[j], wss[j], epi=epi, stream=streams[j])
+    for st in streams:
+        stream.wait_stream(st)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_t = torch.tensor([e0.elapsed_time(e1) * 1e-3 / e2e_steps], dtype=torch.float64, device=dev)
@@ -386,13 +401,15 @@ def run_ours(args, cfg, rank, world, local_rank):
                                  "frac_hbm": q_gbs / peaks["hbm_gbs"]},
             },
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
-                         "frac": achieved / peak_blend, "traffic": DUAL_GEMM_TRAFFIC.get(cfg.name),
+                         "frac": achieved / peak_blend,
+                         "traffic": None if args.hp_fp16 else DUAL_GEMM_TRAFFIC.get((cfg.name,
+                                                                                    fmt_config(args, cfg)["format"])),
                          "traffic_unit": "bytes per launch", "kernel": "dual_gemm",
                          "peak_source": f"{peak_src}: bf16 burst {p16} x4 for the FP4 share, x1 for the "
                                         f"BF16 share (k={plan.k} of K={K})"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * Y.element_size(),
-                    "api": "osm_linear_host"},
+                    "api": f"osm_linear_host, steps rotated over {E2E_STREAMS} streams"},
             "gpu_launches": 2 * n,
             "clocks": clk.summary(),
         }
@@ -516,11 +533,32 @@ def run_ffn(args, cfg, rank, world, local_rank):
     Xh = [torch.from_numpy(b["X"].view(np.int16)).view(torch.bfloat16).pin_memory() for b in blocks]
     Yh = [torch.empty((M, D), dtype=torch.bfloat16).pin_memory() for _ in blocks]
 
+    # Three streams: copies in, the blocks' kernels, copies out. Block l's
+    # input copy waits until the previous step's kernels of block l are done
+    # with its device buffers, its kernels wait for its input, and its output
+    # copy for its kernels, so copies of one block overlap another's compute.
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_done = [torch.cuda.Event() for _ in blocks]
+    comp_done = [torch.cuda.Event() for _ in blocks]
+    out_done = [torch.cuda.Event() for _ in blocks]
+    for l in range(len(blocks)):
+        comp_done[l].record(stream)
+        out_done[l].record(stream)
+
     def e2e_step():
-        for b, xh, yh in zip(blocks, Xh, Yh):
-            b["Xd"].copy_(xh, non_blocking=True)
+        for l, (b, xh, yh) in enumerate(zip(blocks, Xh, Yh)):
+            s_in.wait_event(comp_done[l])
+            with torch.cuda.stream(s_in):
+                b["Xd"].copy_(xh, non_blocking=True)
+            in_done[l].record(s_in)
+            stream.wait_event(in_done[l])
+            stream.wait_event(out_done[l])
             block(b)
-            yh.copy_(b["Y"], non_blocking=True)
+            comp_done[l].record(stream)
+            s_out.wait_event(comp_done[l])
+            with torch.cuda.stream(s_out):
+                yh.copy_(b["Y"], non_blocking=True)
+            out_done[l].record(s_out)
 
     e2e_steps = max(3, min(10, n))
     e2e_step()
@@ -529,8 +567,12 @@ def run_ffn(args, cfg, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
     for _ in range(e2e_steps):
         e2e_step()
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_t = torch.tensor([e0.elapsed_time(e1) * 1e-3 / e2e_steps], dtype=torch.float64, device=dev)
@@ -573,7 +615,7 @@ def run_ffn(args, cfg, rank, world, local_rank):
                                         f"share (k_up={up0.k}, k_down={dn0.k})"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": L * M * D * 2, "d2h_bytes_per_step": L * M * D * 2,
-                    "api": "quantize_act + dual_gemm (Python binding), pinned host copies"},
+                    "api": "quantize_act + dual_gemm (Python binding); pinned host copies on their own in / out streams, overlapping other blocks' kernels"},
             "gpu_launches": 3 * L * n,
             "clocks": clk.summary(),
         }
