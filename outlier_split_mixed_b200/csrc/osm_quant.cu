@@ -124,25 +124,55 @@ __global__ void __launch_bounds__(128) act_amax_kernel(const uint16_t* __restric
 // histograms padded so that equal buckets of different channels fall in
 // different banks.
 constexpr int PCT_THREADS = 256;
+constexpr int PCT_SPLIT = 4;   // CTAs of a cluster, each taking a quarter of the rows
+constexpr int PCT_UNROLL = 8;  // rows per warp loaded before their histogram updates
 
-__global__ void __launch_bounds__(PCT_THREADS) act_percentile_kernel(const uint16_t* __restrict__ X, int64_t T,
-                                                                     int64_t K, int64_t rank,
-                                                                     float* __restrict__ score) {
+// score[j] = the rank-th smallest |x_tj| (1-based) for 32 channels per
+// cluster of PCT_SPLIT CTAs: BF16 magnitudes are 15-bit keys, so two
+// histogram passes (the high 8 bits, then the low 7 bits inside the chosen
+// bucket) find the rank exactly. Each CTA histograms its share of the rows
+// (eight independent row loads per warp in flight), the shares are added
+// into the first CTA's histogram through distributed shared memory, the
+// first CTA picks the bucket and hands it back to the others.
+__global__ void __cluster_dims__(PCT_SPLIT, 1, 1) __launch_bounds__(PCT_THREADS)
+    act_percentile_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t K, int64_t rank,
+                          float* __restrict__ score) {
     __shared__ unsigned hist[32][257];
     __shared__ unsigned pick[32], rem[32];
+    constexpr int NW = PCT_THREADS / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;  // K % 32 == 0
+    const uint32_t crank = ptx::cluster_ctarank();
+    const int64_t j = static_cast<int64_t>(blockIdx.y) * 32 + lane;  // K % 32 == 0
+    const int64_t chunk = (T + PCT_SPLIT - 1) / PCT_SPLIT;
+    const int64_t t0 = static_cast<int64_t>(crank) * chunk;
+    const int64_t t1 = min(T, t0 + chunk);
+    const uint32_t hist0 = ptx::mapa(ptx::smem_u32(&hist[0][0]), 0);
     for (int pass = 0; pass < 2; ++pass) {
         for (int i = threadIdx.x; i < 32 * 257; i += PCT_THREADS) (&hist[0][0])[i] = 0;
         __syncthreads();
         const unsigned hi = pass ? pick[lane] : 0u;
-        for (int64_t t = warp; t < T; t += PCT_THREADS / 32) {
-            const unsigned key = X[t * K + j] & 0x7FFFu;
-            if (pass == 0) atomicAdd(&hist[lane][key >> 7], 1u);
-            else if ((key >> 7) == hi) atomicAdd(&hist[lane][key & 127u], 1u);
+        for (int64_t t = t0 + warp; t < t1; t += PCT_UNROLL * NW) {
+            unsigned key[PCT_UNROLL];
+#pragma unroll
+            for (int u = 0; u < PCT_UNROLL; ++u) {
+                const int64_t tu = t + u * NW;
+                key[u] = tu < t1 ? (__ldg(X + tu * K + j) & 0x7FFFu) : 0xFFFFFFFFu;
+            }
+#pragma unroll
+            for (int u = 0; u < PCT_UNROLL; ++u) {
+                if (key[u] == 0xFFFFFFFFu) continue;
+                if (pass == 0) atomicAdd(&hist[lane][key[u] >> 7], 1u);
+                else if ((key[u] >> 7) == hi) atomicAdd(&hist[lane][key[u] & 127u], 1u);
+            }
         }
-        __syncthreads();
-        if (threadIdx.x < 32) {
+        ptx::cluster_sync();  // every share complete
+        if (crank != 0)
+            for (int i = threadIdx.x; i < 32 * 257; i += PCT_THREADS) {
+                const unsigned v = (&hist[0][0])[i];
+                if (v) ptx::red_add_cluster_u32(hist0 + 4u * i, v);
+            }
+        ptx::cluster_sync();  // the first CTA holds the whole histogram
+        if (crank == 0 && threadIdx.x < 32) {
             const int c = threadIdx.x;
             unsigned need = pass ? rem[c] : static_cast<unsigned>(rank);
             const int nb = pass ? 128 : 256;
@@ -154,11 +184,13 @@ __global__ void __launch_bounds__(PCT_THREADS) act_percentile_kernel(const uint1
             if (pass == 0) {
                 pick[c] = static_cast<unsigned>(b);
                 rem[c] = need;
+                for (uint32_t r = 1; r < PCT_SPLIT; ++r)
+                    ptx::st_cluster_u32(ptx::mapa(ptx::smem_u32(&pick[c]), r), static_cast<unsigned>(b));
             } else {
-                score[static_cast<int64_t>(blockIdx.x) * 32 + c] = __uint_as_float(((pick[c] << 7) | b) << 16);
+                score[static_cast<int64_t>(blockIdx.y) * 32 + c] = __uint_as_float(((pick[c] << 7) | b) << 16);
             }
         }
-        __syncthreads();
+        ptx::cluster_sync();  // the bucket of pass 0 is known everywhere; no CTA touches another's memory after
     }
 }
 
@@ -738,7 +770,8 @@ int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaSt
 }
 
 int launch_act_percentile(const uint16_t* X, int64_t T, int64_t K, int64_t rank, float* score, cudaStream_t st) {
-    act_percentile_kernel<<<static_cast<unsigned>(K / 32), PCT_THREADS, 0, st>>>(X, T, K, rank, score);
+    act_percentile_kernel<<<dim3(PCT_SPLIT, static_cast<unsigned>(K / 32)), PCT_THREADS, 0, st>>>(X, T, K, rank,
+                                                                                              score);
     return check_cuda(cudaGetLastError(), "act_percentile launch");
 }
 
