@@ -618,6 +618,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_before();
     ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
     ptx::tc_fence_after();
+    // Everything above overlaps the tail of the previous kernel on the stream
+    // (a dependent launch); operands and outputs are touched only after it.
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const uint32_t tmem = S.tmem_base;
     // Warpgroup-uniform register split (for the epilogues that need it). Each
     // side ends with its own copy of the teardown, so that no code is shared
@@ -801,8 +805,19 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
     if (tiles > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "dual_gemm: too many tiles");
     const int pairs = static_cast<int>(tiles < li.max_pairs ? tiles : li.max_pairs);
-    kernel<<<2 * pairs, NUM_THREADS, smem, st>>>(p);
-    return check_cuda(cudaGetLastError(), "dual_gemm launch");
+    // a dependent launch: the prologue may run while the previous kernel on
+    // the stream (normally quantize_act) finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return check_cuda(cudaLaunchKernelEx(&cfg, kernel, p), "dual_gemm launch");
 }
 
 }  // namespace osm

@@ -254,6 +254,14 @@ __device__ __forceinline__ void tma_store_2d_hint(const void* tmap, int32_t x, i
                  : "memory");
 }
 
+// ---------------------------------------------------- dependent launches
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel on the stream is still running; grid_dep_wait blocks
+// until that kernel has completed and its memory operations are visible.
+// grid_dep_launch lets the next such kernel start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -477,6 +477,7 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p);
 template <int R, int MODE>
 __global__ void __launch_bounds__(QA_THREADS) quantize_act_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
+    ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
     extern __shared__ __align__(16) uint8_t sbuf[];
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
@@ -630,6 +631,7 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 template <int R, int S, int NT, int TR, int MODE>
 __global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
+    ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
     extern __shared__ __align__(128) uint8_t smem[];
     const int nb = p.Kbp >> 5;
     const int stride = qa_row_stride(nb, p.kp);
