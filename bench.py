@@ -101,6 +101,28 @@ def blended_peak(peaks, parts):
     return (f4 + f16) / t_ideal / 1e12, p16
 
 
+# ------------------------------------------------------------------ L2 flush
+
+L2_NOTE = ("flushed between timed steps (untimed): a 256 MiB write, then a 256 MiB read so that the "
+           "written lines are evicted before the step")
+
+
+class L2Flush:
+    """Between timed steps: write a 256 MiB buffer (twice the 126 MB L2), then
+    read another 256 MiB buffer, so that the step starts with none of its
+    inputs in L2 and without dirty lines of the flush still to be written back
+    (which would otherwise be charged to the step's first kernel)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self, v: float = 1.0):
+        self.w.fill_(v)
+        self._sink = self.r.sum()
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -299,14 +321,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M, dev)
     Y = torch.empty((M, N), dtype=torch.float32 if epi == osm.EPI_F32 else torch.bfloat16, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
+    flush = L2Flush(dev)
 
     def step():
         osm.quantize_act(plan, Xd, ac, asc, ah)
         osm.dual_gemm(plan, ac, asc, ah, M, wc, wsc, wh, Y, epi=epi)
 
     for _ in range(args.warmup):
-        flush.fill_(1.0)
+        flush(1.0)
         step()
     torch.cuda.synchronize()
 
@@ -322,13 +344,13 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(n):
-            flush.fill_(float(i))                    # evict L2 between timed steps (untimed)
+            flush(float(i))                          # evict L2 between timed steps (untimed)
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         for i in range(n):
-            flush.fill_(float(i))
+            flush(float(i))
             evs[i][0].record(stream)
             osm.quantize_act(plan, Xd, ac, asc, ah)
             evs[i][1].record(stream)
@@ -402,7 +424,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                        **fmt_config(args, cfg), "g": [plan.g_act, plan.g_w] if args.nvfp4 else None,
                        "out": "bf16" if cfg.out_bf16 else "f32",
                        "outlier_branch": "fp16" if args.hp_fp16 else "bf16",
-                       "l2": "flushed between timed steps (256 MiB write, untimed)",
+                       "l2": L2_NOTE,
                        "parallelism": f"dp{world} (token shards, no data-path collective)"},
             "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
             "kernels": {
@@ -491,7 +513,7 @@ def run_ffn(args, cfg, rank, world, local_rank):
     for b in blocks:
         b["Xd"] = to_dev(b["X"])
         b["Y"] = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
 
     def block(b, ev=None):
         if ev is not None:
@@ -508,7 +530,7 @@ def run_ffn(args, cfg, rank, world, local_rank):
             ev[3].record(stream)
 
     for _ in range(args.warmup):
-        flush.fill_(1.0)
+        flush(1.0)
         for b in blocks:
             block(b)
     torch.cuda.synchronize()
@@ -526,14 +548,14 @@ def run_ffn(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(n):
-            flush.fill_(float(i))                    # evict L2 between timed steps (untimed)
+            flush(float(i))                          # evict L2 between timed steps (untimed)
             evt[i][0].record(stream)
             for b in blocks:
                 block(b)
             evt[i][1].record(stream)
         torch.cuda.synchronize()
         for i in range(n):
-            flush.fill_(float(i))
+            flush(float(i))
             for l, b in enumerate(blocks):
                 block(b, ev[i][l])
         torch.cuda.synchronize()
@@ -622,7 +644,7 @@ def run_ffn(args, cfg, rank, world, local_rank):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
-            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
+            "config": dict(workload_config(cfg), l2=L2_NOTE,
                            parallelism=f"dp{world} (token shards, no data-path collective)",
                            outlier_branch="fp16" if args.hp_fp16 else "bf16"),
             "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
@@ -674,7 +696,7 @@ def run_refresh(args, cfg, rank, world, local_rank):
     amax = torch.zeros(K, dtype=torch.float32, device=dev)
     plan = osm.Plan(K, N, cfg.k, np.ones(K, np.float32), np.arange(cfg.k, dtype=np.int32), cfg.wmode)
     wc, wsc, wh = plan.alloc_packed(N, dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
 
     score = torch.empty(K, dtype=torch.float32, device=dev) if args.percentile else None
 
@@ -698,14 +720,14 @@ def run_refresh(args, cfg, rank, world, local_rank):
             ev[3].record(stream)
 
     for _ in range(args.warmup):
-        flush.fill_(1.0)
+        flush(1.0)
         step()
     torch.cuda.synchronize()
     n = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     with ClockSampler(local_rank) as clk:
         for i in range(n):
-            flush.fill_(float(i))
+            flush(float(i))
             step(ev[i])
         torch.cuda.synchronize()
     if plan.status() != 0:
@@ -721,7 +743,7 @@ def run_refresh(args, cfg, rank, world, local_rank):
             "value": step_s * 1e6, "unit": "us", "n_gpus": world, "steps": n, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 in, mxfp4+bf16 out", "data": "synthetic",
-            "config": dict(workload_config(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
+            "config": dict(workload_config(cfg), l2=L2_NOTE,
                            channel_score=f"percentile {args.percentile}" if args.percentile else "maximum"),
             "kernels": {
                 "act_stats": {"us": t[0] * 1e6, "gbs": M * K * 2 * (2 if args.percentile else 1) / t[0] / 1e9},

@@ -245,33 +245,47 @@ struct PackParams {
 
 constexpr int PK_THREADS = 256;
 
-// Load rows src_row(r) of W (r < nrows; a negative row is zero), columns
-// n0 .. n0+127 (packed order: W column col_order[n] when col_order is set),
-// as w' = bf16(fp32(w) * s[row]) into tile[r][0..63] (BF16 pairs).
+// Load rows src_row(r) of W (r < nrows <= 128; a negative row is zero),
+// columns n0 .. n0+127 (packed order: W column col_order[n] when col_order
+// is set), as w' = bf16(fp32(w) * s[row]) into tile[r][0..63] (BF16
+// pairs). Each thread issues all its 16-byte row loads (up to eight) before
+// it folds and stores any of them, so that they are in flight together.
 template <bool F16, typename RowOf>
 __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0, int nrows, RowOf src_row,
                                                  uint32_t (*tile)[64]) {
-    for (int t = threadIdx.x; t < nrows * 16; t += PK_THREADS) {
+    constexpr int PER = 128 * 16 / PK_THREADS;
+    uint4 w[PER];
+    float sj[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int t = threadIdx.x + i * PK_THREADS;
+        w[i] = make_uint4(0, 0, 0, 0);
+        sj[i] = 0.0f;
+        if (t >= nrows * 16) continue;
         const int r = t >> 4, c = t & 15;
         const int64_t j = src_row(r);
         const int64_t n = n0 + 8 * c;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (j >= 0 && n < p.N) {
-            const float sj = __ldg(p.s + j);
-            const float2 s2 = make_float2(sj, sj);
-            uint4 w;
-            if (p.col_order == nullptr) {
-                w = ldg_nc_v4(p.W + j * p.N + n);
-            } else {
-                uint32_t e[8];
+        if (j < 0 || n >= p.N) continue;
+        sj[i] = __ldg(p.s + j);
+        if (p.col_order == nullptr) {
+            w[i] = ldg_nc_v4(p.W + j * p.N + n);
+        } else {
+            uint32_t e[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) e[i] = p.W[j * p.N + __ldg(p.col_order + n + i)];
-                w = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
-            }
-            const uint32_t m = F16 ? 0xFFFFFFFFu : 0u;
-            v = make_uint4(smooth2_mixed(w.x, s2, m), smooth2_mixed(w.y, s2, m), smooth2_mixed(w.z, s2, m),
-                           smooth2_mixed(w.w, s2, m));
+            for (int u = 0; u < 8; ++u) e[u] = p.W[j * p.N + __ldg(p.col_order + n + u)];
+            w[i] = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
         }
+    }
+    const uint32_t m = F16 ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int t = threadIdx.x + i * PK_THREADS;
+        if (t >= nrows * 16) continue;
+        const int r = t >> 4, c = t & 15;
+        const float2 s2 = make_float2(sj[i], sj[i]);
+        // a zero row (j < 0 or n >= N) folds to +0 either way
+        const uint4 v = make_uint4(smooth2_mixed(w[i].x, s2, m), smooth2_mixed(w[i].y, s2, m),
+                                   smooth2_mixed(w[i].z, s2, m), smooth2_mixed(w[i].w, s2, m));
         *reinterpret_cast<uint4*>(&tile[r][4 * c]) = v;
     }
 }
