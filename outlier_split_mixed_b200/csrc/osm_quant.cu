@@ -71,58 +71,67 @@ __device__ __forceinline__ uint32_t slot_mask(int2 dv, int slot0) {
 
 // ------------------------------------------------------------ calibration
 
-constexpr int AMAX_ROWS = 32;
+constexpr int AMAX_THREADS = 256;
+constexpr int AMAX_ROWS = 256;  // rows per CTA: 32 per warp
 
-// amax[j] = max(amax[j], max_t |X[t][j]|). One thread per 8 channels and
-// AMAX_ROWS rows, eight 16-byte row loads in flight; the maxima are kept as
-// packed u16 pairs of |x| bit patterns (integer order, so a NaN pattern
-// propagates and the finiteness check of the calibration sees it) and
-// merged with atomicMax on the IEEE bit pattern of the FP32 value
-// (monotone for non-negative floats).
-__global__ void __launch_bounds__(128) act_amax_kernel(const uint16_t* __restrict__ X, int64_t T,
-                                                       int64_t K, float* __restrict__ amax) {
-    const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (v * 8 >= K) return;
+// amax[j] = max(amax[j], max_t |X[t][j]|). A CTA covers 256 channels (a
+// lane takes 8 channels, 16 bytes of a row) and AMAX_ROWS rows (warp w
+// takes rows w, w + 8, ...), with eight 16-byte row loads per lane in
+// flight; the maxima are kept as packed u16 pairs of |x| bit patterns
+// (integer order, so a NaN pattern propagates and the finiteness check of
+// the calibration sees it), combined over the warps in shared memory and
+// merged with one atomicMax per channel and CTA on the IEEE bit pattern of
+// the FP32 value (monotone for non-negative floats).
+__global__ void __launch_bounds__(AMAX_THREADS) act_amax_kernel(const uint16_t* __restrict__ X, int64_t T,
+                                                                int64_t K, float* __restrict__ amax) {
+    constexpr int NW = AMAX_THREADS / 32;
+    __shared__ uint32_t red[NW][32][4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t v = static_cast<int64_t>(blockIdx.x) * 32 + lane;  // 8-channel group
+    const bool active = v * 8 < K;
     const int64_t t0 = static_cast<int64_t>(blockIdx.y) * AMAX_ROWS;
     const int64_t t1 = min(T, t0 + AMAX_ROWS);
     uint32_t m[4] = {0, 0, 0, 0};
     const uint16_t* src = X + v * 8;
-    int64_t t = t0;
-    for (; t + 8 <= t1; t += 8) {
-        uint4 q[8];
+    if (active) {
+        for (int64_t t = t0 + warp; t < t1; t += 8 * NW) {
+            uint4 q[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) q[u] = ldg_nc_v4(src + (t + u) * K);
+            for (int u = 0; u < 8; ++u) {
+                const int64_t tu = t + u * NW;
+                q[u] = tu < t1 ? ldg_nc_v4(src + tu * K) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            m[0] = vmax_u16x2(m[0], q[u].x & 0x7FFF7FFFu);
-            m[1] = vmax_u16x2(m[1], q[u].y & 0x7FFF7FFFu);
-            m[2] = vmax_u16x2(m[2], q[u].z & 0x7FFF7FFFu);
-            m[3] = vmax_u16x2(m[3], q[u].w & 0x7FFF7FFFu);
+            for (int u = 0; u < 8; ++u) {
+                m[0] = vmax_u16x2(m[0], q[u].x & 0x7FFF7FFFu);
+                m[1] = vmax_u16x2(m[1], q[u].y & 0x7FFF7FFFu);
+                m[2] = vmax_u16x2(m[2], q[u].z & 0x7FFF7FFFu);
+                m[3] = vmax_u16x2(m[3], q[u].w & 0x7FFF7FFFu);
+            }
         }
     }
-    for (; t < t1; ++t) {
-        const uint4 q = ldg_nc_v4(src + t * K);
-        m[0] = vmax_u16x2(m[0], q.x & 0x7FFF7FFFu);
-        m[1] = vmax_u16x2(m[1], q.y & 0x7FFF7FFFu);
-        m[2] = vmax_u16x2(m[2], q.z & 0x7FFF7FFFu);
-        m[3] = vmax_u16x2(m[3], q.w & 0x7FFF7FFFu);
-    }
-    unsigned int* dst = reinterpret_cast<unsigned int*>(amax) + v * 8;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        atomicMax(dst + 2 * i, (m[i] & 0xFFFFu) << 16);
-        atomicMax(dst + 2 * i + 1, m[i] & 0xFFFF0000u);
+    for (int i = 0; i < 4; ++i) red[warp][lane][i] = m[i];
+    __syncthreads();
+    if (warp == 0 && active) {
+#pragma unroll
+        for (int w = 1; w < NW; ++w)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m[i] = vmax_u16x2(m[i], red[w][lane][i]);
+        unsigned int* dst = reinterpret_cast<unsigned int*>(amax) + v * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            atomicMax(dst + 2 * i, (m[i] & 0xFFFFu) << 16);
+            atomicMax(dst + 2 * i + 1, m[i] & 0xFFFF0000u);
+        }
     }
 }
 
 // Tail-aware channel score (the activation-tail-aware percentile
 // calibration of the Tail-Aware HiFloat4 page): score[j] = the rank-th
 // smallest |x_tj| over the T tokens (rank 1-based; the host derives it from
-// the percentile q as ceil(q T)). One CTA per 32 channels, lane = channel,
-// warps over rows; a two-pass radix select on the 15-bit |x| pattern (high
-// 8 bits, then the low 7 within the chosen bucket) with per-channel shared
-// histograms padded so that equal buckets of different channels fall in
-// different banks.
+// the percentile q as ceil(q T)). Per-channel shared histograms are padded
+// so that equal buckets of different channels fall in different banks.
 constexpr int PCT_THREADS = 256;
 constexpr int PCT_SPLIT = 4;   // CTAs of a cluster, each taking a quarter of the rows
 constexpr int PCT_UNROLL = 8;  // rows per warp loaded before their histogram updates
@@ -779,9 +788,9 @@ size_t stream_smem_bytes(int K, int stride) {
 
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st) {
     if (T == 0) return OSM_OK;
-    dim3 grid(static_cast<unsigned>(ceil_div(K / 8, 128)), static_cast<unsigned>(ceil_div(T, AMAX_ROWS)));
+    dim3 grid(static_cast<unsigned>(ceil_div(K / 8, 32)), static_cast<unsigned>(ceil_div(T, AMAX_ROWS)));
     if (grid.y > 65535u) return fail(OSM_ERR_UNSUPPORTED, "act_amax: T too large for one launch");
-    act_amax_kernel<<<grid, 128, 0, st>>>(X, T, K, amax);
+    act_amax_kernel<<<grid, AMAX_THREADS, 0, st>>>(X, T, K, amax);
     return check_cuda(cudaGetLastError(), "act_amax launch");
 }
 
