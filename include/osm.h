@@ -42,7 +42,12 @@
  *          (r%32)*16 + ((r%128)/32)*4 + b%4. Rows are padded to a multiple
  *          of 128; a block with no real element (and every padding row)
  *          holds 0.
- *   hp     [R][kp] BF16    the outlier channels O_0..O_{k-1}, zero padded.
+ *          NVFP4 plans (osm_plan_set_format) store one UE4M3 scale per
+ *          16-block b = p/16 in the same atom layout with four 16-blocks
+ *          per atom row: Kbp/64 atoms per 128 rows, Kbp/16 bytes per row.
+ *   hp     [R][kp] BF16    the outlier channels O_0..O_{k-1}, zero padded
+ *          (binary16 for an FP16 outlier branch; NVFP4 plans store them
+ *          times 2^-g, see osm_plan_set_format).
  */
 #ifndef OSM_H
 #define OSM_H
@@ -311,6 +316,8 @@ OSM_API int osm_error_norms(const float* Y, const float* Yref, int64_t count, do
  *   bulk x'[J_p] -> MXFP4 with the exponent floor(log2 amax_b) - 2 of each
  *   32-block (clamped to [-127,127]; amax 0 -> -127), elements E2M1 RNE,
  *   saturating at 6; the sign bit is the sign of x'.
+ * (NVFP4 plans: 16-blocks with UE4M3 scales and 2^-g_act outlier slots, as
+ * osm_plan_set_format defines.)
  * Writes a_codes [M][Kbp/2], a_scales (rows padded to 128), a_hp [M][kp].
  * Rows stream through shared memory by asynchronous bulk copies; a copy
  * that does not arrive within the plan's wait limit sets OSM_STATUS_TIMEOUT
@@ -323,6 +330,8 @@ OSM_API int osm_quantize_act(const osm_plan* plan, const uint16_t* X, int64_t M,
  *   acc[t][n] = sum_b 2^(Xa(t,b)+Xw(n,b)) sum_{p in b} e2m1(a_tp) e2m1(w_np)
  *             + sum_{i<kp} a_hp[t][i] w_hp[n][i]             (FP32 accumulate)
  *   y = acc (+ bias[n] if bias != NULL).
+ * NVFP4 plans: kind::mxf4nvf4 MMAs with the 16-block UE4M3 scales, and
+ *   y = 2^(g_act + g_w) acc (+ bias[n]).
  * Both branches accumulate into one tensor-memory accumulator on tcgen05
  * (block-scaled MXFP4 MMA, then BF16 MMA) before a single epilogue.
  * Operands come from osm_quantize_act / osm_pack_weights with the same
