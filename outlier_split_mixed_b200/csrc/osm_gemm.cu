@@ -1,10 +1,10 @@
 // Dual-branch W4A4 GEMM for sm_100a: Eq. (5) of "W4A4 Quantization for
 // Inference on Wan2.2-I2V-A14B" with Eq. (3)'s group scales taken per
-// 32-element block (OCP MXFP4).
+// 32-element block (OCP MXFP4), or per 16-element block (NVFP4).
 //
 //   acc = sum over bulk K-steps of tcgen05.mma kind::mxf4 (block-scaled,
-//         E8M0 scales in tensor memory)
-//       + sum over outlier K-steps of tcgen05.mma kind::f16 (BF16 x BF16)
+//         E8M0 scales in tensor memory) or kind::mxf4nvf4 (UE4M3 scales)
+//       + sum over outlier K-steps of tcgen05.mma kind::f16 (BF16 or FP16)
 //
 // Both branches accumulate into the same FP32 tensor-memory accumulator
 // before one epilogue.
@@ -16,21 +16,22 @@
 // 128 x 256 share of the output.
 //
 // Roles in each CTA (warp-specialised):
-//   warp 0     TMA producer: 128B-swizzled tiles of its A rows and B rows,
+//   warps 0-7  epilogue: each warp drains 32 lanes x 128 columns of its
+//              CTA's accumulator into registers (two per TMEM lane
+//              quadrant), hands tensor memory back (arrivals counted in the
+//              leader), then converts and stores straight from registers
+//              in full 32-byte sectors while the next tile's MMAs run.
+//   warp 8     TMA producer: 128B-swizzled tiles of its A rows and B rows,
 //              and the scale atoms (its 128 A rows; all 256 B rows), into
-//              a 6-deep shared-memory ring. All copies of both CTAs
-//              complete on the LEADER CTA's ring barrier.
-//   warp 1     tensor-memory allocation for the pair; in the leader CTA the
-//              single MMA-issuing thread: tcgen05.cp of the scale atoms
-//              into tensor memory (both CTAs), the MMAs, and a multicast
-//              tcgen05.commit that frees the ring slot in both CTAs.
-//   warps 2-9  epilogue: each warp drains 32 lanes x 128 columns of its
-//              CTA's accumulator half into registers (16x256b loads: four
-//              lanes per row), hands tensor memory back (arrivals counted in
-//              the leader), then adds the bias and stores FP32 or BF16
-//              straight from registers in full 32-byte sectors while the
-//              next tile's MMAs run. Keeping shared memory for the operand
-//              ring (6 stages) matters more than store coalescing here.
+//              a shared-memory ring (6 slots for MXFP4, 5 for NVFP4). All
+//              copies of both CTAs complete on the LEADER CTA's ring
+//              barrier.
+//   warp 9     in the leader CTA the single MMA-issuing thread: tcgen05.cp
+//              of the scale atoms into tensor memory (both CTAs), the MMAs,
+//              and multicast tcgen05.commits that free the ring slot and
+//              publish the finished accumulator in both CTAs.
+//   warp 1     allocates and frees the pair's tensor memory; warps 10-11
+//              only complete the control warpgroup.
 // Every wait is bounded by %globaltimer; a wait that runs out sets the
 // plan's status word and raises a CTA-wide abort flag; the CTA then lets
 // its in-flight copies and MMAs finish, frees tensor memory and returns.
