@@ -489,10 +489,11 @@ __host__ __device__ constexpr int qa_row_stride(int nb, int kp) { return (nb * Q
 //           outlier slot); consecutive lanes write into one 128-byte window,
 //           so the stores are conflict-free (eight channels per lane would
 //           put a warp's stores 16 bytes apart: a 4-way bank conflict);
-//  phase 2: one thread per (row, 32-block): four 128-bit shared loads,
-//           amax by packed u16 max, E8M0 exponent, sixteen E2M1x2
-//           conversions, one 128-bit code store and one scale byte;
-//  phase 3: the outlier slots go out as 128-bit stores.
+//  phases 2 and 3 (encode_staged): one thread per (row, 32-block) encodes
+//           the block (MXFP4, or two NVFP4 16-blocks) from four 128-bit
+//           shared loads; the outlier slots go out as 128-bit stores.
+// This staged, phase-serial form serves rows too wide for the streaming
+// form's ring (quantize_act_stream_kernel below).
 template <int MODE>
 __device__ __forceinline__ void encode_staged(const QuantParams& p, uint32_t sbuf, int stride, int row0, int nrows);
 __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p);
