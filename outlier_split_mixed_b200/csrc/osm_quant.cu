@@ -652,8 +652,11 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 //  are encoded (encode_staged).
 // Every wait on a slot is bounded; a wait that runs out sets
 // OSM_STATUS_TIMEOUT, and the CTA lets its copies land before it returns.
+// Two CTAs per SM, except with more than six register-held pairs per
+// thread (one CTA per SM then has the registers and the shared memory for
+// a deeper ring).
 template <int R, int S, int NT, int TR, int MODE>
-__global__ void __launch_bounds__(NT, 2) quantize_act_stream_kernel(QuantParams p) {
+__global__ void __launch_bounds__(NT, (TR > 6 ? 1 : 2)) quantize_act_stream_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
     ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
     extern __shared__ __align__(128) uint8_t smem[];
@@ -918,6 +921,12 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
         return launch_stream<2, 3, STREAM_NT, 0>(p, mode, stride, st);
     }
     if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3, STREAM_NT, 0>(p, mode, stride, st);
+    // rows whose ring would get only two slots at two CTAs per SM (e.g. K =
+    // 13824): one CTA per SM with five slots, each thread's (up to 14)
+    // channel pairs and routes held in registers
+    const size_t one_per_sm = 220 * 1024;
+    if (npairs <= 14 * STREAM_NT && stream_smem_bytes<1, 5>(p.K, stride) <= one_per_sm)
+        return launch_stream<1, 5, STREAM_NT, 14>(p, mode, stride, st);
     if (stream_smem_bytes<1, 2>(p.K, stride) <= two_per_sm) return launch_stream<1, 2, STREAM_NT, 0>(p, mode, stride, st);
     // very wide rows: the staged, phase-serial form
     const size_t row_bytes = static_cast<size_t>(stride);
