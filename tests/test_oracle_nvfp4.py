@@ -262,3 +262,31 @@ def test_library_host_exponents_equal_the_oracle():
         amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
         s, inv_s, O = oracle.calibrate(amax, wmax, 0.6, k)
         assert osm.nvfp4_plan_exponents(amax, wmax, s, inv_s, O) == oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+
+
+def _golden_lines(name):
+    from conftest import golden_path
+    with open(golden_path(name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                yield line
+
+
+def test_e4m3_encode_hand_table():
+    for line in _golden_lines("e4m3_rounding.txt"):
+        v, code = line.split()
+        assert oracle.e4m3_encode(float(v)) == int(code, 16), line
+
+
+def test_nvfp4_blocks_hand_derived():
+    for line in _golden_lines("nvfp4_blocks.txt"):
+        g, vals, sc, codes = (x.strip() for x in line.split("|"))
+        v = np.array([float(x) for x in vals.split()], np.float32)
+        X = np.zeros((1, 32), np.uint16)
+        X[0, :16] = synth.to_bf16_bits(v)
+        # every value but 0.1 is a BF16 number; bf16(0.1) = 0.10009766 still codes to 0
+        c, s, _ = oracle.quantize_act_nv(X, np.ones(32, np.float32), np.zeros(0, np.int32), int(g))
+        assert s[0, 0] == int(sc, 16), line
+        assert c[0, :8].tolist() == [int(x, 16) for x in codes.split()], line
+        assert s[0, 1] == 0 and not c[0, 8:].any()                         # the all-zero second block
