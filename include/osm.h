@@ -287,7 +287,10 @@ OSM_API int osm_pack_weights_for_next(const osm_plan* plan, const osm_plan* next
  * again (osm_pack_weights): s is folded into them and J has changed; data
  * packed for the old plan must not be used with the new one. A non-finite
  * statistic sets OSM_STATUS_NONFINITE and leaves the plan unchanged.
- * alpha in (0, 1). */
+ * alpha in (0, 1). The format and an NVFP4 plan's exponents g_act, g_w are
+ * kept as set (they are host-side settings); a caller that wants them to
+ * follow the new s sets them again with osm_plan_set_format before
+ * packing. */
 OSM_API int osm_plan_refresh(osm_plan* plan, const float* amax, const float* wmax, float alpha, void* stream);
 
 /* As osm_plan_refresh, with the top-k taken by a separate device score
