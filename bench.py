@@ -314,9 +314,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     s, inv_s, O = odist.calibrate_from_local_stats(amax, wmax, cfg.alpha, cfg.k)
     plan = osm.Plan(K, N, cfg.k, s, O, osm.WSCALE_1x32 if args.nvfp4 else cfg.wmode, hp_fp16=args.hp_fp16)
     if args.nvfp4:
-        amax_all = odist.allreduce_max_(amax.clone())
-        plan.set_format(osm.FMT_NVFP4, *osm.nvfp4_plan_exponents(amax_all.cpu().numpy(), wmax.cpu().numpy(), s,
-                                                                 inv_s, O))
+        plan.set_format(osm.FMT_NVFP4, *odist.nvfp4_exponents_from_local_stats(amax, wmax, s, inv_s, O))
     wc, wsc, wh = plan.alloc_packed(N, dev)
     osm.pack_weights(plan, Wd, wc, wsc, wh)
     ac, asc, ah = plan.alloc_packed(M, dev)

@@ -41,3 +41,14 @@ def calibrate_from_local_stats(amax_local, wmax, alpha: float, k: int, group=Non
     return osm.calibrate_finalize(amax.cpu().numpy().astype(np.float32),
                                   np.asarray(wmax.cpu().numpy() if hasattr(wmax, "cpu") else wmax, np.float32),
                                   alpha, k)
+
+
+def nvfp4_exponents_from_local_stats(amax_local, wmax, s, inv_s, O, group=None):
+    """The NVFP4 per-tensor exponents (g_act, g_w) of a plan from per-rank
+    activation maxima combined across ranks (all-reduce MAX), so that every
+    rank encodes with the same factors (osm_nvfp4_plan_exponents)."""
+    import outlier_split_mixed_b200 as osm
+    amax = allreduce_max_(amax_local.clone(), group)
+    return osm.nvfp4_plan_exponents(amax.cpu().numpy().astype(np.float32),
+                                    np.asarray(wmax.cpu().numpy() if hasattr(wmax, "cpu") else wmax, np.float32),
+                                    s, inv_s, O)

@@ -2,7 +2,8 @@
 calibration all-reduce. Each rank computes the activation maxima of its own
 token shard (oracle, CPU), the ranks combine them with an all-reduce (MAX),
 and the library's host-side Eq. (2)/(4) finalisation must then reproduce,
-bit for bit, the calibration of the whole batch on one process."""
+bit for bit, the calibration of the whole batch on one process (and the
+same NVFP4 per-tensor exponents)."""
 import os
 import socket
 
@@ -48,7 +49,8 @@ def _worker(rank, world, port, out_q):
         amax_local = torch.from_numpy(oracle.act_amax(X[lo:hi]) if hi > lo else np.zeros(256, np.float32))
         wmax = oracle.weight_amax(W)
         s, inv_s, O = odist2.calibrate_from_local_stats(amax_local, wmax, 0.6, 24)
-        out_q.put((rank, s.view(np.uint32).tolist(), O.tolist()))
+        g = odist2.nvfp4_exponents_from_local_stats(amax_local, wmax, s, inv_s, O)
+        out_q.put((rank, s.view(np.uint32).tolist(), O.tolist(), g))
     finally:
         dist.destroy_process_group()
 
@@ -68,7 +70,10 @@ def test_two_rank_calibration_matches_single_process():
         assert p.exitcode == 0
     X = synth.acts_heavy_tailed(520, 256, seed=90, frac=0.03)
     W = synth.weights_gaussian(256, 64, seed=91, sigma=0.05)
-    s, _, O = oracle.calibrate(oracle.act_amax(X), oracle.weight_amax(W), 0.6, 24)
-    for rank, s_bits, O_r in results:
+    amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
+    s, inv_s, O = oracle.calibrate(amax, wmax, 0.6, 24)
+    g = oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+    for rank, s_bits, O_r, g_r in results:
         assert s_bits == s.view(np.uint32).tolist(), rank
         assert O_r == O.tolist(), rank
+        assert tuple(g_r) == tuple(g), rank     # NVFP4 exponents of the whole batch on every rank
