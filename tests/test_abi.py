@@ -108,3 +108,20 @@ def test_argument_errors_need_no_gpu():
     assert rc == osm.ERR_INVALID_ARG   # s must be positive
     assert L.osm_dual_gemm(None, *([None] * 3), 1, *([None] * 4), 0, None, None, None, None, None, None) \
         == osm.ERR_INVALID_ARG
+
+
+def test_nvfp4_host_helpers_reject_bad_statistics():
+    for bad in (-1.0, float("nan"), float("inf")):
+        with pytest.raises(osm.OsmError) as e:
+            osm.nvfp4_tensor_exponent(bad)
+        assert e.value.code == osm.ERR_INVALID_ARG
+    ones = np.ones(64, np.float32)
+    with pytest.raises(osm.OsmError):
+        osm.nvfp4_plan_exponents(ones, ones, ones, ones, np.array([64], np.int32))      # O out of range
+    nan_stats = ones.copy()
+    nan_stats[5] = np.nan
+    with pytest.raises(osm.OsmError):
+        osm.nvfp4_plan_exponents(nan_stats, ones, ones, ones, np.zeros(0, np.int32))
+    # a NaN on an outlier channel does not enter the bulk maxima
+    assert osm.nvfp4_plan_exponents(nan_stats, ones, ones, ones, np.array([5], np.int32)) == (
+        osm.nvfp4_tensor_exponent(1.0), osm.nvfp4_tensor_exponent(1.0))
