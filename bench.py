@@ -1,24 +1,29 @@
 """Benchmark of the smoothed, outlier-split W4A4 linear layer on B200.
 
-One step = one pass of the hot path over one batch of synthetic tokens:
-quantize_act (smooth, split, MXFP4-encode) followed by dual_gemm (block-
-scaled MXFP4 tcgen05 MMAs + BF16 outlier MMAs into one TMEM accumulator),
-with inputs resident in HBM. Default workload: the Wan-like FFN
-up-projection, 4096 tokens x 5120 -> 13824, alpha 0.6, k = 128 outliers,
-128x1 weight stripes, FP32 output.
+One step = one pass of the hot path over one batch of synthetic tokens,
+with inputs resident in HBM. Default workload (the largest single-GPU
+configuration): four Wan-like FFN blocks of 32760 tokens, each
+quantize_act (smooth, split, MXFP4-encode), the up-projection 5120 -> 13824
+(block-scaled MXFP4 tcgen05 MMAs + BF16 outlier MMAs into one TMEM
+accumulator) with GELU, the down-projection's smoothing and its MXFP4
+requantisation fused into the epilogue, then the down-projection
+13824 -> 5120 to BF16 -- one osm_ffn_block call per block.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload up|down|long|tiny|ffn]
+                  [--workload ffn|up|down|long|tiny|refresh|search|errk]
 
-`--workload ffn` runs four FFN blocks of 32760 tokens (up 5120 -> 13824
-with GELU, smoothing and requantisation fused into its epilogue, then down
-13824 -> 5120 to BF16); one step is all four blocks.
+The single-layer workloads (`up` 4096 x 5120 -> 13824, `down` 32760 x
+13824 -> 5120, `long` 75600 x 5120 -> 13824, `tiny`) time quantize_act +
+dual_gemm of one layer; `errk` reports the layer's relative error against
+the unquantised product for k in {0, 16, 64, 128, 256}.
 
-Multi-GPU (torchrun, one rank per GPU): tokens are data-parallel, each rank
-runs its own batch with no collective on the data path (weak scaling); the
-step time is the max over ranks. `--impl reference` times the CPU oracle
-(the only reference implementation of this method) on a bounded sample of
-the same workload, on rank 0 only.
+Multi-GPU: `--gpus N` without a torchrun environment starts N ranks itself
+(torch.distributed.run, one rank per GPU, NCCL); tokens are data-parallel,
+each rank runs its own batch with no collective on the data path (weak
+scaling; calibration statistics are all-reduced with MAX), and the step
+time is the max over ranks. `--impl reference` times the CPU oracle (the
+only reference implementation of this method) on a bounded sample of the
+same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -265,7 +270,7 @@ def oracle_ffn_throughput(cfg, rows_per_step: int, steps: int, warmup: int, cali
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return 0
-    is_ffn = cfg.name == workloads()["ffn"].name
+    is_ffn = hasattr(cfg, "layers")
     rows = max(1, args.ref_rows if not is_ffn else max(1, args.ref_rows // 8))
     if is_ffn:
         tflops, t, cores = oracle_ffn_throughput(cfg, rows, args.steps, args.warmup)
@@ -437,8 +442,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                          "traffic": None if args.hp_fp16 else DUAL_GEMM_TRAFFIC.get((cfg.name,
                                                                                     fmt_config(args, cfg)["format"])),
                          "traffic_unit": "bytes per launch", "kernel": "dual_gemm",
-                         "peak_source": f"{peak_src}: bf16 burst {p16} x4 for the FP4 share, x1 for the "
-                                        f"BF16 share (k={plan.k} of K={K})"},
+                         "pct_fp4_spec_peak": 100.0 * achieved / FP4_SPEC_TFLOPS,
+                         "peak_source": f"derived from {peak_src} peaks: BF16 burst {p16} TFLOP/s x4 (nominal "
+                                        f"FP4:BF16 dense ratio) for the FP4 share, x1 for the BF16 share "
+                                        f"(k={plan.k} of K={K}); FP4 itself is not measured"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * Y.element_size(),
                     "api": f"osm_linear_host, steps rotated over {E2E_STREAMS} streams"},
@@ -456,10 +463,10 @@ def run_ours(args, cfg, rank, world, local_rank):
 
 
 def run_ffn(args, cfg, rank, world, local_rank):
-    """Four FFN blocks on one stream. Per block and step: quantize_act of the
-    block input for the up-projection; dual_gemm up with the fused GELU +
-    smoothing + MXFP4 requantisation epilogue, writing the down-projection's
-    packed activations; dual_gemm down to BF16."""
+    """Four FFN blocks on one stream, each one call of osm_ffn_block:
+    quantize_act of the block input for the up-projection; dual_gemm up with
+    the fused GELU + smoothing + MXFP4 requantisation epilogue, writing the
+    down-projection's packed activations; dual_gemm down to BF16."""
     import torch
     import torch.distributed as dist
 
@@ -506,27 +513,30 @@ def run_ffn(args, cfg, rank, world, local_rank):
         osm.pack_weights(down, Wd, *wd)
         del Wu, Wd, Xc
         blocks.append(dict(up=up, down=down, wu=wu, wd=wd, X=cfg.make_x(l)))
-    # activation buffers shared by the blocks; each block has its own input and output
-    a_up = blocks[0]["up"].alloc_packed(M, dev)
-    a_dn = blocks[0]["down"].alloc_packed(M, dev)
+    # the device workspace (both layers' packed activations) is shared by the
+    # blocks, which run one after another; each block has its own input and output
+    ws = torch.empty(max(osm.ffn_workspace_size(b["up"], b["down"], M) for b in blocks), dtype=torch.uint8,
+                     device=dev)
     for b in blocks:
         b["Xd"] = to_dev(b["X"])
         b["Y"] = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    # the same buffers split per kernel, for the pass with events between kernels
+    a_up = blocks[0]["up"].alloc_packed(M, dev)
+    a_dn = blocks[0]["down"].alloc_packed(M, dev)
     flush = L2Flush(dev)
 
-    def block(b, ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def block(b):
+        osm.ffn_block(b["up"], b["down"], b["Xd"], b["wu"], b["wd"], b["Y"], ws)
+
+    def block_split(b, ev):
+        ev[0].record(stream)
         osm.quantize_act(b["up"], b["Xd"], *a_up)
-        if ev is not None:
-            ev[1].record(stream)
+        ev[1].record(stream)
         osm.dual_gemm(b["up"], *a_up, M, *b["wu"], None, epi=osm.EPI_GELU_REQUANT, next_plan=b["down"],
                       next_buffers=a_dn)
-        if ev is not None:
-            ev[2].record(stream)
+        ev[2].record(stream)
         osm.dual_gemm(b["down"], *a_dn, M, *b["wd"], b["Y"], epi=osm.EPI_BF16)
-        if ev is not None:
-            ev[3].record(stream)
+        ev[3].record(stream)
 
     for _ in range(args.warmup):
         flush(1.0)
@@ -534,10 +544,10 @@ def run_ffn(args, cfg, rank, world, local_rank):
             block(b)
     torch.cuda.synchronize()
 
-    # The timed region: K steps with events at the step boundaries only (events
-    # between kernels would stop each dual_gemm's dependent launch); the
-    # kernel split comes from the same K steps run again with events between
-    # the kernels.
+    # The timed region: K steps of the four blocks with events at the step
+    # boundaries only (events between kernels would stop each dual_gemm's
+    # dependent launch); the kernel split comes from the same K steps run
+    # again with events between the kernels.
     n = args.steps
     L = cfg.layers
     evt = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
@@ -556,7 +566,7 @@ def run_ffn(args, cfg, rank, world, local_rank):
         for i in range(n):
             flush(float(i))
             for l, b in enumerate(blocks):
-                block(b, ev[i][l])
+                block_split(b, ev[i][l])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -572,37 +582,19 @@ def run_ffn(args, cfg, rank, world, local_rank):
         dist.all_reduce(loc, op=dist.ReduceOp.MAX)
     step_s, quant_s, up_s, down_s = (float(x) for x in loc.cpu())
 
-    # end to end through the public API: every block input copied in from
-    # pinned host memory and every block output copied out, inside the region
+    # End to end through the host entry point osm_ffn_block_host: every block
+    # input copied in from pinned host memory and every block output copied
+    # out, inside the timed region. Each block runs on its own stream with its
+    # own device workspace, so one block's copies overlap another's kernels.
     Xh = [torch.from_numpy(b["X"].view(np.int16)).view(torch.bfloat16).pin_memory() for b in blocks]
     Yh = [torch.empty((M, D), dtype=torch.bfloat16).pin_memory() for _ in blocks]
-
-    # Three streams: copies in, the blocks' kernels, copies out. Block l's
-    # input copy waits until the previous step's kernels of block l are done
-    # with its device buffers, its kernels wait for its input, and its output
-    # copy for its kernels, so copies of one block overlap another's compute.
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    in_done = [torch.cuda.Event() for _ in blocks]
-    comp_done = [torch.cuda.Event() for _ in blocks]
-    out_done = [torch.cuda.Event() for _ in blocks]
-    for l in range(len(blocks)):
-        comp_done[l].record(stream)
-        out_done[l].record(stream)
+    streams = [torch.cuda.Stream(device=dev) for _ in blocks]
+    wss = [torch.empty(osm.ffn_host_workspace_size(b["up"], b["down"], M), dtype=torch.uint8, device=dev)
+           for b in blocks]
 
     def e2e_step():
-        for l, (b, xh, yh) in enumerate(zip(blocks, Xh, Yh)):
-            s_in.wait_event(comp_done[l])
-            with torch.cuda.stream(s_in):
-                b["Xd"].copy_(xh, non_blocking=True)
-            in_done[l].record(s_in)
-            stream.wait_event(in_done[l])
-            stream.wait_event(out_done[l])
-            block(b)
-            comp_done[l].record(stream)
-            s_out.wait_event(comp_done[l])
-            with torch.cuda.stream(s_out):
-                yh.copy_(b["Y"], non_blocking=True)
-            out_done[l].record(s_out)
+        for b, xh, yh, st, w in zip(blocks, Xh, Yh, streams, wss):
+            osm.ffn_block_host(b["up"], b["down"], xh, b["wu"], b["wd"], yh, w, stream=st)
 
     e2e_steps = max(3, min(10, n))
     e2e_step()
@@ -611,18 +603,22 @@ def run_ffn(args, cfg, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
+    for st in streams:
+        st.wait_event(e0)
     for _ in range(e2e_steps):
         e2e_step()
-    stream.wait_stream(s_in)
-    stream.wait_stream(s_out)
+    for st in streams:
+        stream.wait_stream(st)
     e1.record(stream)
     torch.cuda.synchronize()
+    for b in blocks:
+        if b["up"].status() != 0 or b["down"].status() != 0:
+            raise RuntimeError("device status reports a timeout during the end-to-end region")
     e2e_t = torch.tensor([e0.elapsed_time(e1) * 1e-3 / e2e_steps], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
     e2e_s = float(e2e_t.item())
+    del wss
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -631,13 +627,14 @@ def run_ffn(args, cfg, rank, world, local_rank):
         up0, dn0 = blocks[0]["up"], blocks[0]["down"]
         f_up = L * 2.0 * M * F * D
         f_dn = L * 2.0 * M * D * F
-        parts = [(L * 2.0 * M * F * b["up"].Kb, L * 2.0 * M * F * b["up"].k) for b in blocks[:1]] + \
-                [(L * 2.0 * M * D * b["down"].Kb, L * 2.0 * M * D * b["down"].k) for b in blocks[:1]]
-        peak_blend, p16 = blended_peak(peaks, parts)
-        gemm_s = up_s + down_s
-        achieved = (f_up + f_dn) / gemm_s / 1e12
+        # the dominant kernel: the up-projection with the fused epilogue
+        peak_up, p16 = blended_peak(peaks, [(2.0 * M * F * up0.Kb, 2.0 * M * F * up0.k)])
+        peak_dn, _ = blended_peak(peaks, [(2.0 * M * D * dn0.Kb, 2.0 * M * D * dn0.k)])
+        ach_up = f_up / up_s / 1e12
+        ach_dn = f_dn / down_s / 1e12
         cb, sb, hb = up0.sizes(M)
         q_bytes = L * (M * D * 2 + cb + sb + hb)
+        traffic = None if args.hp_fp16 else DUAL_GEMM_TRAFFIC.get((cfg.name, "up_gelu_requant"))
         line = {
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
@@ -645,26 +642,35 @@ def run_ffn(args, cfg, rank, world, local_rank):
             "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate", "data": "synthetic",
             "config": dict(workload_config(cfg), l2=L2_NOTE,
                            parallelism=f"dp{world} (token shards, no data-path collective)",
-                           outlier_branch="fp16" if args.hp_fp16 else "bf16"),
+                           outlier_branch="fp16" if args.hp_fp16 else "bf16",
+                           step="osm_ffn_block per block (quantize_act, up with fused GELU requant, down to BF16)"),
             "pct_fp4_spec_peak": 100.0 * value / world / FP4_SPEC_TFLOPS,
             "kernels": {
-                "dual_gemm_up_gelu_requant": {"ms": up_s * 1e3, "tflops": f_up / up_s / 1e12},
-                "dual_gemm_down_bf16": {"ms": down_s * 1e3, "tflops": f_dn / down_s / 1e12},
+                "dual_gemm_up_gelu_requant": {"ms": up_s * 1e3, "tflops": ach_up, "frac": ach_up / peak_up,
+                                              "pct_fp4_spec_peak": 100.0 * ach_up / FP4_SPEC_TFLOPS},
+                "dual_gemm_down_bf16": {"ms": down_s * 1e3, "tflops": ach_dn, "frac": ach_dn / peak_dn,
+                                        "pct_fp4_spec_peak": 100.0 * ach_dn / FP4_SPEC_TFLOPS,
+                                        "traffic": None if args.hp_fp16 else
+                                        DUAL_GEMM_TRAFFIC.get((cfg.name, "down_bf16"))},
                 "quantize_act": {"ms": quant_s * 1e3, "gbs": q_bytes / quant_s / 1e9, "bytes": q_bytes,
                                  "frac_hbm": q_bytes / quant_s / 1e9 / peaks["hbm_gbs"]},
             },
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
-                         "frac": achieved / peak_blend, "traffic": None, "kernel": "dual_gemm (up + down)",
-                         "peak_source": f"{peak_src}: bf16 burst {p16} x4 for the FP4 share, x1 for the BF16 "
-                                        f"share (k_up={up0.k}, k_down={dn0.k})"},
+            "roofline": {"bound": "tensor", "achieved": ach_up, "peak": peak_up, "unit": "TFLOP/s",
+                         "frac": ach_up / peak_up, "traffic": traffic, "traffic_unit": "bytes per launch",
+                         "kernel": "dual_gemm up-projection, fused GELU + smoothing + MXFP4 requantisation",
+                         "pct_fp4_spec_peak": 100.0 * ach_up / FP4_SPEC_TFLOPS,
+                         "peak_source": f"derived from {peak_src} peaks: BF16 burst {p16} TFLOP/s x4 (nominal "
+                                        f"FP4:BF16 dense ratio) for the FP4 share, x1 for the BF16 share "
+                                        f"(k={up0.k} of K={D}); FP4 itself is not measured"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": L * M * D * 2, "d2h_bytes_per_step": L * M * D * 2,
-                    "api": "quantize_act + dual_gemm (Python binding); pinned host copies on their own in / out streams, overlapping other blocks' kernels"},
+                    "copies_declared": True,
+                    "api": "osm_ffn_block_host per block (pinned X in, Y out); each block on its own stream"},
             "gpu_launches": 3 * L * n,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            rows = max(1, args.cpu_rows // 16)
+            rows = max(1, args.cpu_rows // 4)
             tf, t1, cores = oracle_ffn_throughput(cfg, rows, 2, 1)
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                     "sample": f"{rows} of {M} tokens per block per step (2 steps), calibration "
@@ -792,13 +798,69 @@ def run_search(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_errk(args, cfg, rank, world, local_rank):
+    """The paper's Eq. (5) argument measured on the CUDA path: relative
+    Frobenius error of the layer output against the unquantised product of
+    the same BF16 operands (PyTorch FP32 matmul) for k in {0, 16, 64, 128,
+    256} outlier channels, on the layer workload's synthetic batch."""
+    import torch
+    import outlier_split_mixed_b200 as osm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    X, W = cfg.make_x(), cfg.make_w()
+    Xd = torch.from_numpy(X.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+    ref = Xd.float() @ Wd.float()
+    table = []
+    for k in (0, 16, 64, 128, 256):
+        s, _, O, _, _ = osm.calibrate([Xd], Wd, cfg.alpha, k)
+        plan = osm.Plan(cfg.K, cfg.N, k, s, O, cfg.wmode)
+        wc, wsc, wh = plan.alloc_packed(cfg.N, dev)
+        osm.pack_weights(plan, Wd, wc, wsc, wh)
+        ac, asc, ah = plan.alloc_packed(cfg.M, dev)
+        osm.quantize_act(plan, Xd, ac, asc, ah)
+        Y = torch.empty((cfg.M, cfg.N), dtype=torch.float32, device=dev)
+        osm.dual_gemm(plan, ac, asc, ah, cfg.M, wc, wsc, wh, Y)
+        e, nrm = osm.error_norms(Y, ref)
+        if plan.status() != 0:
+            raise RuntimeError("plan status reports an error")
+        plan.close()
+        table.append({"k": k, "rel_err": float(np.sqrt(e / nrm))})
+    if rank == 0:
+        rel = [r["rel_err"] for r in table]
+        line = {
+            "metric": "relative Frobenius error of Y against the unquantised FP32 XW, by outlier count k",
+            "value": rel[-1], "unit": "relative error at k=256", "n_gpus": 1, "steps": len(table), "warmup": 0,
+            "higher_is_better": False, "vs_baseline": None, "dtype": "mxfp4(e2m1,e8m0)+bf16, fp32 accumulate",
+            "data": "synthetic", "config": dict(workload_config(cfg), wscale=WSCALE_NAMES[cfg.wmode]),
+            "error_vs_k": table,
+            "falls_monotonically": all(b <= a for a, b in zip(rel, rel[1:])),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def relaunch_ranks(n: int) -> int:
+    """Start n ranks of this same command under torch.distributed.run (one
+    process per GPU, rendezvous on 127.0.0.1) and return its exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["up", "down", "long", "tiny", "ffn", "refresh", "search"], default="up")
+    ap.add_argument("--workload", choices=["ffn", "up", "down", "long", "tiny", "refresh", "search", "errk"],
+                    default="ffn")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -816,10 +878,16 @@ def main():
     if args.nvfp4 and (args.workload in ("ffn", "refresh", "search") or args.hp_fp16):
         ap.error("--nvfp4 applies to the layer workloads (up, down, long, tiny) with the BF16 outlier branch")
 
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch_ranks(args.gpus)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = workloads()[args.workload if args.workload not in ("refresh", "search") else "up"]
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {world} ranks")
+    cfg = workloads()[args.workload if args.workload not in ("refresh", "search", "errk") else "up"]
     if args.tokens or args.blocks:
         import dataclasses
         changes = {}
@@ -847,6 +915,8 @@ def main():
             return run_refresh(args, cfg, rank, world, local_rank)
         if args.workload == "search":
             return run_search(args, cfg, rank, world, local_rank)
+        if args.workload == "errk":
+            return run_errk(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:

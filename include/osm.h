@@ -92,13 +92,14 @@ typedef enum {
     OSM_WSCALE_STRIP128x1 = 2
 } osm_wscale_mode;
 
-/* Epilogues of osm_dual_gemm. GELU below is the tanh form in FP32,
- * 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated exactly as
- * this library specifies it, with only IEEE round-to-nearest-even adds,
+/* Epilogues of osm_dual_gemm. GELU below is the FFN's tanh form,
+ * 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated by this
+ * library's own FP32 routine (only IEEE round-to-nearest-even adds,
  * multiplies and fused multiply-adds: 0.5 (1 + tanh(u)) = sigma(2u) is
- * 1/(1 + E) for x >= 0 and E/(1 + E) for x < 0, E = exp(-2|u|) (Cody-Waite
- * reduction, degree-7 Taylor polynomial, 0 below 2^-126), the reciprocal
- * by a linear seed and three Newton steps. */
+ * 1/(1 + E) for x >= 0 and E/(1 + E) for x < 0, E = exp(-2|u|) by
+ * Cody-Waite reduction and a degree-7 Taylor polynomial, the reciprocal by
+ * a linear seed and three Newton steps). It stays within 5e-7 |GELU(x)| +
+ * 2e-8 |x| of the exact function; a BF16 result adds one rounding. */
 typedef enum {
     OSM_EPI_F32 = 0,          /* Y [M][N] float32                                     */
     OSM_EPI_BF16 = 1,         /* Y [M][N] BF16 (RNE of the FP32 accumulator)          */
@@ -313,7 +314,7 @@ OSM_API int osm_error_norms(const float* Y, const float* Yref, int64_t count, do
 /* ---- runtime activation path ----------------------------------------------
  * "activations are divided in-place by s, quantized ..., and routed through
  * either the W4A4 bulk path or a narrow FP16 outlier path" (implementation
- * paragraph). X [M][K] BF16 row-major, M >= 1. For each row:
+ * paragraph). X [M][K] BF16 row-major, 1 <= M < 2^31. For each row:
  *   x' = bf16(fp32(x_j) * inv_s_j);
  *   a_hp[t][i] = x'[O_i];
  *   bulk x'[J_p] -> MXFP4 with the exponent floor(log2 amax_b) - 2 of each
@@ -338,7 +339,7 @@ OSM_API int osm_quantize_act(const osm_plan* plan, const uint16_t* X, int64_t M,
  * Both branches accumulate into one tensor-memory accumulator on tcgen05
  * (block-scaled MXFP4 MMA, then BF16 MMA) before a single epilogue.
  * Operands come from osm_quantize_act / osm_pack_weights with the same
- * plan. M >= 1.
+ * plan. 1 <= M < 2^31.
  *   epi = OSM_EPI_F32:       Y is float [M][N].
  *   epi = OSM_EPI_BF16:      Y is BF16  [M][N].
  *   epi = OSM_EPI_GELU_BF16: Y is BF16  [M][N] = bf16(GELU(acc + bias)).
@@ -371,11 +372,51 @@ OSM_API int osm_linear_host(const osm_plan* plan, const uint16_t* X_host, int64_
                     const uint8_t* w_scales, const uint16_t* w_hp, const float* bias, int epi,
                     void* Y_host, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- one FFN block (up-projection, GELU, down-projection) -----------------
+ * The FFN of a transformer block as the implementation paragraph deploys it:
+ * every FFN linear map runs the smoothed, outlier-split W4A4 path, and the
+ * hidden activations are "divided in-place by s, quantized ..., and routed"
+ * before the down-projection. One call enqueues
+ *   osm_quantize_act(up, X)                      -> up's packed activations,
+ *   osm_dual_gemm(up, OSM_EPI_GELU_REQUANT, down) -> down's packed activations
+ *                                                   (GELU, smoothing by down's
+ *                                                   s, MXFP4 encoding fused),
+ *   osm_dual_gemm(down, OSM_EPI_BF16)            -> Y [M][down->N] BF16
+ *                                                   (+ bias_down[n] if given).
+ * up->N must equal down->K; both plans MXFP4. Weights: wu_* packed by
+ * osm_pack_weights_for_next(up, down, W_up), wd_* by osm_pack_weights(down,
+ * W_down). X [M][up->K] BF16 and Y are device pointers; workspace is
+ * caller-owned device memory of at least osm_ffn_workspace_size(up, down, M)
+ * bytes (both layers' packed activations; contents need no clearing). The
+ * result is bit-identical to issuing the three calls on separate buffers.
+ * 1 <= M < 2^31. Returns the first failing call's error; a failure of the
+ * second or third call leaves the earlier work enqueued. */
+OSM_API size_t osm_ffn_workspace_size(const osm_plan* up, const osm_plan* down, int64_t M);
+OSM_API int osm_ffn_block(const osm_plan* up, const osm_plan* down, const uint16_t* X, int64_t M,
+                          const uint8_t* wu_codes, const uint8_t* wu_scales, const uint16_t* wu_hp,
+                          const uint8_t* wd_codes, const uint8_t* wd_scales, const uint16_t* wd_hp,
+                          const float* bias_down, uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* As osm_ffn_block for a host (preferably pinned) X_host [M][up->K] BF16 and
+ * a host Y_host [M][down->N] BF16: copies X in, runs the block and copies Y
+ * out, all enqueued on `stream` (the caller synchronises before reading
+ * Y_host). workspace: device memory of at least
+ * osm_ffn_host_workspace_size(up, down, M) bytes (the device X and Y plus
+ * osm_ffn_workspace_size). */
+OSM_API size_t osm_ffn_host_workspace_size(const osm_plan* up, const osm_plan* down, int64_t M);
+OSM_API int osm_ffn_block_host(const osm_plan* up, const osm_plan* down, const uint16_t* X_host, int64_t M,
+                               const uint8_t* wu_codes, const uint8_t* wu_scales, const uint16_t* wu_hp,
+                               const uint8_t* wd_codes, const uint8_t* wd_scales, const uint16_t* wd_hp,
+                               const float* bias_down, uint16_t* Y_host, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* ---- allocation-free device forward --------------------------------------
  * The paper has no counterpart to this entry point; it serves callers that
- * build their plans and pack their weights at load time but may not
- * allocate device memory while the layer runs (code captured into a CUDA
- * graph, or a runtime whose device memory belongs to its own pool).
+ * build their plans and pack their weights at load time but cannot
+ * allocate device memory while the layer runs: a serving runtime that
+ * reserves the GPU's memory up front for its own pool (a cudaMalloc would
+ * find none, and cudaMalloc / cudaFree synchronise the device), or a
+ * plug-in that its host framework hands only tensors and a stream.
  *
  * Same result as osm_quantize_act followed by osm_dual_gemm, on device
  * X [M][K] BF16 and device Y [M][N] (F32 or BF16, per epi), with no
@@ -384,7 +425,9 @@ OSM_API int osm_linear_host(const osm_plan* plan, const uint16_t* X_host, int64_
  * (every GPU that loads the library holds one until the process exits).
  * It calls no allocator. A call whose packed activations (codes + scales +
  * outlier slots, each rounded up to 256 bytes; see osm_plan_sizes) exceed
- * the array returns OSM_ERR_UNSUPPORTED before launching anything.
+ * the array -- at K = 5120, k = 128 about 5 700 tokens -- returns
+ * OSM_ERR_UNSUPPORTED before launching anything (so does any M above
+ * OSM_NOALLOC_SCRATCH_BYTES, checked before the sizes are computed).
  * The first call on a device looks up the array's device address; make
  * that first call before any stream capture. All calls share the array:
  * calls whose work overlaps on the GPU (different streams, or different

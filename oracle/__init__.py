@@ -17,8 +17,8 @@ score), smoothing/folding
 (Eq. (1)), quantize_act, pack_weights (all three block-scale modes),
 dual_gemm_rows (Eq. (5)), and the NVFP4 forms (E4M3 codec, block scale,
 element multiplier, per-tensor exponent, quantize_act_nv, pack_weights_nv,
-dual_gemm_rows_nv). The FP32 tanh-form GELU is pinned only to libm within an
-error bound ("parity unpinned" for its exact bits).
+dual_gemm_rows_nv), and the FFN's tanh-form GELU (its FP64 definition) with
+the one-step FP64 -> BF16 rounding.
 """
 from __future__ import annotations
 
@@ -89,12 +89,11 @@ def _load():
             lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
             lib.oracle_f16_to_f64.restype = ctypes.c_double
             lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
-            lib.oracle_gelu_tanh_f32.restype = ctypes.c_float
-            lib.oracle_gelu_tanh_f32.argtypes = [ctypes.c_float]
-            lib.oracle_gelu_exp_neg.restype = ctypes.c_float
-            lib.oracle_gelu_exp_neg.argtypes = [ctypes.c_float]
-            lib.oracle_gelu_recip.restype = ctypes.c_float
-            lib.oracle_gelu_recip.argtypes = [ctypes.c_float]
+            lib.oracle_gelu_tanh.restype = ctypes.c_double
+            lib.oracle_gelu_tanh.argtypes = [ctypes.c_double]
+            lib.oracle_f64_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
+            lib.oracle_gelu_rows.argtypes = [P, I64, P]
             lib.oracle_gelu_bf16_rows.argtypes = [P, I64, P]
             lib.oracle_e4m3_decode.restype = ctypes.c_double
             lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -160,16 +159,14 @@ def mx_scale_exponent(amax: float) -> int:
     return int(_load().oracle_mx_scale_exponent(float(amax)))
 
 
-def gelu_tanh_f32(x: float) -> float:
-    return float(_load().oracle_gelu_tanh_f32(float(np.float32(x))))
+def gelu_tanh(x: float) -> float:
+    """GELU(x) = 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3))) in FP64."""
+    return float(_load().oracle_gelu_tanh(float(x)))
 
 
-def gelu_exp_neg(x: float) -> float:
-    return float(_load().oracle_gelu_exp_neg(float(np.float32(x))))
-
-
-def gelu_recip(d: float) -> float:
-    return float(_load().oracle_gelu_recip(float(np.float32(d))))
+def f64_to_bf16(v: float) -> int:
+    """RNE of an FP64 value to BF16 in one step (bit pattern)."""
+    return int(_load().oracle_f64_to_bf16(float(v)))
 
 
 # ---- arrays --------------------------------------------------------------
@@ -305,8 +302,17 @@ def pack_weights(W: np.ndarray, s: np.ndarray, O: np.ndarray, mode: int, hp_fp16
     return codes, scales, w_hp
 
 
+def gelu(y: np.ndarray) -> np.ndarray:
+    """GELU_tanh(y) element-wise in FP64."""
+    y = _c(y, np.float64)
+    out = np.empty(y.shape, np.float64)
+    _load().oracle_gelu_rows(_p(y), y.size, _p(out))
+    return out
+
+
 def gelu_bf16(y: np.ndarray) -> np.ndarray:
-    """h = bf16(GELU_tanh(fp32(y))) element-wise for FP64 accumulators y."""
+    """h = bf16(GELU_tanh(y)) element-wise for FP64 accumulators y (GELU in
+    FP64, rounded once to BF16)."""
     y = _c(y, np.float64)
     out = np.empty(y.shape, np.uint16)
     _load().oracle_gelu_bf16_rows(_p(y), y.size, _p(out))

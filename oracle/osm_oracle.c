@@ -27,9 +27,7 @@
  * NVFP4 (a second 4-bit block format on the same dual product) has its
  * own section at the end of the file.
  *
- * Parity pins: see tests/test_oracle_*.py. Every function below is pinned
- * except the tanh-form GELU, which is pinned only against libm's tanh
- * within a stated error bound.
+ * Parity pins: see tests/test_oracle_*.py. Every function below is pinned.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -590,89 +588,62 @@ void oracle_dual_gemm_rows(const uint8_t* a_codes, const uint8_t* a_scales, cons
 }
 
 /* ------------------------------------------------------------------ */
-/* GELU (tanh form) in FP32 for the fused FFN epilogue                   */
+/* GELU (tanh form) of the FFN, by its definition in FP64               */
 /* ------------------------------------------------------------------ */
 
 /*
- * exp(a) for a <= 0 in FP32, with explicit operations: a is first clamped
- * to -100; Cody-Waite reduction a = n*ln2 + r (|r| <= ln2/2) with ln2 split
- * into a 12-bit high part and a low remainder; exp(r) by its Taylor series
- * to degree 7 in Horner form with fused multiply-adds (fmaf, one rounding
- * each). n is a*log2(e) rounded to the nearest integer (ties to even) in one
- * fused step: t = fmaf(a, LOG2E, 1.5*2^23) lies in [2^23, 2^24), where the
- * FP32 spacing is 1, and n = t - 1.5*2^23 exactly. The result is 0 for
- * n < -126 (exp(a) < 2^-126), else p * 2^n rounded once (exact unless it
- * is subnormal). Constants are the binary32 values of log2(e), ln2 split,
- * and 1/k!.
+ * GELU in the tanh form that the FFN uses: 0.5 x (1 + tanh(u)) with
+ * u = sqrt(2/pi) (x + 0.044715 x^3), evaluated in FP64 with libm's tanh.
+ * The pages fix no bits for it; this is the plain definition, and the CUDA
+ * epilogue's own FP32 routine is held to it by an error bound.
  */
-float oracle_gelu_exp_neg(float a)
+double oracle_gelu_tanh(double x)
 {
-    if (a < -100.0f) a = -100.0f;
-    if (a > 0.0f) a = 0.0f;
-    const float LOG2E = 0x1.715476p+0f;
-    const float LN2_HI = 0x1.62e4p-1f;      /* 12 significant bits */
-    const float LN2_LO = 0x1.7f7d1cp-20f;   /* ln2 - LN2_HI */
-    const float SHIFT = 0x1.8p+23f;         /* 1.5 * 2^23 */
-    float t = fmaf(a, LOG2E, SHIFT);
-    float n = t - SHIFT;
-    float r = fmaf(-n, LN2_HI, a);
-    r = fmaf(-n, LN2_LO, r);
-    float p = 0x1.a01a02p-13f;              /* 1/7! */
-    p = fmaf(p, r, 0x1.6c16c2p-10f);        /* 1/6! */
-    p = fmaf(p, r, 0x1.111112p-7f);         /* 1/5! */
-    p = fmaf(p, r, 0x1.555556p-5f);         /* 1/4! */
-    p = fmaf(p, r, 0x1.555556p-3f);         /* 1/3! */
-    p = fmaf(p, r, 0.5f);
-    p = fmaf(p, r, 1.0f);
-    p = fmaf(p, r, 1.0f);
-    if (n < -126.0f) return 0.0f;
-    return p * ldexpf(1.0f, (int)n);
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    double u = c * (x + 0.044715 * x * x * x);
+    return 0.5 * x * (1.0 + tanh(u));
 }
 
 /*
- * 1/d for d in [1, 2] by Newton's iteration for the reciprocal: the linear
- * seed y0 = 24/17 - (8/17) d (relative error at most 1/17 on [1, 2]), then
- * three steps y <- y + y (1 - d y), each as e = fmaf(-d, y, 1),
- * y = fmaf(y, e, y). The error squares at each step: 1/17 -> 2^-8.2 ->
- * 2^-16.3 -> below FP32 rounding.
+ * Round an FP64 value to the nearest BF16 value (8 significant bits,
+ * binary32's exponent range), ties to the even significand, in one step
+ * (no intermediate binary32 rounding). From the definition: with
+ * |v| = m 2^e, m in [1/2, 1), the BF16 quantum is 2^(e-8) for normal
+ * results and 2^-133 below 2^-126; v / quantum is rounded to an integer
+ * by rint (round-half-even in the default rounding mode) and scaled back,
+ * both exactly. Results of magnitude 2^128 or more are infinite.
  */
-float oracle_gelu_recip(float d)
+uint16_t oracle_f64_to_bf16(double v)
 {
-    float y = fmaf(-0x1.e1e1e2p-2f, d, 0x1.69696ap+0f);   /* 24/17 - (8/17) d */
-    for (int i = 0; i < 3; ++i) {
-        float e = fmaf(-d, y, 1.0f);
-        y = fmaf(y, e, y);
+    if (isnan(v)) return 0x7fc0;
+    double a = fabs(v);
+    double r;
+    if (a == 0.0 || isinf(a)) {
+        r = a;
+    } else {
+        int e;
+        frexp(a, &e);                       /* a = m 2^e, m in [0.5, 1) */
+        int qexp = e - 8;                   /* quantum of an 8-bit significand */
+        if (qexp < -133) qexp = -133;       /* BF16 subnormal quantum */
+        r = ldexp(rint(ldexp(a, -qexp)), qexp);
+        if (r >= ldexp(1.0, 128)) r = INFINITY;
     }
-    return y;
+    float f = (float)r;                     /* exact: r is a BF16 value (or inf) */
+    uint16_t h = (uint16_t)(f32_as_u32(f) >> 16);
+    return signbit(v) ? (uint16_t)(h | 0x8000u) : h;
 }
 
-/*
- * GELU in its tanh form, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi)(x + 0.044715
- * x^3), for finite x, evaluated through the identity 0.5 (1 + tanh(u)) =
- * sigma(2u) = 1 / (1 + exp(-2u)): with E = exp(-2|u|),
- *   x sigma(2u) = x / (1 + E)  for u >= 0,   x E / (1 + E)  for u < 0,
- * and u has the sign of x, so the numerator is max(x, x E) (0 <= E <= 1).
- * Every operation in FP32 in the order written: x2 = x*x;
- * k = fmaf(C1, x2, 1); u = (C0*x)*k; E = exp(-2|u|) as above;
- * y = recip(1 + E); result fmaxf(x, x*E) * y.
- */
-float oracle_gelu_tanh_f32(float x)
+/* GELU of FP64 accumulators: g[i] = GELU(y[i]) in FP64. */
+void oracle_gelu_rows(const double* y, int64_t n, double* g)
 {
-    const float C0 = 0x1.988454p-1f;   /* sqrt(2/pi) */
-    const float C1 = 0x1.6e4e26p-5f;   /* 0.044715 */
-    float x2 = x * x;
-    float k = fmaf(C1, x2, 1.0f);
-    float u = (C0 * x) * k;
-    float E = oracle_gelu_exp_neg(-2.0f * fabsf(u));
-    float y = oracle_gelu_recip(1.0f + E);
-    return fmaxf(x, x * E) * y;
+    for (int64_t i = 0; i < n; ++i) g[i] = oracle_gelu_tanh(y[i]);
 }
 
-/* FFN hidden activations from FP64 accumulators: h = bf16(GELU(fp32(y))),
- * y [n] FP64 -> h [n] BF16 words. */
+/* FFN hidden activations from FP64 accumulators: h = bf16(GELU(y)),
+ * rounded once from FP64. */
 void oracle_gelu_bf16_rows(const double* y, int64_t n, uint16_t* h)
 {
-    for (int64_t i = 0; i < n; ++i) h[i] = oracle_f32_to_bf16(oracle_gelu_tanh_f32((float)y[i]));
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_f64_to_bf16(oracle_gelu_tanh(y[i]));
 }
 
 /* ------------------------------------------------------------------ */

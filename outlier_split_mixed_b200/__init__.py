@@ -64,6 +64,10 @@ _SIGNATURES = {
     "osm_linear_host": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "osm_scales_to_logical": (_I, [_P, _I64, _I64, _P]),
     "osm_linear_noalloc": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P]),
+    "osm_ffn_workspace_size": (_SZ, [_P, _P, _I64]),
+    "osm_ffn_host_workspace_size": (_SZ, [_P, _P, _I64]),
+    "osm_ffn_block": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "osm_ffn_block_host": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "osm_last_error": (ctypes.c_char_p, []),
 }
 
@@ -441,15 +445,72 @@ def linear_host(plan: Plan, X_host, M: int, w_codes, w_scales, w_hp, Y_host, wor
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def ffn_workspace_size(up: Plan, down: Plan, M: int) -> int:
+    """Device bytes osm_ffn_block needs for M tokens (both layers' packed activations)."""
+    return int(lib().osm_ffn_workspace_size(up.handle, down.handle, M))
+
+
+def ffn_host_workspace_size(up: Plan, down: Plan, M: int) -> int:
+    """Device bytes osm_ffn_block_host needs for M tokens."""
+    return int(lib().osm_ffn_host_workspace_size(up.handle, down.handle, M))
+
+
+def _ffn_weight_ptrs(up: Plan, down: Plan, wu, wd):
+    cu, su, hu = up.sizes(up.N)
+    cd, sd, hd = down.sizes(down.N)
+    return (_ptr(wu[0], "wu_codes", _u8_types(), cu, allow_none=cu == 0),
+            _ptr(wu[1], "wu_scales", _u8_types(), su, allow_none=su == 0),
+            _ptr(wu[2], "wu_hp", _bf16_types(), hu, allow_none=hu == 0),
+            _ptr(wd[0], "wd_codes", _u8_types(), cd, allow_none=cd == 0),
+            _ptr(wd[1], "wd_scales", _u8_types(), sd, allow_none=sd == 0),
+            _ptr(wd[2], "wd_hp", _bf16_types(), hd, allow_none=hd == 0))
+
+
+def ffn_block(up: Plan, down: Plan, X, wu, wd, Y, workspace, bias_down=None, stream=None):
+    """One FFN block on the device (osm_ffn_block): quantize_act(up), the
+    up-projection with the fused GELU + smoothing + requantisation epilogue,
+    the down-projection to BF16. wu = (codes, scales, hp) packed by
+    pack_weights_for_next(up, down), wd packed by pack_weights(down).
+    X: [M][up.K] BF16, Y: [M][down.N] BF16, both CUDA tensors."""
+    import torch
+    M, K = X.shape
+    if K != up.K or tuple(Y.shape) != (M, down.N):
+        raise ValueError("X must be [M][up.K] and Y [M][down.N]")
+    _check(lib().osm_ffn_block(up.handle, down.handle, _ptr(X, "X", _bf16_types()), M,
+                               *_ffn_weight_ptrs(up, down, wu, wd),
+                               _ptr(bias_down, "bias_down", (torch.float32,), down.N * 4, allow_none=True),
+                               _ptr(Y, "Y", _bf16_types(), M * down.N * 2), _ptr(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ffn_block_host(up: Plan, down: Plan, X_host, wu, wd, Y_host, workspace, bias_down=None, stream=None):
+    """osm_ffn_block_host: host (pinned) X in, the block on the device, host
+    Y out, all enqueued on `stream`; the caller synchronises."""
+    import torch
+    for t, n in ((X_host, "X_host"), (Y_host, "Y_host")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous host tensor")
+    M, K = X_host.shape
+    if K != up.K or tuple(Y_host.shape) != (M, down.N):
+        raise ValueError("X_host must be [M][up.K] and Y_host [M][down.N]")
+    _check(lib().osm_ffn_block_host(up.handle, down.handle, ctypes.c_void_p(X_host.data_ptr()), M,
+                                    *_ffn_weight_ptrs(up, down, wu, wd),
+                                    _ptr(bias_down, "bias_down", (torch.float32,), down.N * 4, allow_none=True),
+                                    ctypes.c_void_p(Y_host.data_ptr()), _ptr(workspace, "workspace"),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def linear_noalloc(plan: Plan, X, w_codes, w_scales, w_hp, Y, bias=None, epi: int = EPI_F32, stream=None):
     """quantize_act + dual_gemm with the packed activations in the library's
     static scratch (osm_linear_noalloc): nothing is allocated, for callers
-    that may not allocate device memory at run time (CUDA-graph capture,
-    pool-owned device memory). Calls that overlap on the GPU race on the
-    shared scratch; the first call on a device should precede any capture."""
+    that cannot allocate device memory at run time (a runtime whose pool
+    owns the GPU's memory, a plug-in handed only tensors and a stream).
+    Calls that overlap on the GPU race on the shared scratch; the first call
+    on a device looks up the scratch address and should precede any stream
+    capture."""
     import torch
     M, K = X.shape
     if K != plan.K:

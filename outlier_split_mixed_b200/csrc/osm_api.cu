@@ -456,7 +456,7 @@ int osm_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* a
                      uint16_t* a_hp, void* stream) {
     g_err[0] = 0;
     OSM_TRY(check_plan(p));
-    OSM_REQUIRE(M >= 1, "quantize_act: M must be >= 1");
+    OSM_REQUIRE(M >= 1 && M <= (int64_t(1) << 31) - 1, "quantize_act: need 1 <= M < 2^31");
     OSM_REQUIRE(X && aligned16(X), "quantize_act: X must be a 16-byte aligned device pointer");
     OSM_REQUIRE(p->Kbp == 0 || (a_codes && aligned16(a_codes) && a_scales && aligned16(a_scales)),
                 "quantize_act: a_codes / a_scales null or misaligned");
@@ -502,7 +502,7 @@ int osm_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_sc
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t osm_linear_workspace_size(const osm_plan* p, int64_t M, int epi) {
-    if (!p || M < 1) return 0;
+    if (!p || M < 1 || M > (int64_t(1) << 31) - 1) return 0;
     size_t cb, sb, hb;
     osm_plan_sizes(p, M, &cb, &sb, &hb);
     const size_t yb = static_cast<size_t>(M * p->N) * (epi == OSM_EPI_BF16 ? 2 : 4);
@@ -515,7 +515,7 @@ int osm_linear_host(const osm_plan* p, const uint16_t* X_host, int64_t M, const 
     g_err[0] = 0;
     OSM_TRY(check_plan(p));
     OSM_REQUIRE(X_host && Y_host, "linear_host: X_host / Y_host is NULL");
-    OSM_REQUIRE(M >= 1, "linear_host: M must be >= 1");
+    OSM_REQUIRE(M >= 1 && M <= (int64_t(1) << 31) - 1, "linear_host: need 1 <= M < 2^31");
     OSM_REQUIRE(epi == OSM_EPI_F32 || epi == OSM_EPI_BF16, "linear_host: epilogue must be F32 or BF16");
     const size_t need = osm_linear_workspace_size(p, M, epi);
     OSM_REQUIRE(workspace && aligned16(workspace) && workspace_bytes >= need,
@@ -540,6 +540,88 @@ int osm_linear_host(const osm_plan* p, const uint16_t* X_host, int64_t M, const 
     OSM_TRY(osm_dual_gemm(p, codes, scales, hp, M, w_codes, w_scales, w_hp, bias, epi, dY, nullptr, nullptr,
                           nullptr, nullptr, stream));
     return check_cuda(cudaMemcpyAsync(Y_host, dY, yb, cudaMemcpyDeviceToHost, st), "linear_host: copy Y");
+}
+
+// ---- one FFN block: quantize_act(up) -> dual_gemm(up, GELU_REQUANT) -> dual_gemm(down, BF16)
+
+size_t osm_ffn_workspace_size(const osm_plan* up, const osm_plan* down, int64_t M) {
+    if (!up || !down || M < 1 || M > (int64_t(1) << 31) - 1 || up->N != down->K) return 0;
+    size_t cu, su, hu, cd, sd, hd;
+    osm_plan_sizes(up, M, &cu, &su, &hu);
+    osm_plan_sizes(down, M, &cd, &sd, &hd);
+    return align256(cu) + align256(su) + align256(hu) + align256(cd) + align256(sd) + align256(hd);
+}
+
+size_t osm_ffn_host_workspace_size(const osm_plan* up, const osm_plan* down, int64_t M) {
+    const size_t inner = osm_ffn_workspace_size(up, down, M);
+    if (!inner) return 0;
+    return inner + align256(static_cast<size_t>(M * up->K * 2)) + align256(static_cast<size_t>(M * down->N * 2));
+}
+
+int osm_ffn_block(const osm_plan* up, const osm_plan* down, const uint16_t* X, int64_t M, const uint8_t* wu_codes,
+                  const uint8_t* wu_scales, const uint16_t* wu_hp, const uint8_t* wd_codes, const uint8_t* wd_scales,
+                  const uint16_t* wd_hp, const float* bias_down, uint16_t* Y, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(up));
+    OSM_TRY(check_plan(down));
+    OSM_REQUIRE(up->N == down->K, "ffn_block: up->N (%lld) must equal down->K (%lld)", (long long)up->N,
+                (long long)down->K);
+    OSM_REQUIRE(M >= 1 && M <= (int64_t(1) << 31) - 1, "ffn_block: need 1 <= M < 2^31");
+    const size_t need = osm_ffn_workspace_size(up, down, M);
+    OSM_REQUIRE(workspace && aligned16(workspace) && workspace_bytes >= need, "ffn_block: workspace needs %zu bytes",
+                need);
+    size_t cu, su, hu, cd, sd, hd;
+    osm_plan_sizes(up, M, &cu, &su, &hu);
+    osm_plan_sizes(down, M, &cd, &sd, &hd);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* a_codes = ws;
+    ws += align256(cu);
+    uint8_t* a_scales = ws;
+    ws += align256(su);
+    uint16_t* a_hp = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(hu);
+    uint8_t* h_codes = ws;
+    ws += align256(cd);
+    uint8_t* h_scales = ws;
+    ws += align256(sd);
+    uint16_t* h_hp = reinterpret_cast<uint16_t*>(ws);
+    // every argument of the three calls is checked by them before anything is
+    // enqueued; a failure of the second or third leaves the earlier work queued
+    OSM_TRY(osm_quantize_act(up, X, M, a_codes, a_scales, a_hp, stream));
+    OSM_TRY(osm_dual_gemm(up, a_codes, a_scales, a_hp, M, wu_codes, wu_scales, wu_hp, nullptr, OSM_EPI_GELU_REQUANT,
+                          nullptr, down, h_codes, h_scales, h_hp, stream));
+    return osm_dual_gemm(down, h_codes, h_scales, h_hp, M, wd_codes, wd_scales, wd_hp, bias_down, OSM_EPI_BF16, Y,
+                         nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+int osm_ffn_block_host(const osm_plan* up, const osm_plan* down, const uint16_t* X_host, int64_t M,
+                       const uint8_t* wu_codes, const uint8_t* wu_scales, const uint16_t* wu_hp,
+                       const uint8_t* wd_codes, const uint8_t* wd_scales, const uint16_t* wd_hp,
+                       const float* bias_down, uint16_t* Y_host, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    g_err[0] = 0;
+    OSM_TRY(check_plan(up));
+    OSM_TRY(check_plan(down));
+    OSM_REQUIRE(X_host && Y_host, "ffn_block_host: X_host / Y_host is NULL");
+    OSM_REQUIRE(up->N == down->K, "ffn_block_host: up->N (%lld) must equal down->K (%lld)", (long long)up->N,
+                (long long)down->K);
+    OSM_REQUIRE(M >= 1 && M <= (int64_t(1) << 31) - 1, "ffn_block_host: need 1 <= M < 2^31");
+    const size_t need = osm_ffn_host_workspace_size(up, down, M);
+    OSM_REQUIRE(workspace && aligned16(workspace) && workspace_bytes >= need,
+                "ffn_block_host: workspace needs %zu bytes", need);
+    const size_t xb = static_cast<size_t>(M * up->K * 2), yb = static_cast<size_t>(M * down->N * 2);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint16_t* dX = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(xb);
+    uint16_t* dY = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(yb);
+    const size_t inner = osm_ffn_workspace_size(up, down, M);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    OSM_TRY(check_cuda(cudaMemcpyAsync(dX, X_host, xb, cudaMemcpyHostToDevice, st), "ffn_block_host: copy X"));
+    OSM_TRY(osm_ffn_block(up, down, dX, M, wu_codes, wu_scales, wu_hp, wd_codes, wd_scales, wd_hp, bias_down, dY, ws,
+                          inner, stream));
+    return check_cuda(cudaMemcpyAsync(Y_host, dY, yb, cudaMemcpyDeviceToHost, st), "ffn_block_host: copy Y");
 }
 
 int osm_scales_to_logical(const uint8_t* sw, int64_t rows, int64_t nblocks, uint8_t* logical) {

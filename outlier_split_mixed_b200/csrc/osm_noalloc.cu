@@ -3,11 +3,13 @@
 // file-scope static device array instead of caller-provided buffers.
 //
 // Who needs this: callers that create their plans and pack their weights
-// at load time but must not allocate device memory when the layer runs --
-// for example code that is being captured into a CUDA graph, or a serving
-// runtime whose device memory is owned by its own pool allocator, where a
-// cudaMalloc (or an allocating library call) at run time is not allowed.
-// They pass only X, the packed weights and Y; the scratch is in this file.
+// at load time but cannot allocate device memory when the layer runs. A
+// serving runtime that reserves the GPU's memory up front for its own pool
+// leaves nothing for a cudaMalloc, and a plug-in that a host framework
+// hands only tensors and a stream has no access to that framework's
+// allocator; cudaMalloc and cudaFree would also synchronise the whole
+// device in the middle of other streams' work. Such callers pass only X,
+// the packed weights and Y; the scratch is in this file.
 //
 // The array is module data: every GPU that loads the library holds its own
 // copy of it until the process exits. In host code `g_act_scratch` is only
@@ -57,6 +59,14 @@ extern "C" OSM_API int osm_linear_noalloc(const osm_plan* p, const uint16_t* X, 
     using namespace osm;
     if (!p) return fail(OSM_ERR_INVALID_ARG, "linear_noalloc: plan is NULL");
     if (M < 1) return fail(OSM_ERR_INVALID_ARG, "linear_noalloc: M must be >= 1");
+    // Every row takes at least one byte of packed activations, so a batch
+    // above this many rows cannot fit; checked before the size arithmetic
+    // below, whose 64-bit products would wrap for absurd M.
+    if (M > static_cast<int64_t>(OSM_NOALLOC_SCRATCH_BYTES))
+        return fail(OSM_ERR_UNSUPPORTED,
+                    "linear_noalloc: M=%lld rows cannot fit the static scratch of %u bytes; split the batch or use "
+                    "osm_quantize_act + osm_dual_gemm",
+                    (long long)M, (unsigned)OSM_NOALLOC_SCRATCH_BYTES);
     if (epi != OSM_EPI_F32 && epi != OSM_EPI_BF16)
         return fail(OSM_ERR_INVALID_ARG, "linear_noalloc: epilogue must be OSM_EPI_F32 or OSM_EPI_BF16");
     size_t cb = 0, sb = 0, hb = 0;

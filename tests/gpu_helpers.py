@@ -142,3 +142,16 @@ def compare_layer(g, o, rows=None, check_weights_rows=None):
     assert_bitexact("a_scales", g["a_scales_full"][:M][r], o["a_scales"])
     assert np.all(g["a_scales_full"][M:] == 0), "padding rows of a_scales must be 0"
     assert_bitexact("a_hp", g["a_hp"], o["a_hp"])
+
+
+def gelu_tolerance(y, T, g):
+    """Bound on |h_gpu - GELU(y)| for h_gpu = bf16(GELU_f32(acc)), with y the
+    oracle's FP64 sum, T = sum |a w| and g = GELU(y) in FP64:
+      1.13 (1e-5 T + 1e-6)        the FP32 accumulation bound through GELU
+                                  (|GELU'| <= 1.129);
+      5e-7 |g| + 2e-8 |y|         the epilogue's FP32 routine against the
+                                  definition (the relative error of
+                                  exp(-2|u|) grows with |u| in the left tail);
+      2^-8 |g| (1 + 1e-6)         one rounding to BF16 (half an ulp)."""
+    return (1.13 * (1e-5 * T + 1e-6) + 5e-7 * np.abs(g) + 2e-8 * np.abs(y)
+            + 2.0 ** -8 * (1.0 + 1e-6) * np.abs(g) + 1e-30)

@@ -108,6 +108,11 @@ def test_argument_errors_need_no_gpu():
     assert rc == osm.ERR_INVALID_ARG   # s must be positive
     assert L.osm_dual_gemm(None, *([None] * 3), 1, *([None] * 4), 0, None, None, None, None, None, None) \
         == osm.ERR_INVALID_ARG
+    # the FFN block entry points refuse missing plans before touching a device
+    assert L.osm_ffn_workspace_size(None, None, 128) == 0
+    assert L.osm_ffn_host_workspace_size(None, None, 128) == 0
+    assert L.osm_ffn_block(None, None, None, 128, *([None] * 7), None, None, 0, None) == osm.ERR_INVALID_ARG
+    assert L.osm_ffn_block_host(None, None, None, 128, *([None] * 7), None, None, 0, None) == osm.ERR_INVALID_ARG
 
 
 def test_nvfp4_host_helpers_reject_bad_statistics():

@@ -1,0 +1,204 @@
+"""The full FFN block workload end to end against the oracle: four blocks of
+32760 tokens, each up-projection 5120 -> 13824 with GELU, smoothing and
+MXFP4 requantisation fused into its epilogue, then the down-projection
+13824 -> 5120 to BF16 (the implementation paragraph of "W4A4 Quantization
+for Inference on Wan2.2-I2V-A14B": every FFN linear map smoothed and split,
+activations divided by s, quantised and routed; per-layer statistics from
+calibration data).
+
+Per block, through the C ABI (the final Y through osm_ffn_block_host, from
+pinned host memory):
+  * calibration on a separate 2048-token batch: up-projection statistics,
+    s and O bit-exact; the down-projection's statistics come from the
+    unquantised GELU(X_cal W_up) (the GPU runs a k = K, s = 1 plan with the
+    GELU_BF16 epilogue; the oracle takes an FP64 matmul of the same BF16
+    operands and its FP64 GELU). The two sides accumulate in different
+    precisions, so their maxima agree to one BF16 ulp; s and O of the
+    down-projection are then bit-exact against the oracle's calibration of
+    the GPU's statistics (the FP decision taken in the kernel's precision),
+    and every channel on which the two outlier sets differ lies within one
+    ulp of the k-th largest statistic;
+  * both packed weight sets bit-exact (every row);
+  * on 48 stratified token rows (including the ragged last 128-row tile):
+    the up-projection's activation codes, scales and outlier slots
+    bit-exact; the GPU's hidden activations (GELU_BF16 epilogue, same
+    accumulators as the fused one) within the accumulation bound carried
+    through GELU of the oracle's FP64 GELU; the fused requantisation bit-exact
+    against the oracle's quantize_act of those hidden activations; the
+    down-projection's BF16 output within 1e-5 sum|a w| + 1e-6 + 2^-8 |y| of
+    the oracle's FP64 product of those codes;
+  * the oracle's own chain (its own BF16 GELU, requantisation and product)
+    agrees with the GPU's Y to a small relative error, since the two chains
+    differ only where a hidden activation rounds to a neighbouring BF16
+    value.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import outlier_split_mixed_b200 as osm  # noqa: E402
+from outlier_split_mixed_b200 import synth  # noqa: E402
+from gpu_helpers import (assert_bitexact, assert_y_close, gelu_tolerance, to_dev_bf16, to_np_u16,  # noqa: E402
+                         unswizzle)
+
+pytestmark = pytest.mark.gpu
+
+CFG = synth.FFN
+ROWS = 48
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    osm.lib()
+
+
+def _bf16_f64(h):
+    return synth.bf16_bits_to_f32(h).astype(np.float64)
+
+
+def _order(K, O):
+    return np.concatenate([np.setdiff1d(np.arange(K), O), O]).astype(np.int32)
+
+
+@pytest.mark.parametrize("layer", range(CFG.layers))
+def test_ffn_block_end_to_end(layer):
+    M, D, F = CFG.M, CFG.d_model, CFG.d_ff
+    Xc, Wu, Wd, X = CFG.make_calib(layer), CFG.make_w_up(layer), CFG.make_w_down(layer), CFG.make_x(layer)
+    Tc = Xc.shape[0]
+
+    # ------------------------------------------------------------ CUDA path
+    Xcd, Wud, Wdd = to_dev_bf16(Xc), to_dev_bf16(Wu), to_dev_bf16(Wd)
+    s_u, inv_u, O_u, amax_u, wmax_u = osm.calibrate([Xcd], Wud, CFG.alpha_up, CFG.k_up)
+    full = osm.Plan(D, F, D, np.ones(D, np.float32), np.arange(D, dtype=np.int32), CFG.wmode_up)
+    fa, fw = full.alloc_packed(Tc), full.alloc_packed(F)
+    osm.quantize_act(full, Xcd, *fa)
+    osm.pack_weights(full, Wud, *fw)
+    Hc = torch.empty((Tc, F), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(full, *fa, Tc, *fw, Hc, epi=osm.EPI_GELU_BF16)
+    s_d, inv_d, O_d, amax_d, wmax_d = osm.calibrate([Hc], Wdd, CFG.alpha_down, CFG.k_down)
+    assert full.status() == 0
+    full.close()
+    del fa, fw, Hc
+
+    up = osm.Plan(D, F, CFG.k_up, s_u, O_u, CFG.wmode_up)
+    down = osm.Plan(F, D, CFG.k_down, s_d, O_d, CFG.wmode_down)
+    wu, wd = up.alloc_packed(F), down.alloc_packed(D)
+    osm.pack_weights_for_next(up, down, Wud, *wu)
+    osm.pack_weights(down, Wdd, *wd)
+
+    # the block through the host entry point: pinned X in, Y out
+    Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, D), dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(osm.ffn_host_workspace_size(up, down, M), dtype=torch.uint8, device="cuda")
+    osm.ffn_block_host(up, down, Xh, wu, wd, Yh, ws)
+
+    # the same block by separate calls, keeping every intermediate
+    Xd = to_dev_bf16(X)
+    a_up = up.alloc_packed(M)
+    osm.quantize_act(up, Xd, *a_up)
+    h_dn = down.alloc_packed(M)
+    osm.dual_gemm(up, *a_up, M, *wu, None, epi=osm.EPI_GELU_REQUANT, next_plan=down, next_buffers=h_dn)
+    Y2 = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(down, *h_dn, M, *wd, Y2, epi=osm.EPI_BF16)
+    wu_nat = up.alloc_packed(F)
+    osm.pack_weights(up, Wud, *wu_nat)
+    H = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    osm.dual_gemm(up, *a_up, M, *wu_nat, H, epi=osm.EPI_GELU_BF16)
+    torch.cuda.synchronize()
+    assert up.status() == 0 and down.status() == 0
+    assert torch.equal(Yh.view(torch.int16), Y2.cpu().view(torch.int16)), "ffn_block_host differs from the calls"
+
+    R = synth.sample_rows(M, ROWS)
+    Rd = torch.from_numpy(R).cuda()
+    g_a_codes = a_up[0].view(M, up.Kbp // 2)[Rd].cpu().numpy()
+    g_a_scales = unswizzle(a_up[1].cpu().numpy(), M, up.Kbp // 32)[R]
+    g_a_hp = to_np_u16(a_up[2].view(M, up.kp)[Rd])
+    g_h_codes = h_dn[0].view(M, down.Kbp // 2)[Rd].cpu().numpy()
+    g_h_scales_full = unswizzle(h_dn[1].cpu().numpy(), M, down.Kbp // 32)
+    g_h_hp = to_np_u16(h_dn[2].view(M, down.kp)[Rd])
+    g_H = to_np_u16(H[Rd])
+    g_Y = Yh.numpy().view(np.uint16)[R]
+    g_wu = (wu[0].cpu().numpy().reshape(F, up.Kbp // 2), unswizzle(wu[1].cpu().numpy(), F, up.Kbp // 32),
+            to_np_u16(wu[2]).reshape(F, up.kp))
+    g_wd = (wd[0].cpu().numpy().reshape(D, down.Kbp // 2), unswizzle(wd[1].cpu().numpy(), D, down.Kbp // 32),
+            to_np_u16(wd[2]).reshape(D, down.kp))
+    order = down.channel_order()
+    del H, Y2, Xd, a_up, h_dn, wu_nat, ws
+    up.close()
+    down.close()
+
+    # ------------------------------------------------------------ oracle
+    # up-projection calibration
+    amax_u_o, wmax_u_o = oracle.act_amax(Xc), oracle.weight_amax(Wu)
+    so_u, invo_u, Oo_u = oracle.calibrate(amax_u_o, wmax_u_o, CFG.alpha_up, CFG.k_up)
+    assert_bitexact("amax (up)", amax_u, amax_u_o)
+    assert_bitexact("wmax (up)", wmax_u, wmax_u_o)
+    assert_bitexact("s (up)", s_u, so_u)
+    assert_bitexact("inv_s (up)", inv_u, invo_u)
+    assert_bitexact("O (up)", O_u, Oo_u)
+
+    # down-projection statistics from the unquantised GELU(X_cal W_up)
+    y_cal = _bf16_f64(Xc) @ _bf16_f64(Wu)         # exact BF16 products, FP64 sums
+    amax_d_o = oracle.act_amax(oracle.gelu_bf16(y_cal))
+    del y_cal
+    wmax_d_o = oracle.weight_amax(Wd)
+    assert_bitexact("wmax (down)", wmax_d, wmax_d_o)
+    ulp = np.ldexp(1.0, np.frexp(amax_d_o)[1] - 8)  # BF16 ulp of each maximum
+    assert np.all(np.abs(amax_d.astype(np.float64) - amax_d_o) <= ulp), "down statistics beyond one BF16 ulp"
+    # s and O from the GPU's statistics, decided as the oracle decides them
+    so_d, invo_d, Oo_d = oracle.calibrate(amax_d, wmax_d_o, CFG.alpha_down, CFG.k_down)
+    assert_bitexact("s (down)", s_d, so_d)
+    assert_bitexact("inv_s (down)", inv_d, invo_d)
+    assert_bitexact("O (down)", O_d, Oo_d)
+    # the oracle's own outlier set differs only at near-ties of the k-th statistic
+    Oo_own = oracle.calibrate(amax_d_o, wmax_d_o, CFG.alpha_down, CFG.k_down)[2]
+    kth = np.sort(amax_d_o)[::-1][CFG.k_down - 1]
+    for j in np.setxor1d(Oo_own, Oo_d):
+        assert abs(amax_d_o[j] - kth) <= 2 * ulp[j], ("outlier sets differ away from the k-th statistic", j)
+    assert np.array_equal(order, _order(F, Oo_d))
+
+    # both packed weight sets, every row
+    wu_o = oracle.pack_weights(Wu[:, order], so_u, Oo_u, CFG.wmode_up)
+    for name, g, o in zip(("codes", "scales", "hp"), g_wu, wu_o):
+        assert_bitexact(f"W_up {name}", g[:F], o)
+    wd_o = oracle.pack_weights(Wd, so_d, Oo_d, CFG.wmode_down)
+    for name, g, o in zip(("codes", "scales", "hp"), g_wd, wd_o):
+        assert_bitexact(f"W_down {name}", g[:D], o)
+
+    # sampled tokens: the up-projection's activations
+    a_o = oracle.quantize_act(X[R], invo_u, Oo_u)
+    assert_bitexact("a codes", g_a_codes, a_o[0])
+    assert_bitexact("a scales", g_a_scales, a_o[1])
+    assert_bitexact("a outlier slots", g_a_hp, a_o[2])
+    # hidden activations: the GPU's GELU_BF16 against the FP64 GELU of the oracle's sums
+    r = np.arange(len(R))
+    y_perm, T_perm = oracle.dual_gemm_rows(*a_o, r, *wu_o)   # output channels in the down plan's order
+    y_up = np.empty_like(y_perm)
+    T_up = np.empty_like(T_perm)
+    y_up[:, order], T_up[:, order] = y_perm, T_perm
+    g = oracle.gelu(y_up)
+    err = np.abs(_bf16_f64(g_H) - g)
+    assert np.all(err <= gelu_tolerance(y_up, T_up, g)), "hidden activations outside the GELU bound"
+    # the fused requantisation = the oracle's quantize_act of those activations
+    h_o = oracle.quantize_act(g_H, invo_d, Oo_d)
+    assert_bitexact("hidden codes", g_h_codes, h_o[0])
+    assert_bitexact("hidden scales", g_h_scales_full[R], h_o[1])
+    assert np.all(g_h_scales_full[M:] == 0), "padding rows of the hidden scales must be 0"
+    assert_bitexact("hidden outlier slots", g_h_hp, h_o[2])
+    # the block output
+    y_dn, T_dn = oracle.dual_gemm_rows(*h_o, r, *wd_o)
+    Yg = _bf16_f64(g_Y)
+    assert_y_close(Yg, y_dn, T_dn, bf16=True)
+
+    # the oracle's own chain end to end
+    c_o = oracle.quantize_act(oracle.gelu_bf16(y_up), invo_d, Oo_d)
+    y_chain, _ = oracle.dual_gemm_rows(*c_o, r, *wd_o)
+    rel = float(np.linalg.norm(Yg - y_chain) / np.linalg.norm(y_chain))
+    flips = int(np.sum(g_H != oracle.gelu_bf16(y_up)))
+    print(f"block {layer}: relative error of Y against the oracle's own chain {rel:.2e}; "
+          f"{flips} of {g_H.size} hidden activations round to a neighbouring BF16 value")
+    assert rel <= 1e-3

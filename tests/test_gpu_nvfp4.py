@@ -59,18 +59,19 @@ def test_nvfp4_layer_parity(case):
 
 
 def test_nvfp4_gelu_bf16_epilogue():
-    # GELU_BF16 applies GELU to 2^(g_a+g_w) acc: the output equals the oracle's
-    # bf16(GELU(y)) wherever y is exactly representable; check by tolerance
+    # GELU_BF16 applies GELU to 2^(g_a+g_w) acc: checked by tolerance against
+    # the FP64 GELU of the oracle's accumulators
     M, K, N, k = 128, 512, 256, 32
     X, W = _inputs(M, K, N, "heavy", 5)
     g = gpu_layer(X, W, 0.5, k, osm.WSCALE_1x32, epi=osm.EPI_GELU_BF16, nv=True)
     o = oracle_layer(X, W, 0.5, k, osm.WSCALE_1x32, nv=True)
     compare_layer(g, o)
     import oracle
-    h = oracle.gelu_bf16(o["y"])
-    want = synth.bf16_bits_to_f32(h).astype(np.float64)
-    # |GELU'| <= 1.13: the accumulation bound carried through GELU, plus one BF16 rounding each side
-    tol = 1.13 * (1e-5 * o["T"] + 1e-6) + 2.0 ** -7 * np.abs(want) + 1e-30
+    want = oracle.gelu(o["y"])
+    # |GELU'| <= 1.13: the accumulation bound carried through GELU, plus one
+    # BF16 rounding and the FP32 routine's error against the FP64 definition
+    tol = (1.13 * (1e-5 * o["T"] + 1e-6) + 5e-7 * np.abs(want) + 2e-8 * np.abs(o["y"])
+           + 2.0 ** -8 * (1.0 + 1e-6) * np.abs(want) + 1e-30)
     assert np.all(np.abs(g["Y"] - want) <= tol)
 
 

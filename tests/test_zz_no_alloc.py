@@ -2,10 +2,13 @@
 entry points (osm_quantize_act + osm_dual_gemm on caller-owned buffers).
 
 osm_linear_noalloc exists for callers that cannot allocate device memory
-while the layer runs (work captured into a CUDA graph, or a runtime whose
-device memory belongs to its own pool); its packed activations live in a
-static device array inside the library. This module is self-contained so
-it passes alone in a fresh process and after the rest of the suite."""
+while the layer runs (a serving runtime whose pool owns the GPU's memory,
+a plug-in that its host framework hands only tensors and a stream); its
+packed activations live in a static device array inside the library. Both
+paths run the same kernels on the same operands, so their outputs must be
+bit-identical: any difference would be a fault in the shared scratch's
+layout. This module is self-contained so it passes alone in a fresh
+process and after the rest of the suite."""
 import numpy as np
 import pytest
 
@@ -45,11 +48,11 @@ def _reference(plan, X, wpack, bias, epi):
     return Y
 
 
-def _close(a, b, bf16):
-    # the tolerance the parity tests use, relative to the regular path's output
-    a, b = a.double(), b.double()
-    tol = 1e-5 * b.abs().max().item() + 1e-6 + (2.0 ** -8 * b.abs() if bf16 else 0.0)
-    assert torch.all((a - b).abs() <= tol)
+def _same(a, b):
+    # bit for bit: the same kernels on the same packed operands
+    assert a.dtype == b.dtype and a.shape == b.shape
+    assert torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a.view(torch.int16),
+                       b.view(torch.int32) if b.dtype == torch.float32 else b.view(torch.int16))
 
 
 @pytest.mark.parametrize("epi", [osm.EPI_F32, osm.EPI_BF16])
@@ -66,8 +69,8 @@ def test_two_calls_in_a_row_match_the_regular_path(layer, epi):
     osm.linear_noalloc(plan, X2, *wpack, Y2, bias=bias, epi=epi)
     torch.cuda.synchronize()
     assert plan.status() == 0
-    _close(Y1, _reference(plan, X1, wpack, bias, epi), epi == osm.EPI_BF16)
-    _close(Y2, _reference(plan, X2, wpack, bias, epi), epi == osm.EPI_BF16)
+    _same(Y1, _reference(plan, X1, wpack, bias, epi))
+    _same(Y2, _reference(plan, X2, wpack, bias, epi))
 
 
 def test_allocates_nothing_and_rejects_oversized_batches(layer):
@@ -92,3 +95,14 @@ def test_allocates_nothing_and_rejects_oversized_batches(layer):
                                                 osm._ptr(wpack[2], "h"), None, osm.EPI_F32, osm._ptr(Ybig, "Y"),
                                                 osm._stream(None)))
     assert e.value.code == osm.ERR_UNSUPPORTED and "static scratch" in str(e.value)
+    # absurd batch sizes are refused before the size arithmetic (whose 64-bit
+    # products would wrap to a small number at M = 2^59 for this plan)
+    for huge in (1 << 59, (1 << 63) - 1, osm.NOALLOC_SCRATCH_BYTES + 1):
+        with pytest.raises(osm.OsmError) as e:
+            osm._check(osm.lib().osm_linear_noalloc(plan.handle, osm._ptr(Xbig, "X"), huge,
+                                                    osm._ptr(wpack[0], "w"), osm._ptr(wpack[1], "s"),
+                                                    osm._ptr(wpack[2], "h"), None, osm.EPI_F32,
+                                                    osm._ptr(Ybig, "Y"), osm._stream(None)))
+        assert e.value.code == osm.ERR_UNSUPPORTED and "static scratch" in str(e.value)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
