@@ -95,11 +95,13 @@ def fmt_config(args, cfg):
     return {"format": "mxfp4", "wscale": WSCALE_NAMES[cfg.wmode]} if hasattr(cfg, "wmode") else {"format": "mxfp4"}
 
 
-def blended_peak(peaks, parts):
+def blended_peak(peaks, parts, sustained: bool = False):
     """Tensor-pipe peak for a mix of FP4 and BF16 MMAs: parts is a list of
-    (fp4_flops, bf16_flops); FP4 runs at the measured BF16 burst x 4 (the
-    nominal dense ratio), BF16 at the measured BF16 burst."""
-    p16 = peaks["bf16_tflops"]
+    (fp4_flops, bf16_flops); FP4 runs at the measured BF16 rate x 4 (the
+    nominal dense ratio), BF16 at the measured BF16 rate -- the burst rate
+    for a kernel timed alone, the sustained (power-capped) rate for a kernel
+    timed inside a long step."""
+    p16 = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     p4 = p16 * FP4_PER_BF16
     f4 = sum(a for a, _ in parts)
     f16 = sum(b for _, b in parts)
@@ -628,8 +630,11 @@ def run_ffn(args, cfg, rank, world, local_rank):
         f_up = L * 2.0 * M * F * D
         f_dn = L * 2.0 * M * D * F
         # the dominant kernel: the up-projection with the fused epilogue
-        peak_up, p16 = blended_peak(peaks, [(2.0 * M * F * up0.Kb, 2.0 * M * F * up0.k)])
-        peak_dn, _ = blended_peak(peaks, [(2.0 * M * D * dn0.Kb, 2.0 * M * D * dn0.k)])
+        # the kernels run back to back for the whole ~10 ms step (and the
+        # clocks settle under the power cap), so the sustained BF16 rate sets
+        # the peak
+        peak_up, p16 = blended_peak(peaks, [(2.0 * M * F * up0.Kb, 2.0 * M * F * up0.k)], sustained=True)
+        peak_dn, _ = blended_peak(peaks, [(2.0 * M * D * dn0.Kb, 2.0 * M * D * dn0.k)], sustained=True)
         ach_up = f_up / up_s / 1e12
         ach_dn = f_dn / down_s / 1e12
         cb, sb, hb = up0.sizes(M)
@@ -659,8 +664,8 @@ def run_ffn(args, cfg, rank, world, local_rank):
                          "frac": ach_up / peak_up, "traffic": traffic, "traffic_unit": "bytes per launch",
                          "kernel": "dual_gemm up-projection, fused GELU + smoothing + MXFP4 requantisation",
                          "pct_fp4_spec_peak": 100.0 * ach_up / FP4_SPEC_TFLOPS,
-                         "peak_source": f"derived from {peak_src} peaks: BF16 burst {p16} TFLOP/s x4 (nominal "
-                                        f"FP4:BF16 dense ratio) for the FP4 share, x1 for the BF16 share "
+                         "peak_source": f"derived from {peak_src} peaks: sustained BF16 {p16} TFLOP/s x4 "
+                                        f"(nominal FP4:BF16 dense ratio) for the FP4 share, x1 for the BF16 share "
                                         f"(k={up0.k} of K={D}); FP4 itself is not measured"},
             "e2e": {"value": world * flops / e2e_s / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": L * M * D * 2, "d2h_bytes_per_step": L * M * D * 2,

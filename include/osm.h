@@ -93,13 +93,11 @@ typedef enum {
 } osm_wscale_mode;
 
 /* Epilogues of osm_dual_gemm. GELU below is the FFN's tanh form,
- * 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated by this
- * library's own FP32 routine (only IEEE round-to-nearest-even adds,
- * multiplies and fused multiply-adds: 0.5 (1 + tanh(u)) = sigma(2u) is
- * 1/(1 + E) for x >= 0 and E/(1 + E) for x < 0, E = exp(-2|u|) by
- * Cody-Waite reduction and a degree-7 Taylor polynomial, the reciprocal by
- * a linear seed and three Newton steps). It stays within 5e-7 |GELU(x)| +
- * 2e-8 |x| of the exact function; a BF16 result adds one rounding. */
+ * 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated in FP32
+ * as x / (1 + 2^z), z = -2 u log2(e), with the power of two and the
+ * reciprocal on the special-function unit (osm_gelu_f32 exposes the
+ * routine). It stays within 5e-7 |GELU(x)| + 2e-8 |x| of the exact
+ * function; a BF16 result adds one rounding. */
 typedef enum {
     OSM_EPI_F32 = 0,          /* Y [M][N] float32                                     */
     OSM_EPI_BF16 = 1,         /* Y [M][N] BF16 (RNE of the FP32 accumulator)          */
@@ -310,6 +308,12 @@ OSM_API int osm_plan_tables(const osm_plan* plan, float* s_host, float* inv_s_ho
  * sum (Y - Yref)^2 and sum Yref^2 over `count` FP32 values, accumulated in
  * FP64 (the summation order varies between runs in the last bits). */
 OSM_API int osm_error_norms(const float* Y, const float* Yref, int64_t count, double* out, void* stream);
+
+/* The FP32 GELU routine of the FFN epilogues (OSM_EPI_GELU_BF16 and
+ * OSM_EPI_GELU_REQUANT) applied element-wise: y[i] = GELU(x[i]) with exactly
+ * the epilogues' arithmetic, so that tests can hold the routine to the exact
+ * function. x, y: device float[n], n >= 1. */
+OSM_API int osm_gelu_f32(const float* x, float* y, int64_t n, void* stream);
 
 /* ---- runtime activation path ----------------------------------------------
  * "activations are divided in-place by s, quantized ..., and routed through

@@ -64,6 +64,7 @@ _SIGNATURES = {
     "osm_linear_host": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "osm_scales_to_logical": (_I, [_P, _I64, _I64, _P]),
     "osm_linear_noalloc": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _P]),
+    "osm_gelu_f32": (_I, [_P, _P, _I64, _P]),
     "osm_ffn_workspace_size": (_SZ, [_P, _P, _I64]),
     "osm_ffn_host_workspace_size": (_SZ, [_P, _P, _I64]),
     "osm_ffn_block": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -289,6 +290,17 @@ def error_norms(Y, Yref, stream=None):
                                  _ptr(out, "out", (torch.float64,)), _stream(stream)))
     e, n = out.cpu().tolist()
     return e, n
+
+
+def gelu_f32(x, y=None, stream=None):
+    """The FFN epilogues' FP32 GELU routine element-wise (osm_gelu_f32)."""
+    import torch
+    if y is None:
+        y = torch.empty_like(x)
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be float32 tensors of one size")
+    _check(lib().osm_gelu_f32(_ptr(x, "x"), _ptr(y, "y"), x.numel(), _stream(stream)))
+    return y
 
 
 def weight_amax(W, wmax, stream=None):

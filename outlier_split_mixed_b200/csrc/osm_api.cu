@@ -452,6 +452,15 @@ int osm_error_norms(const float* Y, const float* Yref, int64_t count, double* ou
     return launch_error_norms(Y, Yref, count, out, static_cast<cudaStream_t>(stream));
 }
 
+int osm_gelu_f32(const float* x, float* y, int64_t n, void* stream) {
+    g_err[0] = 0;
+    OSM_REQUIRE(n >= 1, "gelu_f32: n must be >= 1");
+    OSM_REQUIRE(x && y && (reinterpret_cast<uintptr_t>(x) & 3) == 0 && (reinterpret_cast<uintptr_t>(y) & 3) == 0,
+                "gelu_f32: null or misaligned pointer");
+    OSM_TRY(check_device());
+    return launch_gelu_f32(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 int osm_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* a_codes, uint8_t* a_scales,
                      uint16_t* a_hp, void* stream) {
     g_err[0] = 0;

@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -80,7 +81,13 @@ static_assert(LAUNCH_REGS * 3 <= 512 && CTRL_REGS % 8 == 0 && EPI_REGS % 8 == 0,
 __host__ __device__ constexpr bool uses_register_split(int epi) { return epi == OSM_EPI_GELU_REQUANT; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;       // scale factors live after the accumulator
-constexpr int GROUP_M = 8;              // raster: 8 M-tiles sweep the N-tiles together
+// Tile raster. When the packed weights fit comfortably in L2 (the FFN
+// projections: about 40 MB), every M-tile sweeps all N-tiles before the next
+// (group of 1): all of W stays resident and each activation tile is read
+// from HBM once. Larger weights use groups of GROUP_M M-tiles, which bound
+// the weight bytes streamed per group.
+constexpr int GROUP_M = 8;
+constexpr int64_t W_RESIDENT_BYTES = 48ll << 20;
 constexpr uint16_t PAIR_MASK = 0x3;
 
 // Ring shape per 4-bit format. A slot carries one K-step of 256 FP4 values;
@@ -148,6 +155,7 @@ struct GemmParams {
     int n_fp4;       // K-steps of the bulk branch: ceil(Kbp / 256)
     int n_hp;        // K-steps of the outlier branch: kp / 64
     int num_m, num_n;
+    int group_m;     // tile raster: groups of group_m M-tiles sweep the N-tiles (M fastest inside a group)
     int n_row_tiles; // ceil(N / 128): scale-atom rows of W
     int epi;
     uint32_t idesc_hp;        // instruction descriptor of the outlier K-steps (BF16 or FP16 operands)
@@ -162,11 +170,11 @@ struct GemmParams {
     int64_t m_pad;            // M rounded up to 128 (rows of next_scales)
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
-    const int group = GROUP_M * num_n;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& m_blk, int& n_blk) {
+    const int group = group_m * num_n;
     const int g = tile / group;
-    const int first_m = g * GROUP_M;
-    const int gm = min(num_m - first_m, GROUP_M);
+    const int first_m = g * group_m;
+    const int gm = min(num_m - first_m, group_m);
     const int local = tile % group;
     m_blk = first_m + local % gm;
     n_blk = local / gm;
@@ -232,8 +240,8 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
             b = __fadd2_rn(b, bb);
         }
         if constexpr (EPI == OSM_EPI_GELU_BF16) {
-            a = mx::gelu_tanh2(a);
-            b = mx::gelu_tanh2(b);
+            a = mx::gelu2(a);
+            b = mx::gelu2(b);
         }
         if constexpr (EPI == OSM_EPI_F32) {
             if (ra < p.M) *reinterpret_cast<float2*>(static_cast<float*>(p.Y) + ra * p.N + col) = a;
@@ -286,8 +294,8 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float4 sv = __ldg(iv + i);
-        const float2 g0 = mx::gelu_tanh2(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])));
-        const float2 g1 = mx::gelu_tanh2(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+        const float2 g0 = mx::gelu2(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])));
+        const float2 g1 = mx::gelu2(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
         const uint32_t h0 = mx::bf16x2_bits(g0.x, g0.y), h1 = mx::bf16x2_bits(g1.x, g1.y);
         const float2 x0 = __fmul2_rn(make_float2(__uint_as_float(h0 << 16), __uint_as_float(h0 & 0xFFFF0000u)),
                                      make_float2(sv.x, sv.y));
@@ -304,19 +312,29 @@ __device__ __forceinline__ void requant_group(const GemmParams& p, int64_t row, 
         }
     }
     if (c0 < p.nKb) {
-        const int nreal = static_cast<int>(p.nKb - c0 < 32 ? p.nKb - c0 : 32);
         uint32_t bw[16];
-        uint32_t m = 0;
+        if (p.nKb - c0 >= 32) {  // a whole bulk block (the same for every lane of the warp)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t lo = (2 * i < nreal) ? (hw[i] & 0xFFFFu) : 0u;
-            const uint32_t hi = (2 * i + 1 < nreal) ? (hw[i] & 0xFFFF0000u) : 0u;
-            bw[i] = lo | hi;
-            const uint32_t a = bw[i] & 0x7FFF7FFFu;
-            m = max(m, max(a & 0xFFFFu, a >> 16));
+            for (int i = 0; i < 16; ++i) bw[i] = hw[i];
+        } else {                 // the last, partial block: positions >= nKb are padding (0)
+            const int nreal = static_cast<int>(p.nKb - c0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t lo = (2 * i < nreal) ? (hw[i] & 0xFFFFu) : 0u;
+                const uint32_t hi = (2 * i + 1 < nreal) ? (hw[i] & 0xFFFF0000u) : 0u;
+                bw[i] = lo | hi;
+            }
         }
-        const int X = mx::exponent(mx::bf16_bits_to_f32(m));
-        const float inv = mx::exp2_neg(X);
+        // block maximum of |x'| by a tree of packed BF16 abs-max (sign bits cleared after)
+        uint32_t t8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t8[i] = mx::bf16x2_absmax(bw[2 * i], bw[2 * i + 1]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t8[i] = mx::bf16x2_absmax(t8[2 * i], t8[2 * i + 1]);
+        t8[0] = mx::bf16x2_absmax(mx::bf16x2_absmax(t8[0], t8[1]), mx::bf16x2_absmax(t8[2], t8[3]));
+        const uint32_t amax = max(t8[0] & 0x7FFFu, (t8[0] >> 16) & 0x7FFFu);
+        float inv;
+        const int X = mx::bf16_block_exponent(amax, &inv);
         const uint4 out = make_uint4(mx::encode8_words(bw[0], bw[1], bw[2], bw[3], inv),
                                      mx::encode8_words(bw[4], bw[5], bw[6], bw[7], inv),
                                      mx::encode8_words(bw[8], bw[9], bw[10], bw[11], inv),
@@ -372,7 +390,7 @@ __device__ __forceinline__ void producer_role(const GemmParams& p, Smem<NV>& S, 
         bool ok = true;
         for (int tile = pair; tile < tiles && ok; tile += npairs) {
             int m_blk, n_blk;
-            tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
+            tile_coords(tile, p.num_m, p.num_n, p.group_m, m_blk, n_blk);
             const int arow = m_blk * 2 * BM + static_cast<int>(rank) * BM;        // this CTA's A rows
             const int brow = n_blk * BN + static_cast<int>(rank) * (BN / 2);      // this CTA's B rows
             const int nbt = min(2, p.n_row_tiles - 2 * n_blk);                   // valid B scale row tiles
@@ -511,7 +529,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem<NV>& S, 
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < tiles; tile += npairs) {
         int m_blk, n_blk;
-        tile_coords(tile, p.num_m, p.num_n, m_blk, n_blk);
+        tile_coords(tile, p.num_m, p.num_n, p.group_m, m_blk, n_blk);
         int ok = 1;
         if (lane == 0)
             ok = ptx::mbar_wait_bounded(ptx::smem_u32(&S.acc_full), acc_phase, p.wait_limit_ns, abort) ? 1 : 0;
@@ -674,8 +692,25 @@ struct LaunchInfo {
     bool ready = false;
 };
 
+// The epilogues' GELU routine applied element-wise (a test hook for its
+// accuracy): y[i] = GELU(x[i]) exactly as the FFN epilogues compute it.
+__global__ void gelu_f32_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x * 2) {
+        const float2 v = mx::gelu2(make_float2(x[i], i + 1 < n ? x[i + 1] : 0.0f));
+        y[i] = v.x;
+        if (i + 1 < n) y[i + 1] = v.y;
+    }
+}
+
 }  // namespace
 
+
+int launch_gelu_f32(const float* x, float* y, int64_t n, cudaStream_t st) {
+    const int64_t blocks = std::min<int64_t>((n + 511) / 512, 148 * 8);
+    gelu_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, y, n);
+    return check_cuda(cudaGetLastError(), "gelu_f32 launch");
+}
 
 int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* a_scales, const uint16_t* a_hp,
                      int64_t M, const uint8_t* w_codes, const uint8_t* w_scales, const uint16_t* w_hp,
@@ -726,6 +761,11 @@ int launch_dual_gemm(const osm_plan* pl, const uint8_t* a_codes, const uint8_t* 
     p.n_hp = static_cast<int>(pl->kp / 64);
     p.num_m = static_cast<int>(ceil_div(M, 2 * BM));
     p.num_n = static_cast<int>(ceil_div(pl->N, BN));
+    {
+        size_t wc = 0, ws = 0, wh = 0;
+        osm_plan_sizes(pl, pl->N, &wc, &ws, &wh);
+        p.group_m = static_cast<int64_t>(wc + ws + wh) <= W_RESIDENT_BYTES ? 1 : GROUP_M;
+    }
     p.n_row_tiles = static_cast<int>(ceil_div(pl->N, 128));
     p.epi = epi;
     p.idesc_hp = pl->hp_fp16 ? IDESC_F16 : IDESC_BF16;

@@ -68,6 +68,7 @@ int launch_pack_weights(const osm_plan* p, const uint16_t* W, const int32_t* col
 int launch_plan_refresh(osm_plan* p, const float* amax, const float* score, const float* wmax, float alpha,
                         cudaStream_t st);
 int launch_error_norms(const float* y, const float* r, int64_t count, double* out, cudaStream_t st);
+int launch_gelu_f32(const float* x, float* y, int64_t n, cudaStream_t st);
 int launch_quantize_act(const osm_plan* p, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st);
 int launch_dual_gemm(const osm_plan* p, const uint8_t* a_codes, const uint8_t* a_scales,

@@ -121,7 +121,7 @@ def test_ffn_block_end_to_end(layer):
     g_h_scales_full = unswizzle(h_dn[1].cpu().numpy(), M, down.Kbp // 32)
     g_h_hp = to_np_u16(h_dn[2].view(M, down.kp)[Rd])
     g_H = to_np_u16(H[Rd])
-    g_Y = Yh.numpy().view(np.uint16)[R]
+    g_Y = Yh.view(torch.int16).numpy().view(np.uint16)[R]
     g_wu = (wu[0].cpu().numpy().reshape(F, up.Kbp // 2), unswizzle(wu[1].cpu().numpy(), F, up.Kbp // 32),
             to_np_u16(wu[2]).reshape(F, up.kp))
     g_wd = (wd[0].cpu().numpy().reshape(D, down.Kbp // 2), unswizzle(wd[1].cpu().numpy(), D, down.Kbp // 32),
