@@ -71,12 +71,13 @@ WSCALE_NAMES = {0: "1x32", 1: "32x32", 2: "128x1"}
 E2E_STREAMS = 3
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one dual_gemm
-# launch, from one ncu capture of the current kernel on the workload, per
-# (workload, bulk format); a workload without a capture of the current
-# kernel reports null.
-# (The last captures, 270.3 MB for MXFP4 and 276.1 MB for NVFP4 on the
-# 4096-token up-projection, predate dual_gemm's dependent-launch prologue.)
-DUAL_GEMM_TRAFFIC = {}
+# launch, from one ncu capture of the current kernel on the full-size
+# workload (one pass), per (workload, kernel); a workload or kernel without a
+# capture of the current code reports null.
+DUAL_GEMM_TRAFFIC = {
+    ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 377.87e6,
+    ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 708.12e6,
+}
 
 
 def workload_config(cfg):
@@ -640,6 +641,12 @@ def run_ffn(args, cfg, rank, world, local_rank):
         cb, sb, hb = up0.sizes(M)
         q_bytes = L * (M * D * 2 + cb + sb + hb)
         traffic = None if args.hp_fp16 else DUAL_GEMM_TRAFFIC.get((cfg.name, "up_gelu_requant"))
+        # algorithmic bytes of one launch: packed activations in, packed weights, output out
+        cd_, sd_, hd_ = dn0.sizes(M)
+        cwu, swu, hwu = up0.sizes(F)
+        cwd, swd, hwd = dn0.sizes(D)
+        alg_up = (cb + sb + hb) + (cwu + swu + hwu) + (cd_ + sd_ + hd_)
+        alg_dn = (cd_ + sd_ + hd_) + (cwd + swd + hwd) + M * D * 2
         line = {
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n, "warmup": args.warmup,
@@ -656,12 +663,14 @@ def run_ffn(args, cfg, rank, world, local_rank):
                 "dual_gemm_down_bf16": {"ms": down_s * 1e3, "tflops": ach_dn, "frac": ach_dn / peak_dn,
                                         "pct_fp4_spec_peak": 100.0 * ach_dn / FP4_SPEC_TFLOPS,
                                         "traffic": None if args.hp_fp16 else
-                                        DUAL_GEMM_TRAFFIC.get((cfg.name, "down_bf16"))},
+                                        DUAL_GEMM_TRAFFIC.get((cfg.name, "down_bf16")),
+                                        "algorithmic_bytes": alg_dn},
                 "quantize_act": {"ms": quant_s * 1e3, "gbs": q_bytes / quant_s / 1e9, "bytes": q_bytes,
                                  "frac_hbm": q_bytes / quant_s / 1e9 / peaks["hbm_gbs"]},
             },
             "roofline": {"bound": "tensor", "achieved": ach_up, "peak": peak_up, "unit": "TFLOP/s",
                          "frac": ach_up / peak_up, "traffic": traffic, "traffic_unit": "bytes per launch",
+                         "algorithmic_bytes": alg_up,
                          "kernel": "dual_gemm up-projection, fused GELU + smoothing + MXFP4 requantisation",
                          "pct_fp4_spec_peak": 100.0 * ach_up / FP4_SPEC_TFLOPS,
                          "peak_source": f"derived from {peak_src} peaks: sustained BF16 {p16} TFLOP/s x4 "

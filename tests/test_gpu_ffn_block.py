@@ -28,9 +28,10 @@ pinned host memory):
     down-projection's BF16 output within 1e-5 sum|a w| + 1e-6 + 2^-8 |y| of
     the oracle's FP64 product of those codes;
   * the oracle's own chain (its own BF16 GELU, requantisation and product)
-    agrees with the GPU's Y to a small relative error, since the two chains
-    differ only where a hidden activation rounds to a neighbouring BF16
-    value.
+    agrees with the chain through the GPU's hidden activations to 1e-4
+    (relative Frobenius norm): the two differ only where a hidden activation
+    rounds to a neighbouring BF16 value; the GPU's BF16 Y lies within the
+    BF16 output rounding (~1.6e-3 RMS) of the oracle's own chain.
 """
 import numpy as np
 import pytest
@@ -194,11 +195,17 @@ def test_ffn_block_end_to_end(layer):
     Yg = _bf16_f64(g_Y)
     assert_y_close(Yg, y_dn, T_dn, bf16=True)
 
-    # the oracle's own chain end to end
+    # the oracle's own chain end to end: it differs from the product above
+    # only where a hidden activation rounds to the neighbouring BF16 value
+    # (FP32 against FP64 sums, the FP32 GELU routine against FP64), which
+    # moves Y far less than the BF16 rounding of Y itself (~1.6e-3 RMS)
     c_o = oracle.quantize_act(oracle.gelu_bf16(y_up), invo_d, Oo_d)
     y_chain, _ = oracle.dual_gemm_rows(*c_o, r, *wd_o)
-    rel = float(np.linalg.norm(Yg - y_chain) / np.linalg.norm(y_chain))
+    rel_chain = float(np.linalg.norm(y_dn - y_chain) / np.linalg.norm(y_chain))
+    rel_gpu = float(np.linalg.norm(Yg - y_chain) / np.linalg.norm(y_chain))
     flips = int(np.sum(g_H != oracle.gelu_bf16(y_up)))
-    print(f"block {layer}: relative error of Y against the oracle's own chain {rel:.2e}; "
-          f"{flips} of {g_H.size} hidden activations round to a neighbouring BF16 value")
-    assert rel <= 1e-3
+    print(f"block {layer}: {flips} of {g_H.size} hidden activations round to a neighbouring BF16 value; "
+          f"relative difference of the two FP64 chains {rel_chain:.2e}; GPU Y (BF16) against the oracle's "
+          f"own chain {rel_gpu:.2e}")
+    assert rel_chain <= 1e-4
+    assert rel_gpu <= 2.5e-3
