@@ -9,7 +9,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <algorithm>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -469,8 +468,6 @@ struct QuantParams {
     float nv_k;              // NVFP4: fp32(1/6) * 2^-g_act
     float nv_p2g;            // NVFP4: 2^g_act
     float hp_scale;          // NVFP4: 2^-g_act on the outlier slots
-    const int32_t* J;        // [Kb] bulk position -> channel (the gather form)
-    const int32_t* O;        // [k]  outlier slot -> channel
 };
 
 // Encodings of quantize_act: MXFP4 with BF16 or FP16 outlier slots, NVFP4.
@@ -784,226 +781,6 @@ __global__ void __launch_bounds__(NT, (TR > 6 ? 1 : 2)) quantize_act_stream_kern
     }
 }
 
-// The gather form (MXFP4 with BF16 or FP16 outlier slots, rows of up to
-// 16383 channels). Each 32-value block of a row's packed output -- a bulk
-// block b (positions 32b .. 32b+31 of the compacted bulk index) or an
-// outlier group g (slots 32g .. 32g+31) -- is an item handled by a quad of
-// four lanes, eight values per lane; the items of a row are spread over
-// the quads of the CTA (IT items per quad), and every quad handles its
-// items for every row the CTA takes. Per lane, the source channel of each
-// of its eight values and that channel's inv_s are looked up once, at kernel
-// start, and kept in registers (channel offsets as packed 16-bit words), so
-// a row costs per value one 16-bit shared load of the raw row, one packed
-// FP32 multiply and one packed conversion to BF16; per block a tree of
-// packed BF16 abs-max (two shuffles across the quad), the MX exponent from
-// the BF16 exponent field, two packed multiplies and conversions to E2M1
-// per lane, and a 4x4 byte transpose across the quad (two shuffles and two
-// byte permutes) so that each lane stores 4 contiguous code bytes.
-// Rows arrive in stages of R rows by one bulk asynchronous copy per row into
-// a ring of S stages (row slots of 2K + 16 bytes: the 16-byte tail stays
-// zero and is the source of every padding position). A dedicated producer
-// warp issues the copies; full[s] completes when a stage's rows have
-// landed, empty[s] when every consumer warp is done with it -- no block-wide
-// barrier on the data path. Bank use: lane l of quad q in a warp reads, at
-// its load j, the pair of positions 2l + 8c, c = (j + q/2) % 4, of its block;
-// consecutive quads take consecutive blocks (64 bytes apart), so the 32
-// lanes of a load touch 32 distinct banks when no outlier shifts them.
-// Every wait is bounded; a wait that runs out sets OSM_STATUS_TIMEOUT and an
-// abort flag, and the producer lets every copy it issued land before the
-// CTA exits.
-constexpr int GQ_MAX_K = 16383;      // channel byte offsets fit 16 bits
-// Largest CTA per items-per-quad count, so that the per-lane tables (about
-// 14 registers per item) and the working set fit without spilling.
-__host__ __device__ constexpr int gq_max_threads(int it) { return it == 1 ? 768 : (it == 2 ? 640 : 512); }
-
-template <int IT, int MODE>
-__global__ void __launch_bounds__(gq_max_threads(IT), 1) quantize_act_gather_kernel(QuantParams p, int R, int S) {
-    static_assert(MODE == QA_MX || MODE == QA_MX_F16, "the gather form encodes MXFP4");
-    ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int nw = static_cast<int>(blockDim.x >> 5) - 1;  // consumer warps; warp nw is the producer
-    const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
-    const uint32_t row_slot = 2u * static_cast<uint32_t>(p.K) + 16u;
-    const uint32_t stage_bytes = static_cast<uint32_t>(R) * row_slot;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
-    uint64_t* empty = full + S;
-    __shared__ int abort_flag;
-    __shared__ int never;  // a flag nothing sets
-    const int ngroups = (p.M + R - 1) / R;
-    const int mine = static_cast<int>(blockIdx.x) < ngroups
-                         ? (ngroups - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                         : 0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
-            ptx::mbar_init(ptx::smem_u32(&empty[s]), static_cast<uint32_t>(nw));
-        }
-        abort_flag = 0;
-        never = 0;
-        ptx::fence_mbar_init();
-    }
-    // zero tails of every row slot (the copies never write them)
-    for (int i = static_cast<int>(threadIdx.x); i < S * R; i += static_cast<int>(blockDim.x))
-        *reinterpret_cast<uint4*>(smem + static_cast<size_t>(i) * row_slot + 2u * p.K) = make_uint4(0, 0, 0, 0);
-    if (blockIdx.x == 0) zero_padding_scale_rows(p);
-    __syncthreads();
-
-    if (warp == nw) {
-        // ---------------------------------------------------------- producer
-        if (lane == 0) {
-            int issued = 0;
-            bool ok = true;
-            for (int i = 0; i < mine; ++i) {
-                const int s = i % S;
-                if (i >= S &&
-                    !ptx::mbar_wait_bounded(ptx::smem_u32(&empty[s]), static_cast<uint32_t>((i / S - 1) & 1),
-                                            p.wait_limit_ns, &abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const int g = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
-                const int rows = min(R, p.M - g * R);
-                const uint32_t bar = ptx::smem_u32(&full[s]);
-                ptx::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * 2u * p.K + p.extra_tx);
-                for (int r = 0; r < rows; ++r)
-                    ptx::bulk_load(ptx::smem_u32(smem + static_cast<size_t>(s) * stage_bytes + r * row_slot),
-                                   p.X + (static_cast<size_t>(g) * R + r) * p.K, 2u * p.K, bar);
-                issued = i + 1;
-            }
-            if (!ok) {
-                atomicOr(p.status, OSM_STATUS_TIMEOUT);
-                abort_flag = 1;
-            }
-            // Before the CTA exits, every copy issued must have landed: the
-            // latest stage of each slot is the only one whose completion is
-            // not already implied by an earlier wait.
-            for (int j = max(0, issued - S); j < issued; ++j)
-                if (!ptx::mbar_wait_bounded(ptx::smem_u32(&full[j % S]), static_cast<uint32_t>((j / S) & 1),
-                                            20000000ull, &never))
-                    ptx::spin_ns(1000000);
-        }
-        return;
-    }
-
-    // -------------------------------------------------------------- consumers
-    const int l = lane & 3;
-    const int qw = lane >> 2;                 // quad within the warp
-    const int quad = warp * 8 + qw;
-    const int Q = nw * 8;
-    const int nb = p.Kbp >> 5, ng = p.kp >> 5, nitems = nb + ng;
-    const int rot = qw >> 1;                  // load j takes column c = (j + rot) % 4
-    // per item: channel byte offsets of the lane's 8 values (load j: values
-    // 2j, 2j+1 in the low / high half), their inv_s, the item
-    uint32_t off[IT][4];
-    float2 isv[IT][4];
-    int item[IT];
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-        item[it] = quad + it * Q;
-        const bool bulk = item[it] < nb, outl = !bulk && item[it] < nitems;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = (j + rot) & 3;
-            uint32_t o2 = 0;
-            float iv[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int e = 2 * l + 8 * c + h;  // position within the item
-                int ch = -1;
-                if (bulk) {
-                    const int pos = 32 * item[it] + e;
-                    if (pos < p.Kb) ch = __ldg(p.J + pos);
-                } else if (outl) {
-                    const int slot = 32 * (item[it] - nb) + e;
-                    if (slot < p.k) ch = __ldg(p.O + slot);
-                }
-                const uint32_t o = ch >= 0 ? 2u * static_cast<uint32_t>(ch) : 2u * static_cast<uint32_t>(p.K);
-                o2 |= o << (16 * h);
-                iv[h] = ch >= 0 ? __ldg(p.inv_s + ch) : 0.0f;
-            }
-            off[it][j] = o2;
-            isv[it][j] = make_float2(iv[0], iv[1]);
-        }
-    }
-    // byte permutes: rotate the code bytes (load order) into column order,
-    // then the 4x4 transpose across the quad
-    const uint32_t rot_sel = (((0 - rot) & 3)) | (((1 - rot) & 3) << 4) | (((2 - rot) & 3) << 8) |
-                             (((3 - rot) & 3) << 12);
-    const uint32_t sel1 = (l & 2) ? 0x3276u : 0x5410u;
-    const uint32_t sel2 = (l & 1) ? 0x3715u : 0x6240u;
-    const int katoms = p.katoms;
-    const uint32_t smem0 = ptx::smem_u32(smem);
-
-    for (int i = 0; i < mine; ++i) {
-        const int s = i % S;
-        const int g = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
-        const int rows = min(R, p.M - g * R);
-        int ok = 1;
-        if (lane == 0)
-            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&full[s]), static_cast<uint32_t>((i / S) & 1), p.wait_limit_ns,
-                                        &abort_flag)
-                     ? 1
-                     : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-            if (lane == 0) {
-                atomicOr(p.status, OSM_STATUS_TIMEOUT);
-                abort_flag = 1;
-            }
-            break;
-        }
-        for (int r = 0; r < rows; ++r) {
-            const int t = g * R + r;
-            const uint32_t rb = smem0 + s * stage_bytes + r * row_slot;
-            uint8_t* const codes_row = p.codes + static_cast<size_t>(t) * (p.Kbp >> 1);
-            uint16_t* const hp_row = p.hp + static_cast<size_t>(t) * p.kp;
-            const int64_t sf_t = ((t >> 7) * static_cast<int64_t>(katoms)) * 512 + (t & 31) * 16 + ((t >> 5) & 3) * 4;
-#pragma unroll
-            for (int it = 0; it < IT; ++it) {
-                // Every lane runs the whole sequence (the shuffles need the
-                // full warp); only the stores depend on the item's kind. An
-                // item past the last reads the zero tails.
-                const bool is_bulk = item[it] < nb, is_out = !is_bulk && item[it] < nitems;
-                uint32_t q[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t h0 = ptx::ld_shared_u16(rb + (off[it][j] & 0xFFFFu));
-                    const uint32_t h1 = ptx::ld_shared_u16(rb + (off[it][j] >> 16));
-                    const float2 v = __fmul2_rn(make_float2(__uint_as_float(h0 << 16), __uint_as_float(h1 << 16)),
-                                                isv[it][j]);
-                    q[j] = (MODE == QA_MX_F16 && is_out) ? mx::f16x2_bits(v.x, v.y) : mx::bf16x2_bits(v.x, v.y);
-                }
-                uint32_t m = mx::bf16x2_absmax(mx::bf16x2_absmax(q[0], q[1]), mx::bf16x2_absmax(q[2], q[3]));
-                m = mx::bf16x2_absmax(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                m = mx::bf16x2_absmax(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                const uint32_t amax = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
-                float inv;
-                const int X = mx::bf16_block_exponent(amax, &inv);
-                // byte j of w: the codes of the lane's values 2j, 2j+1 (column (j + rot) % 4)
-                uint32_t w = mx::encode8_words(q[0], q[1], q[2], q[3], inv);
-                w = __byte_perm(w, 0, rot_sel);                                 // byte c: code byte l + 4c
-                w = __byte_perm(w, __shfl_xor_sync(0xffffffffu, w, 2), sel1);
-                w = __byte_perm(w, __shfl_xor_sync(0xffffffffu, w, 1), sel2);  // code bytes 4l .. 4l+3
-                if (is_bulk) {
-                    const int b = item[it];
-                    *reinterpret_cast<uint32_t*>(codes_row + 16 * b + 4 * l) = w;
-                    if (l == 0)
-                        p.scales[sf_t + (b >> 2) * 512 + (b & 3)] = static_cast<uint8_t>(X + 127);
-                } else if (is_out) {
-                    // outlier slots 2l + 8c (+1) of the group: 32-bit word l + 4c of its 64 bytes
-                    uint16_t* const dst = hp_row + 32 * (item[it] - nb) + 2 * l;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint32_t*>(dst + 8 * ((j + rot) & 3)) = q[j];
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
-    }
-}
-
 template <int R, int S>
 size_t stream_smem_bytes(int K, int stride) {
     return static_cast<size_t>(S) * R * K * 2 + static_cast<size_t>(R) * stride + 8 * S;
@@ -1125,31 +902,6 @@ static int launch_stream(const QuantParams& p, int mode, int stride, cudaStream_
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
-// The gather form for IT items per quad; returns 1 (nothing launched) when
-// the CTA it needs does not fit.
-template <int IT>
-static int launch_gather(const QuantParams& p, int mode, int nitems, cudaStream_t st, int* launched) {
-    *launched = 0;
-    const int nw = (nitems + 8 * IT - 1) / (8 * IT);
-    const int threads = 32 * (nw + 1);
-    if (threads > gq_max_threads(IT)) return OSM_OK;
-    const size_t row_slot = 2 * static_cast<size_t>(p.K) + 16;
-    const int R = static_cast<int>(std::max<size_t>(1, std::min<size_t>(16, (48 * 1024) / row_slot)));
-    const int S = static_cast<int>(std::max<size_t>(2, std::min<size_t>(6, (200 * 1024) / (R * row_slot))));
-    const size_t smem = static_cast<size_t>(S) * R * row_slot + 16 * static_cast<size_t>(S);
-    if (smem > 220 * 1024) return OSM_OK;
-    auto kern = mode == QA_MX_F16 ? quantize_act_gather_kernel<IT, QA_MX_F16> : quantize_act_gather_kernel<IT, QA_MX>;
-    int per_sm = 0, sms = 0;
-    int rc = prepare_kernel(reinterpret_cast<const void*>(kern), threads, smem, &per_sm, &sms);
-    if (rc) return rc;
-    if (per_sm < 1) return OSM_OK;
-    const int64_t groups = ceil_div(p.M, R);
-    const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(sms) * per_sm);
-    kern<<<static_cast<unsigned>(grid), threads, smem, st>>>(p, R, S);
-    *launched = 1;
-    return check_cuda(cudaGetLastError(), "quantize_act launch");
-}
-
 int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st) {
     if (M > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: M too large");
@@ -1158,17 +910,8 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
                   static_cast<int>(pl->kp), codes, scales, hp, pl->d_status, pl->wait_limit_ns,
                   (pl->debug_flags & OSM_DEBUG_STARVE_QUANTIZE) ? 16u : 0u, pl->hp_fp16,
                   static_cast<int>(pl->Kbp / (4 * block_elems(pl->fmt))), nvfp4_k(pl->g_act), pow2f(pl->g_act),
-                  pow2f(-pl->g_act), pl->d_J, pl->d_O};
+                  pow2f(-pl->g_act)};
     const int mode = pl->fmt == OSM_FMT_NVFP4 ? QA_NV : (pl->hp_fp16 ? QA_MX_F16 : QA_MX);
-    // MXFP4 rows of up to GQ_MAX_K channels: the gather form
-    if (mode != QA_NV && p.K <= GQ_MAX_K) {
-        const int nitems = static_cast<int>(pl->Kbp / 32 + pl->kp / 32);
-        int launched = 0, rc;
-        if ((rc = launch_gather<1>(p, mode, nitems, st, &launched)) || launched) return rc;
-        if ((rc = launch_gather<2>(p, mode, nitems, st, &launched)) || launched) return rc;
-        if ((rc = launch_gather<3>(p, mode, nitems, st, &launched)) || launched) return rc;
-        if ((rc = launch_gather<4>(p, mode, nitems, st, &launched)) || launched) return rc;
-    }
     const int stride = qa_row_stride(static_cast<int>(pl->Kbp / 32), static_cast<int>(pl->kp));
     // streaming form: two CTAs of at most 110 KB per SM
     const size_t two_per_sm = 110 * 1024;

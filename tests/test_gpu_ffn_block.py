@@ -28,10 +28,11 @@ pinned host memory):
     down-projection's BF16 output within 1e-5 sum|a w| + 1e-6 + 2^-8 |y| of
     the oracle's FP64 product of those codes;
   * the oracle's own chain (its own BF16 GELU, requantisation and product)
-    agrees with the chain through the GPU's hidden activations to 1e-4
-    (relative Frobenius norm): the two differ only where a hidden activation
-    rounds to a neighbouring BF16 value; the GPU's BF16 Y lies within the
-    BF16 output rounding (~1.6e-3 RMS) of the oracle's own chain.
+    differs from the chain through the GPU's hidden activations only in the
+    MX blocks and outlier slots that hold a hidden activation rounded to the
+    neighbouring BF16 value, and rows without one give identical products;
+    the GPU's BF16 Y lies within the BF16 output rounding (~1.6e-3 RMS) of
+    the oracle's own chain.
 """
 import numpy as np
 import pytest
@@ -195,17 +196,31 @@ def test_ffn_block_end_to_end(layer):
     Yg = _bf16_f64(g_Y)
     assert_y_close(Yg, y_dn, T_dn, bf16=True)
 
-    # the oracle's own chain end to end: it differs from the product above
-    # only where a hidden activation rounds to the neighbouring BF16 value
-    # (FP32 against FP64 sums, the FP32 GELU routine against FP64), which
-    # moves Y far less than the BF16 rounding of Y itself (~1.6e-3 RMS)
-    c_o = oracle.quantize_act(oracle.gelu_bf16(y_up), invo_d, Oo_d)
+    # The oracle's own chain (its own BF16 GELU, requantisation and product)
+    # differs from the chain through the GPU's hidden activations only where
+    # a hidden activation rounds to the neighbouring BF16 value (FP32 against
+    # FP64 sums, the FP32 GELU routine against FP64): only the MX blocks and
+    # outlier slots holding such a value may encode differently, and the
+    # products of rows without one are identical.
+    H_own = oracle.gelu_bf16(y_up)
+    flip = g_H != H_own                                  # [rows][F], natural channel order
+    c_o = oracle.quantize_act(H_own, invo_d, Oo_d)
+    J_d = np.setdiff1d(np.arange(F), Oo_d)
+    nb_d = down.Kbp // 32
+    fb = np.zeros((len(R), nb_d), bool)                  # blocks holding a flipped value
+    fpos = flip[:, J_d]
+    fb[:, :(fpos.shape[1] + 31) // 32] = np.pad(fpos, ((0, 0), (0, (-fpos.shape[1]) % 32))).reshape(
+        len(R), -1, 32).any(axis=2)
+    code_diff = (c_o[0] != h_o[0]).reshape(len(R), nb_d, 16).any(axis=2) | (c_o[1] != h_o[1])
+    assert not (code_diff & ~fb).any(), "a block without a flipped value encodes differently"
+    slot_diff = c_o[2][:, :len(Oo_d)] != h_o[2][:, :len(Oo_d)]
+    assert not (slot_diff & ~flip[:, Oo_d]).any(), "an outlier slot without a flipped value differs"
     y_chain, _ = oracle.dual_gemm_rows(*c_o, r, *wd_o)
+    clean = ~flip.any(axis=1)
+    assert np.array_equal(y_dn[clean], y_chain[clean])
     rel_chain = float(np.linalg.norm(y_dn - y_chain) / np.linalg.norm(y_chain))
     rel_gpu = float(np.linalg.norm(Yg - y_chain) / np.linalg.norm(y_chain))
-    flips = int(np.sum(g_H != oracle.gelu_bf16(y_up)))
-    print(f"block {layer}: {flips} of {g_H.size} hidden activations round to a neighbouring BF16 value; "
-          f"relative difference of the two FP64 chains {rel_chain:.2e}; GPU Y (BF16) against the oracle's "
-          f"own chain {rel_gpu:.2e}")
-    assert rel_chain <= 1e-4
+    print(f"block {layer}: {int(flip.sum())} of {flip.size} hidden activations round to a neighbouring BF16 "
+          f"value ({int(code_diff.sum())} MX blocks re-encoded); relative difference of the two FP64 chains "
+          f"{rel_chain:.2e}; GPU Y (BF16) against the oracle's own chain {rel_gpu:.2e}")
     assert rel_gpu <= 2.5e-3
