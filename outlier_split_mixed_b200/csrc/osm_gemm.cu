@@ -254,12 +254,18 @@ __device__ __forceinline__ void store_slab(const GemmParams& p, int64_t row0, in
 }
 // Wait for this warp's tensor-memory loads, then tell the leader CTA's
 // MMA warp that the accumulator may be overwritten (16 arrivals: 8 warps in
-// each CTA of the pair).
+// each CTA of the pair). The only ordering this hand-off needs is that of
+// the tensor-memory reads before the next tile's MMAs: tcgen05.wait::ld
+// returns once the loads have completed and tcgen05.fence::before_thread_sync
+// orders them before the arrival, so the arrival itself is relaxed; the
+// epilogue publishes no memory that the MMA warp reads. (A release arrival
+// at cluster scope waited for this lane's earlier global stores and cost
+// about 0.9 us of idle tensor pipe at every tile boundary.)
 __device__ __forceinline__ void release_accumulator(uint32_t acc_empty_leader, int lane) {
     ptx::tmem_ld_wait();
     ptx::tc_fence_before();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
+    if (lane == 0) ptx::mbar_arrive_remote_relaxed(acc_empty_leader);
 }
 // OSM_EPI_GELU_REQUANT for one 32-column group of one row (the lane's row),
 // columns c0 .. c0+31 (c0 < N; N % 32 == 0, so all 32 are real). Column c
@@ -451,7 +457,34 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem<NV>& S, bool 
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         const uint32_t acc = tmem;  // lane 0, column 0
+        // K-step ks of the slot `stage`: wait for its operands, then copy its
+        // scale atoms into the slot's tensor-memory columns. Neither touches
+        // the accumulator, so a tile's first K-step is prepared before the
+        // epilogue hands the accumulator back (the copies queue behind the
+        // previous tile's MMAs on the tensor pipe).
+        auto prepare = [&](int ks) -> bool {
+            if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.full[stage]), phase, p.wait_limit_ns, abort)) return false;
+            ptx::tc_fence_after();
+            if (ks < p.n_fp4) {
+                constexpr int APS = Fmt<NV>::APS;
+                const int natoms = min(APS, p.katoms - APS * ks);
+                const uint32_t sfa_col = tmem + SF_COL0 + stage * Fmt<NV>::SF_STAGE_COLS;
+                const uint32_t sfb_col = sfa_col + 4 * APS;
+                const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
+                const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
+                for (int a = 0; a < natoms; ++a) {
+                    ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
+                    ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
+                    ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + Fmt<NV>::SFB_HALF + 512 * a));
+                }
+            }
+            return true;
+        };
         for (int tile = pair; tile < tiles && ok; tile += npairs) {
+            if (!prepare(0)) {
+                ok = false;
+                break;
+            }
             if (!ptx::mbar_wait_bounded_cluster(ptx::smem_u32(&S.acc_empty), acc_phase ^ 1u, p.wait_limit_ns,
                                                 abort)) {
                 ok = false;
@@ -460,11 +493,10 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem<NV>& S, bool 
             ptx::tc_fence_after();
             uint32_t accumulate = 0;
             for (int ks = 0; ks < ksteps; ++ks) {
-                if (!ptx::mbar_wait_bounded(ptx::smem_u32(&S.full[stage]), phase, p.wait_limit_ns, abort)) {
+                if (ks > 0 && !prepare(ks)) {
                     ok = false;
                     break;
                 }
-                ptx::tc_fence_after();
                 const uint32_t a_base = ptx::smem_u32(S.a[stage]);
                 const uint32_t b_base = ptx::smem_u32(S.b[stage]);
                 if (ks < p.n_fp4) {
@@ -472,13 +504,6 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, Smem<NV>& S, bool 
                     const int natoms = min(APS, p.katoms - APS * ks);
                     const uint32_t sfa_col = tmem + SF_COL0 + stage * Fmt<NV>::SF_STAGE_COLS;
                     const uint32_t sfb_col = sfa_col + 4 * APS;
-                    const uint32_t sfa_s = ptx::smem_u32(S.sfa[stage]);
-                    const uint32_t sfb_s = ptx::smem_u32(S.sfb[stage]);
-                    for (int a = 0; a < natoms; ++a) {
-                        ptx::tc_cp_32x128_x4_pair(sfa_col + 4 * a, desc_sf(sfa_s + 512 * a));
-                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a, desc_sf(sfb_s + 512 * a));
-                        ptx::tc_cp_32x128_x4_pair(sfb_col + 8 * a + 4, desc_sf(sfb_s + Fmt<NV>::SFB_HALF + 512 * a));
-                    }
                     if constexpr (NV) {
                         // one atom (four 16-blocks per row) per MMA of K = 64
                         for (int kk = 0; kk < natoms; ++kk) {
