@@ -224,7 +224,7 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
     if (e == cudaSuccess) e = cudaMalloc(&p->d_status, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * K);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_inv_s_ord, sizeof(float) * K);
-    if (e == cudaSuccess) e = cudaMalloc(&p->d_s_new, sizeof(float) * 2 * K);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_s_new, sizeof(float) * 3 * K);  // s, inv_s, ranks
     if (e == cudaSuccess) e = cudaMalloc(&p->d_bad, sizeof(uint32_t));
     if (e != cudaSuccess) return cleanup(fail(OSM_ERR_NOMEM, "plan_create: %s", cudaGetErrorString(e)));
     e = cudaMemcpy(p->d_s, s_host, sizeof(float) * K, cudaMemcpyHostToDevice);

@@ -25,7 +25,7 @@ struct osm_plan {
     int32_t* d_order;    // [K]  channel order [J ascending | O ascending] (bulk positions, then slots)
     float* d_inv_s_ord;  // [K]  inv_s in that order: inv_s[d_order[c]]
     uint32_t* d_status;  // OSM_STATUS_* bits written by kernels
-    float* d_s_new;      // [K]  scratch of osm_plan_refresh: s, then inv_s ([2K] floats)
+    float* d_s_new;      // [3K] scratch of osm_plan_refresh: s, inv_s, then the channels' ranks (int32)
     uint32_t* d_bad;     // scratch of osm_plan_refresh: a statistic was not finite
     uint64_t wait_limit_ns;
     uint32_t debug_flags;  // OSM_DEBUG_* (failure-detection tests)

@@ -8,10 +8,16 @@
 // Kernel 1 (one thread per channel): s_j = fp32(max(amax_j,1e-5)^alpha /
 // max(wmax_j,1e-5)^(1-alpha)) in FP64 and inv_s_j = 1.0f / s_j into plan
 // scratch, and a flag if any statistic is not finite.
+// Kernel 1b (K <= RF_RANK_MAX_K, 0 < k < K), over the whole GPU: the rank of
+// every channel's key among all keys (the number of larger keys), each CTA
+// counting for 256 channels against a slice of the keys staged in shared
+// memory and adding its counts atomically; channel j is selected iff its
+// rank is below k (keys are unique).
 // Kernel 2, one CTA of 1024 threads (K <= 65536):
 //  1. flag set -> OSM_STATUS_NONFINITE, every table untouched;
 //  2. s, inv_s adopted from scratch;
 //  3. O = the k channels with the largest key (the score -- amax for Eq. (4),
+//     from the ranks of kernel 1b when it ran, otherwise as follows
 //     or a tail-aware percentile -- mapped to an unsigned integer of the
 //     same order, << 16 | 0xFFFF - j): keys are unique, and their order is
 //     score descending, then channel index ascending.
@@ -24,6 +30,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "osm_internal.h"
@@ -49,7 +56,11 @@ struct RefreshParams {
     int32_t* order;
     float* inv_s_ord;
     uint32_t* status;
+    const int32_t* rank;   // ranks from kernel 1b, or NULL (radix select)
 };
+
+constexpr int RF_RANK_MAX_K = 16384;  // above this the K^2 counting costs more than the radix select
+constexpr int RF_RANK_SLICE = 4096;   // keys per CTA slice (16 KB of shared memory)
 
 constexpr int RF_SMEM_KEYS = 32768;  // statistics staged in shared memory (128 KB)
 
@@ -110,6 +121,26 @@ __global__ void __launch_bounds__(256) refresh_smooth_kernel(const float* __rest
     s_new[K + j] = __fdiv_rn(1.0f, s);
 }
 
+__global__ void __launch_bounds__(256) rank_count_kernel(const float* __restrict__ score, int K, int slice,
+                                                         const uint32_t* __restrict__ bad, int32_t* __restrict__ rank) {
+    __shared__ uint32_t so[RF_RANK_SLICE];
+    if (*bad) return;  // non-finite statistics: the plan stays as it is
+    const int i0 = static_cast<int>(blockIdx.y) * slice;
+    const int n = min(slice, K - i0);
+    if (n <= 0) return;
+    for (int t = threadIdx.x; t < n; t += 256) so[t] = rf_ord(score[i0 + t]);
+    __syncthreads();
+    const int j = static_cast<int>(blockIdx.x) * 256 + threadIdx.x;
+    if (j >= K) return;
+    const uint64_t kj = (static_cast<uint64_t>(rf_ord(score[j])) << 16) | static_cast<uint64_t>(0xFFFF - j);
+    int cnt = 0;
+    for (int t = 0; t < n; ++t) {
+        const uint64_t ki = (static_cast<uint64_t>(so[t]) << 16) | static_cast<uint64_t>(0xFFFF - (i0 + t));
+        cnt += ki > kj ? 1 : 0;
+    }
+    atomicAdd(rank + j, cnt);
+}
+
 __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams p) {
     extern __shared__ uint32_t sk[];  // ordered statistics of the first min(K, RF_SMEM_KEYS) channels
     __shared__ unsigned hist[256];
@@ -137,7 +168,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     uint64_t thresh = 0;  // selected <=> key >= thresh
     if (p.k == 0) {
         thresh = ~0ull;
-    } else if (p.k < p.K) {
+    } else if (p.k < p.K && p.rank == nullptr) {
         if (tid == 0) {
             prefix_sh = 0;
             need_sh = p.k;
@@ -197,7 +228,9 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     for (int c0 = 0; c0 < p.K; c0 += RF_THREADS) {
         const int j = c0 + tid;
         const bool valid = j < p.K;
-        const int sel = valid && rf_key(sk, p.score, valid ? j : 0) >= thresh ? 1 : 0;
+        const int sel = !valid ? 0
+                        : (p.rank != nullptr && p.k > 0 && p.k < p.K) ? (p.rank[j] < p.k ? 1 : 0)
+                                                                       : (rf_key(sk, p.score, j) >= thresh ? 1 : 0);
         const int r_o = block_exclusive_scan(sel, warp_tot, &total) + base_o;
         const int n_sel = total;
         const int r_j = base_j + tid - (r_o - base_o);  // unselected channels before j
@@ -231,9 +264,20 @@ int launch_plan_refresh(osm_plan* pl, const float* amax, const float* score, con
     refresh_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(amax, score, wmax, static_cast<double>(alpha), K,
                                                           pl->d_s_new, pl->d_bad);
     if ((rc = check_cuda(cudaGetLastError(), "plan_refresh smooth launch"))) return rc;
-    RefreshParams p{amax, score, wmax, static_cast<double>(alpha), K, static_cast<int>(pl->k), static_cast<int>(pl->Kb),
+    const int k = static_cast<int>(pl->k);
+    int32_t* rank = nullptr;
+    if (k > 0 && k < K && K <= RF_RANK_MAX_K) {
+        rank = reinterpret_cast<int32_t*>(pl->d_s_new + 2 * static_cast<size_t>(K));
+        if ((rc = check_cuda(cudaMemsetAsync(rank, 0, sizeof(int32_t) * K, st), "plan_refresh ranks"))) return rc;
+        const int cx = (K + 255) / 256;
+        const int g = std::max((K + RF_RANK_SLICE - 1) / RF_RANK_SLICE, std::min(64, 296 / cx));  // ~2 CTAs per SM
+        const int slice = (K + g - 1) / g;  // <= RF_RANK_SLICE
+        rank_count_kernel<<<dim3(cx, (K + slice - 1) / slice), 256, 0, st>>>(score, K, slice, pl->d_bad, rank);
+        if ((rc = check_cuda(cudaGetLastError(), "plan_refresh rank launch"))) return rc;
+    }
+    RefreshParams p{amax, score, wmax, static_cast<double>(alpha), K, k, static_cast<int>(pl->Kb),
                     static_cast<int>(pl->Kbp), pl->d_s_new, pl->d_bad, pl->d_s, pl->d_inv_s, pl->d_route,
-                    pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status};
+                    pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status, rank};
     const size_t smem = sizeof(uint32_t) * static_cast<size_t>(K < RF_SMEM_KEYS ? K : RF_SMEM_KEYS);
     static bool attr_set[64] = {};
     int dev = 0;
