@@ -234,6 +234,9 @@ int osm_plan_create(int64_t K, int64_t N, int64_t k, const float* s_host, const 
         e = cudaMemcpy(p->d_J, J.data(), sizeof(int32_t) * (K - k), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && k > 0) e = cudaMemcpy(p->d_O, O_host, sizeof(int32_t) * k, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(uint32_t));
+    // osm_plan_refresh expects its flag and rank scratch zeroed on entry
+    if (e == cudaSuccess) e = cudaMemset(p->d_bad, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(p->d_s_new + 2 * K, 0, sizeof(float) * K);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_order, order.data(), sizeof(int32_t) * K, cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
         e = cudaMemcpy(p->d_inv_s_ord, inv_s_ord.data(), sizeof(float) * K, cudaMemcpyHostToDevice);

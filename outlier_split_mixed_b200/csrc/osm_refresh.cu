@@ -5,14 +5,14 @@
 // adopted per batch or per denoising step without a host round trip. The
 // arithmetic is that of osm_calibrate_finalize followed by osm_plan_create.
 //
-// Kernel 1 (one thread per channel): s_j = fp32(max(amax_j,1e-5)^alpha /
+// Kernel 1, one thread per channel: s_j = fp32(max(amax_j,1e-5)^alpha /
 // max(wmax_j,1e-5)^(1-alpha)) in FP64 and inv_s_j = 1.0f / s_j into plan
-// scratch, and a flag if any statistic is not finite.
-// Kernel 1b (K <= RF_RANK_MAX_K, 0 < k < K), over the whole GPU: the rank of
-// every channel's key among all keys (the number of larger keys), each CTA
-// counting for 256 channels against a slice of the keys staged in shared
-// memory and adding its counts atomically; channel j is selected iff its
-// rank is below k (keys are unique).
+// scratch, and a flag if any statistic is not finite. For K <=
+// RF_RANK_MAX_K and 0 < k < K the same launch spreads over the whole GPU
+// and also counts, for every channel, the keys larger than its own (its
+// rank), each CTA for 256 channels against a slice of the keys staged in
+// shared memory, adding its counts atomically; channel j is selected iff
+// its rank is below k (keys are unique). Two launches per refresh in all.
 // Kernel 2, one CTA of 1024 threads (K <= 65536):
 //  1. flag set -> OSM_STATUS_NONFINITE, every table untouched;
 //  2. s, inv_s adopted from scratch;
@@ -103,34 +103,39 @@ __device__ __forceinline__ int block_exclusive_scan(int flag, int* warp_tot, int
     return r;
 }
 
-__global__ void __launch_bounds__(256) refresh_smooth_kernel(const float* __restrict__ amax,
-                                                             const float* __restrict__ score,
-                                                             const float* __restrict__ wmax, double alpha, int K,
-                                                             float* __restrict__ s_new, uint32_t* __restrict__ bad) {
-    const int j = blockIdx.x * 256 + threadIdx.x;
-    if (j >= K) return;
-    const float a = amax[j], w = wmax[j];
-    if (!isfinite(a) || !isfinite(w) || !isfinite(score[j])) {
-        atomicOr(bad, 1u);
+// Kernel 1: CTA (x, y) covers channels 256x .. 256x+255. The CTAs of row
+// y = 0 compute s and inv_s of their channels; with `rank` set, the CTAs of
+// row y >= 1 count, for their channels, the larger keys among keys
+// slice*(y-1) .. slice*y-1 and add the counts to rank (zero on entry: the
+// plan is created with it zeroed and plan_refresh_kernel zeroes it again).
+__global__ void __launch_bounds__(256) refresh_stats_kernel(const float* __restrict__ amax,
+                                                            const float* __restrict__ score,
+                                                            const float* __restrict__ wmax, double alpha, int K,
+                                                            int slice, float* __restrict__ s_new,
+                                                            uint32_t* __restrict__ bad, int32_t* __restrict__ rank) {
+    __shared__ uint32_t so[RF_RANK_SLICE];
+    const int j = static_cast<int>(blockIdx.x) * 256 + threadIdx.x;
+    if (blockIdx.y == 0) {
+        if (j >= K) return;
+        const float a = amax[j], w = wmax[j];
+        if (!isfinite(a) || !isfinite(w) || !isfinite(score[j])) {
+            atomicOr(bad, 1u);
+        } else {
+            const double am = fmax(static_cast<double>(a), 1e-5);
+            const double wm = fmax(static_cast<double>(w), 1e-5);
+            const float sj = static_cast<float>(pow(am, alpha) / pow(wm, 1.0 - alpha));
+            s_new[j] = sj;
+            s_new[K + j] = __fdiv_rn(1.0f, sj);
+        }
         return;
     }
-    const double am = fmax(static_cast<double>(a), 1e-5);
-    const double wm = fmax(static_cast<double>(w), 1e-5);
-    const float s = static_cast<float>(pow(am, alpha) / pow(wm, 1.0 - alpha));
-    s_new[j] = s;
-    s_new[K + j] = __fdiv_rn(1.0f, s);
-}
-
-__global__ void __launch_bounds__(256) rank_count_kernel(const float* __restrict__ score, int K, int slice,
-                                                         const uint32_t* __restrict__ bad, int32_t* __restrict__ rank) {
-    __shared__ uint32_t so[RF_RANK_SLICE];
-    if (*bad) return;  // non-finite statistics: the plan stays as it is
-    const int i0 = static_cast<int>(blockIdx.y) * slice;
+    // rows y >= 1 count (with a non-finite statistic the counts are
+    // meaningless, and unused)
+    const int i0 = static_cast<int>(blockIdx.y - 1) * slice;
     const int n = min(slice, K - i0);
     if (n <= 0) return;
     for (int t = threadIdx.x; t < n; t += 256) so[t] = rf_ord(score[i0 + t]);
     __syncthreads();
-    const int j = static_cast<int>(blockIdx.x) * 256 + threadIdx.x;
     if (j >= K) return;
     const uint64_t kj = (static_cast<uint64_t>(rf_ord(score[j])) << 16) | static_cast<uint64_t>(0xFFFF - j);
     int cnt = 0;
@@ -150,9 +155,16 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     __shared__ int need_sh;
     const int tid = threadIdx.x;
 
-    // 1. statistics must be finite
+    // 1. statistics must be finite (the scratch flag and ranks are left
+    // zeroed for the next refresh in every case)
     if (*p.bad) {
-        if (tid == 0) atomicOr(p.status, OSM_STATUS_NONFINITE);
+        __syncthreads();  // every thread has read the flag
+        if (tid == 0) {
+            atomicOr(p.status, OSM_STATUS_NONFINITE);
+            *const_cast<uint32_t*>(p.bad) = 0;
+        }
+        if (p.rank != nullptr)
+            for (int j = tid; j < p.K; j += RF_THREADS) const_cast<int32_t*>(p.rank)[j] = 0;
         return;
     }
 
@@ -252,6 +264,9 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
         base_j += min(RF_THREADS, p.K - c0) - n_sel;
         __syncthreads();
     }
+    if (p.rank != nullptr)
+        for (int j = tid; j < p.K; j += RF_THREADS) const_cast<int32_t*>(p.rank)[j] = 0;
+    if (tid == 0) *const_cast<uint32_t*>(p.bad) = 0;
 }
 
 }  // namespace
@@ -259,22 +274,23 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
 int launch_plan_refresh(osm_plan* pl, const float* amax, const float* score, const float* wmax, float alpha,
                         cudaStream_t st) {
     const int K = static_cast<int>(pl->K);
-    int rc = check_cuda(cudaMemsetAsync(pl->d_bad, 0, sizeof(uint32_t), st), "plan_refresh flag");
-    if (rc) return rc;
-    refresh_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(amax, score, wmax, static_cast<double>(alpha), K,
-                                                          pl->d_s_new, pl->d_bad);
-    if ((rc = check_cuda(cudaGetLastError(), "plan_refresh smooth launch"))) return rc;
     const int k = static_cast<int>(pl->k);
+    int rc;
+    // the flag and the ranks are zero here: zeroed at plan creation and by
+    // every plan_refresh_kernel before it exits
     int32_t* rank = nullptr;
+    const int cx = (K + 255) / 256;
+    int gy = 1, slice = K;
     if (k > 0 && k < K && K <= RF_RANK_MAX_K) {
         rank = reinterpret_cast<int32_t*>(pl->d_s_new + 2 * static_cast<size_t>(K));
-        if ((rc = check_cuda(cudaMemsetAsync(rank, 0, sizeof(int32_t) * K, st), "plan_refresh ranks"))) return rc;
-        const int cx = (K + 255) / 256;
         const int g = std::max((K + RF_RANK_SLICE - 1) / RF_RANK_SLICE, std::min(64, 296 / cx));  // ~2 CTAs per SM
-        const int slice = (K + g - 1) / g;  // <= RF_RANK_SLICE
-        rank_count_kernel<<<dim3(cx, (K + slice - 1) / slice), 256, 0, st>>>(score, K, slice, pl->d_bad, rank);
-        if ((rc = check_cuda(cudaGetLastError(), "plan_refresh rank launch"))) return rc;
+        slice = (K + g - 1) / g;  // <= RF_RANK_SLICE
+        gy = (K + slice - 1) / slice;
     }
+    // row y = 0 of the grid: Eq. (2) per channel; rows 1 .. gy: the rank counts
+    refresh_stats_kernel<<<dim3(cx, rank ? gy + 1 : 1), 256, 0, st>>>(amax, score, wmax, static_cast<double>(alpha), K, slice,
+                                                      pl->d_s_new, pl->d_bad, rank);
+    if ((rc = check_cuda(cudaGetLastError(), "plan_refresh statistics launch"))) return rc;
     RefreshParams p{amax, score, wmax, static_cast<double>(alpha), K, k, static_cast<int>(pl->Kb),
                     static_cast<int>(pl->Kbp), pl->d_s_new, pl->d_bad, pl->d_s, pl->d_inv_s, pl->d_route,
                     pl->d_J, pl->d_O, pl->d_order, pl->d_inv_s_ord, pl->d_status, rank};
