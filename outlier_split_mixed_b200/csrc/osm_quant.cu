@@ -656,7 +656,7 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 // thread (one CTA per SM then has the registers and the shared memory for
 // a deeper ring).
 template <int R, int S, int NT, int TR, int MODE>
-__global__ void __launch_bounds__(NT, (TR > 6 ? 1 : 2)) quantize_act_stream_kernel(QuantParams p) {
+__global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quantize_act_stream_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
     ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
     extern __shared__ __align__(128) uint8_t smem[];
@@ -917,6 +917,13 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
     const size_t two_per_sm = 110 * 1024;
     const int npairs = p.K / 2;
     if (stream_smem_bytes<2, 3>(p.K, stride) <= two_per_sm) {
+        // Large batches: three CTAs of 256 threads per SM with a two-slot ring
+        // (a block barrier spans fewer warps; measured 111.6 against 118.8 us
+        // for 32760 x 5120). Small batches keep two 512-thread CTAs with three
+        // slots (23.6 against 24.6 us for 4096 x 5120), whose deeper ring
+        // matters when each CTA sees only a few row groups.
+        if (p.M >= 8192 && npairs <= 10 * 256 && stream_smem_bytes<2, 2>(p.K, stride) * 3 <= 220 * 1024)
+            return launch_stream<2, 2, 256, 10>(p, mode, stride, st);
         if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, mode, stride, st);
         return launch_stream<2, 3, STREAM_NT, 0>(p, mode, stride, st);
     }
