@@ -307,19 +307,24 @@ __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0
 // lanes); 128x1: the maximum over the strip's four blocks (four warps, via
 // shared memory). NV: the 32 positions are two NVFP4 16-blocks, each with
 // its own E4M3 scale and element multiplier.
-// Encode one strip (128 bulk positions p0 .. p0+127, strip index p0 / 128)
-// of 128 packed output channels n0 .. n0+127 from the folded values: warp w
-// encodes block q = w / 2 for the 64 channel pairs 32 (w % 2) + lane; wv[i]
-// is the pair (channel n, channel n + 1) at position 32 q + i. Every thread
-// of the CTA calls it (it synchronises through red / sxs).
 template <bool NV>
-__device__ __forceinline__ void encode_bulk_strip(const PackParams& p, int64_t n0, int64_t p0, int64_t strip,
-                                                  const uint32_t (&wv)[32], uint32_t (*red)[64],
-                                                  uint32_t (*sxs)[64]) {
+__global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams p) {
+    __shared__ __align__(16) uint32_t tile[128][64];
+    __shared__ uint32_t red[4][64];
+    __shared__ uint32_t sxs[4][64];  // scale codes per quarter and pair: MX (n | n+1 << 8), NV (n: 2 bytes | n+1: 2 bytes)
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
+    const int64_t p0 = static_cast<int64_t>(blockIdx.y) * 128;
     const int64_t katoms = p.katoms;
+    load_folded_rows<false>(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; },
+                            tile);
+    __syncthreads();
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp >> 1;
     const int c = 32 * (warp & 1) + lane;  // channel pair: columns n0 + 2c, n0 + 2c + 1
+    uint32_t wv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) wv[i] = tile[32 * q + i][c];
     using mx::bf16x2_absmax;
     const int64_t n = n0 + 2 * c;
     if constexpr (NV) {
@@ -358,7 +363,7 @@ __device__ __forceinline__ void encode_bulk_strip(const PackParams& p, int64_t n
             uint32_t w0hi = (sxs[0][c] >> 16) | (sxs[1][c] & 0xFFFF0000u), w1hi = (sxs[2][c] >> 16) | (sxs[3][c] & 0xFFFF0000u);
             if (n >= p.N) w0lo = w1lo = 0;
             if (n + 1 >= p.N) w0hi = w1hi = 0;
-            const int64_t b0 = strip * 8;
+            const int64_t b0 = static_cast<int64_t>(blockIdx.y) * 8;
             *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, b0, katoms)) = w0lo;
             *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, b0 + 4, katoms)) = w1lo;
             *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n + 1, b0, katoms)) = w0hi;
@@ -412,91 +417,9 @@ __device__ __forceinline__ void encode_bulk_strip(const PackParams& p, int64_t n
         }
         if (n >= p.N) wlo = 0;
         if (n + 1 >= p.N) whi = 0;
-                *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, strip * 4, katoms)) = wlo;
+        const int64_t strip = blockIdx.y;
+        *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n, strip * 4, katoms)) = wlo;
         *reinterpret_cast<uint32_t*>(p.scales + sf_offset(n + 1, strip * 4, katoms)) = whi;
-    }
-}
-
-template <bool NV>
-__global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams p) {
-    __shared__ __align__(16) uint32_t tile[128][64];
-    __shared__ uint32_t red[4][64];
-    __shared__ uint32_t sxs[4][64];  // scale codes per quarter and pair: MX (n | n+1 << 8), NV (n: 2 bytes | n+1: 2 bytes)
-    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
-    const int64_t p0 = static_cast<int64_t>(blockIdx.y) * 128;
-    load_folded_rows<false>(p, n0, 128, [&](int r) -> int64_t { return p0 + r < p.Kb ? __ldg(p.J + p0 + r) : -1; },
-                            tile);
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp >> 1;
-    const int c = 32 * (warp & 1) + lane;
-    uint32_t wv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) wv[i] = tile[32 * q + i][c];
-    encode_bulk_strip<NV>(p, n0, p0, blockIdx.y, wv, red, sxs);
-}
-
-// The same packing for W in its natural column order, as a persistent kernel
-// whose CTAs take tiles (strip, 128 channels) in turn and fetch the next
-// tile's 128 W rows (raw BF16, 16-byte asynchronous copies; rows past Kb and
-// columns past N zero-filled) and their s while they encode the current one:
-// the loads of one tile overlap the arithmetic of the previous, where the
-// one-tile-per-CTA form alternated between the two. s is folded in as the
-// values are read back from shared memory.
-constexpr int PKS_TILE_WORDS = 128 * 64;
-template <bool NV>
-__global__ void __launch_bounds__(PK_THREADS) pack_bulk_stream_kernel(PackParams p, int tiles_n, int tiles) {
-    extern __shared__ __align__(16) uint32_t pk_smem[];
-    uint32_t* raw = pk_smem;                                               // [2][128][64]
-    float* srow = reinterpret_cast<float*>(pk_smem + 2 * PKS_TILE_WORDS);  // [2][128]
-    __shared__ uint32_t red[4][64];
-    __shared__ uint32_t sxs[4][64];
-    auto issue = [&](int t, int buf) {
-        const int64_t n0 = static_cast<int64_t>(t % tiles_n) * 128;
-        const int64_t p0 = static_cast<int64_t>(t / tiles_n) * 128;
-        const uint32_t dst0 = ptx::smem_u32(raw + buf * PKS_TILE_WORDS);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int u = threadIdx.x + i * PK_THREADS;  // 16-byte chunk u of the tile: row u / 16, chunk u % 16
-            const int r = u >> 4, ch = u & 15;
-            const int64_t pos = p0 + r, n = n0 + 8 * ch;
-            const bool real = pos < p.Kb && n < p.N;
-            const int64_t j = real ? __ldg(p.J + pos) : 0;
-            const uint16_t* src = p.W + (real ? j * p.N + n : 0);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst0 + 16u * u), "l"(src),
-                         "r"(real ? 16 : 0)
-                         : "memory");
-        }
-        if (threadIdx.x < 128) {
-            const int64_t pos = p0 + threadIdx.x;
-            srow[buf * 128 + threadIdx.x] = pos < p.Kb ? __ldg(p.s + __ldg(p.J + pos)) : 0.0f;
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp >> 1;
-    const int c = 32 * (warp & 1) + lane;
-    int t = blockIdx.x;
-    if (t < tiles) issue(t, 0);
-    for (int i = 0; t < tiles; t += gridDim.x, ++i) {
-        const int cur = i & 1;
-        const int tn = t + static_cast<int>(gridDim.x);
-        if (tn < tiles) issue(tn, cur ^ 1);
-        if (tn < tiles) asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();  // the current tile (every thread's copies and s) has landed
-        const uint32_t* tile = raw + cur * PKS_TILE_WORDS;
-        const float* sr = srow + cur * 128;
-        uint32_t wv[32];
-#pragma unroll
-        for (int k2 = 0; k2 < 32; ++k2) {
-            const float sj = sr[32 * q + k2];
-            wv[k2] = smooth2(tile[(32 * q + k2) * 64 + c], make_float2(sj, sj));
-        }
-        const int64_t n0 = static_cast<int64_t>(t % tiles_n) * 128;
-        const int64_t strip = t / tiles_n;
-        encode_bulk_strip<NV>(p, n0, strip * 128, strip, wv, red, sxs);
-        __syncthreads();  // the buffer is refilled two tiles on
     }
 }
 
@@ -892,35 +815,7 @@ int launch_pack_weights(const osm_plan* pl, const uint16_t* W, const int32_t* co
     PackParams p{W, col_order, pl->d_s, pl->d_J, pl->d_O, pl->K, pl->N, pl->k, pl->Kb, pl->Kbp, pl->kp,
                  pl->wmode, codes, scales, hp, static_cast<int>(pl->Kbp / (4 * block_elems(pl->fmt))), nv ? 1 : 0,
                  nvfp4_k(pl->g_w), pow2f(pl->g_w), pow2f(-pl->g_w)};
-    if (pl->Kbp > 0 && col_order == nullptr) {
-        // natural column order: the persistent, double-buffered form
-        const int tiles_n = static_cast<int>(round_up(pl->N, 128) / 128);
-        const int tiles = tiles_n * static_cast<int>(pl->Kbp / 128);
-        const size_t smem = sizeof(uint32_t) * 2 * PKS_TILE_WORDS + sizeof(float) * 2 * 128;
-        auto kern = nv ? pack_bulk_stream_kernel<true> : pack_bulk_stream_kernel<false>;
-        int dev = 0, rc;
-        if ((rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice"))) return rc;
-        static int per_sm_cache[2][64] = {};
-        static int sms_cache[64] = {};
-        if (dev < 0 || dev >= 64) return fail(OSM_ERR_UNSUPPORTED, "device index %d", dev);
-        int& per_sm = per_sm_cache[nv ? 1 : 0][dev];
-        if (per_sm == 0) {
-            if ((rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      static_cast<int>(smem)),
-                                 "pack_weights smem attribute")))
-                return rc;
-            if ((rc = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, PK_THREADS, smem),
-                                 "pack_weights occupancy")))
-                return rc;
-            if ((rc = check_cuda(cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev),
-                                 "SM count")))
-                return rc;
-            if (per_sm < 1) return fail(OSM_ERR_UNSUPPORTED, "pack_weights: no CTA fits");
-        }
-        const int grid = std::min(tiles, sms_cache[dev] * per_sm);
-        kern<<<grid, PK_THREADS, smem, st>>>(p, tiles_n, tiles);
-        if ((rc = check_cuda(cudaGetLastError(), "pack_bulk launch"))) return rc;
-    } else if (pl->Kbp > 0) {
+    if (pl->Kbp > 0) {
         dim3 grid(static_cast<unsigned>(round_up(pl->N, 128) / 128), static_cast<unsigned>(pl->Kbp / 128));
         if (nv) pack_bulk_tiled_kernel<true><<<grid, PK_THREADS, 0, st>>>(p);
         else pack_bulk_tiled_kernel<false><<<grid, PK_THREADS, 0, st>>>(p);
