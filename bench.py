@@ -75,8 +75,8 @@ E2E_STREAMS = 3
 # workload (one pass), per (workload, kernel); a workload or kernel without a
 # capture of the current code reports null.
 DUAL_GEMM_TRAFFIC = {
-    ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 377.87e6,
-    ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 708.12e6,
+    ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 384.38e6,
+    ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 731.06e6,
 }
 
 
