@@ -77,6 +77,7 @@ E2E_STREAMS = 3
 DUAL_GEMM_TRAFFIC = {
     ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 384.38e6,
     ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 731.06e6,
+    ("wan_ffn_up_4096x5120x13824", "mxfp4"): 298.72e6,
 }
 
 
