@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "osm_internal.h"
@@ -655,7 +656,9 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 // Two CTAs per SM, except with more than six register-held pairs per
 // thread (one CTA per SM then has the registers and the shared memory for
 // a deeper ring).
-template <int R, int S, int NT, int TR, int MODE>
+// FP: the threads' register-held pairs cover exactly the K / 2 channel pairs
+// (K / 2 == TR * NT), so no pair needs a bound check.
+template <int R, int S, int NT, int TR, int MODE, bool FP>
 __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quantize_act_stream_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
     ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
@@ -743,12 +746,16 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
         }
         const uint32_t src = raw_u32 + (i % S) * raw_bytes + tid * 4;  // this thread's first pair, row 0
         if constexpr (TR > 0) {
+            // a whole group (rows == R) routes without per-row checks, and
+            // with FP without per-pair checks; only the batch's last group
+            // can be partial
+            auto route_rows = [&](auto rr) {
+                constexpr int RR = decltype(rr)::value;
 #pragma unroll
-            for (int j = 0; j < TR; ++j) {
-                if (tid + j * NT < npairs) {
+                for (int j = 0; j < TR; ++j) {
+                    if (FP || tid + j * NT < npairs) {
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        if (r < rows) {
+                        for (int r = 0; r < RR; ++r) {
                             const uint32_t x = ptx::ld_shared_u32(src + r * row_bytes + j * NT * 4);
                             const uint32_t h = HPF ? smooth2_mixed(x, tsv[j], tmask[j]) : smooth2(x, tsv[j]);
                             ptx::st_shared_u16(tad[j].x + r * stride, h);
@@ -756,6 +763,12 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
                         }
                     }
                 }
+            };
+            if (rows == R) {
+                route_rows(std::integral_constant<int, R>{});
+            } else {
+                static_assert(R <= 2, "a partial group of the register-held form has one row");
+                route_rows(std::integral_constant<int, 1>{});
             }
         } else {
             for (int c = tid; c < npairs; c += NT) {
@@ -889,9 +902,13 @@ static int launch_qa(const QuantParams& p, int mode, size_t smem, cudaStream_t s
 template <int R, int S, int NT, int TR>
 static int launch_stream(const QuantParams& p, int mode, int stride, cudaStream_t st) {
     const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
-    auto kern = mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV>
-                              : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16>
-                                                   : quantize_act_stream_kernel<R, S, NT, TR, QA_MX>);
+    const bool fp = TR > 0 && p.K / 2 == TR * NT;
+    auto kern = fp ? (mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV, true>
+                                    : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16, true>
+                                                         : quantize_act_stream_kernel<R, S, NT, TR, QA_MX, true>))
+                   : (mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV, false>
+                                    : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16, false>
+                                                         : quantize_act_stream_kernel<R, S, NT, TR, QA_MX, false>));
     int per_sm = 0, sms = 0;
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
     if (rc) return rc;
@@ -924,6 +941,7 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
         // matters when each CTA sees only a few row groups.
         if (p.M >= 8192 && npairs <= 10 * 256 && stream_smem_bytes<2, 2>(p.K, stride) * 3 <= 220 * 1024)
             return launch_stream<2, 2, 256, 10>(p, mode, stride, st);
+        if (npairs == 5 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 5>(p, mode, stride, st);
         if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, mode, stride, st);
         return launch_stream<2, 3, STREAM_NT, 0>(p, mode, stride, st);
     }
