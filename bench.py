@@ -75,9 +75,9 @@ E2E_STREAMS = 3
 # workload (one pass), per (workload, kernel); a workload or kernel without a
 # capture of the current code reports null.
 DUAL_GEMM_TRAFFIC = {
-    ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 384.38e6,
-    ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 731.06e6,
-    ("wan_ffn_up_4096x5120x13824", "mxfp4"): 298.72e6,
+    ("wan_ffn_block_x4_32760x5120x13824", "up_gelu_requant"): 380.74e6,
+    ("wan_ffn_block_x4_32760x5120x13824", "down_bf16"): 723.50e6,
+    ("wan_ffn_up_4096x5120x13824", "mxfp4"): 292.47e6,
 }
 
 

@@ -557,7 +557,11 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, Smem<NV>& S, 
         tile_coords(tile, p.num_m, p.num_n, p.group_m, m_blk, n_blk);
         int ok = 1;
         if (lane == 0)
-            ok = ptx::mbar_wait_bounded(ptx::smem_u32(&S.acc_full), acc_phase, p.wait_limit_ns, abort) ? 1 : 0;
+            // the accumulator completes once per tile (about 10 us of MMAs):
+            // a suspending wait polls less (1-2 % on the power-capped FFN step)
+            ok = ptx::mbar_wait_bounded_long(ptx::smem_u32(&S.acc_full), acc_phase, p.wait_limit_ns, abort, 20000u)
+                     ? 1
+                     : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
             if (lane == 0) raise_abort(S, p.status);

@@ -83,6 +83,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// As mbar_try_wait, with a suspend-time hint: a thread whose phase has not
+// completed may stay suspended up to `ns` nanoseconds (it resumes when the
+// phase completes). For long waits: fewer polls.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait_bounded for waits expected to last many microseconds: each poll
+// may suspend the thread for up to hint_ns; the abort flag and the limit are
+// checked every fourth poll.
+__device__ __forceinline__ bool mbar_wait_bounded_long(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                                       const volatile int* abort, uint32_t hint_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+        if ((it & 3u) == 3u) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > limit_ns) return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
