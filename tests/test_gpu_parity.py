@@ -6,9 +6,11 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
+import oracle  # noqa: E402
 import outlier_split_mixed_b200 as osm  # noqa: E402
 from outlier_split_mixed_b200 import synth  # noqa: E402
-from gpu_helpers import assert_y_close, compare_layer, gpu_layer, oracle_layer  # noqa: E402
+from gpu_helpers import (assert_bitexact, assert_y_close, compare_layer, gpu_layer, oracle_layer,  # noqa: E402
+                         to_np_u16, unswizzle)
 
 pytestmark = pytest.mark.gpu
 
@@ -186,3 +188,28 @@ def test_quant_linear_and_host_entry_point_agree():
     osm.linear_host(plan, Xh, cfg.M, lin.w_codes, lin.w_scales, lin.w_hp, Yh, ws)
     torch.cuda.synchronize()
     assert torch.equal(Y.cpu(), Yh)
+
+
+@pytest.mark.parametrize("M", [8191, 8193, 8194])
+def test_quantize_act_large_batches_ragged_last_group(M):
+    # Batches of 8192 rows and more at K = 5120 run the three-CTA form whose
+    # register-held pairs cover K/2 exactly; an odd M leaves its last row
+    # group with one row. Codes, scales (padding rows 0) and outlier slots
+    # are bit-exact against the oracle on every row.
+    K, k = 5120, 128
+    X = synth.acts_heavy_tailed(M, K, 4242 + M, frac=0.02)
+    W = synth.weights_gaussian(K, 256, 4243, sigma=0.04)
+    s, inv_s, O = oracle.calibrate(oracle.act_amax(X), oracle.weight_amax(W), 0.6, k)
+    plan = osm.Plan(K, 256, k, s, O, osm.WSCALE_STRIP128x1)
+    Xd = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).cuda().view(torch.bfloat16)
+    ac, asc, ah = plan.alloc_packed(M)
+    osm.quantize_act(plan, Xd, ac, asc, ah)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    codes, scales, hp = oracle.quantize_act(X, inv_s, O)
+    nb = plan.Kbp // 32
+    assert_bitexact("a_codes", ac.cpu().numpy().reshape(M, plan.Kbp // 2), codes)
+    sc = unswizzle(asc.cpu().numpy(), M, nb)
+    assert_bitexact("a_scales", sc[:M], scales)
+    assert np.all(sc[M:] == 0), "padding rows of a_scales must be 0"
+    assert_bitexact("a_hp", to_np_u16(ah).reshape(M, plan.kp), hp)
