@@ -73,25 +73,25 @@ __device__ __forceinline__ uint32_t slot_mask(int2 dv, int slot0) {
 // ------------------------------------------------------------ calibration
 
 constexpr int AMAX_THREADS = 256;
-constexpr int AMAX_ROWS = 256;  // rows per CTA: 32 per warp
+constexpr int AMAX_ROWS = 256;  // rows per CTA (at most; fewer for small batches)
 
 // amax[j] = max(amax[j], max_t |X[t][j]|). A CTA covers 256 channels (a
-// lane takes 8 channels, 16 bytes of a row) and AMAX_ROWS rows (warp w
-// takes rows w, w + 8, ...), with eight 16-byte row loads per lane in
+// lane takes 8 channels, 16 bytes of a row) and `rows` rows (warp w takes
+// rows w, w + 8, ...), with eight 16-byte row loads per lane in
 // flight; the maxima are kept as packed u16 pairs of |x| bit patterns
 // (integer order, so a NaN pattern propagates and the finiteness check of
 // the calibration sees it), combined over the warps in shared memory and
 // merged with one atomicMax per channel and CTA on the IEEE bit pattern of
 // the FP32 value (monotone for non-negative floats).
 __global__ void __launch_bounds__(AMAX_THREADS) act_amax_kernel(const uint16_t* __restrict__ X, int64_t T,
-                                                                int64_t K, float* __restrict__ amax) {
+                                                                int64_t K, float* __restrict__ amax, int rows) {
     constexpr int NW = AMAX_THREADS / 32;
     __shared__ uint32_t red[NW][32][4];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t v = static_cast<int64_t>(blockIdx.x) * 32 + lane;  // 8-channel group
     const bool active = v * 8 < K;
-    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * AMAX_ROWS;
-    const int64_t t1 = min(T, t0 + AMAX_ROWS);
+    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * rows;
+    const int64_t t1 = min(T, t0 + rows);
     uint32_t m[4] = {0, 0, 0, 0};
     const uint16_t* src = X + v * 8;
     if (active) {
@@ -822,9 +822,18 @@ size_t stream_smem_bytes(int K, int stride) {
 
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st) {
     if (T == 0) return OSM_OK;
-    dim3 grid(static_cast<unsigned>(ceil_div(K / 8, 32)), static_cast<unsigned>(ceil_div(T, AMAX_ROWS)));
-    if (grid.y > 65535u) return fail(OSM_ERR_UNSUPPORTED, "act_amax: T too large for one launch");
-    act_amax_kernel<<<grid, AMAX_THREADS, 0, st>>>(X, T, K, amax);
+    // rows per CTA: AMAX_ROWS, or fewer (a multiple of 64) when that would
+    // leave the GPU with less than about two waves of CTAs (small batches:
+    // 4096 x 5120 took 15.1 us with 256 rows per CTA)
+    const int64_t groups = ceil_div(K / 8, 32);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t target = 2ll * sms * 6;
+    int64_t rows = ceil_div(ceil_div(T * groups, target), 64) * 64;
+    rows = rows < 64 ? 64 : (rows > AMAX_ROWS ? AMAX_ROWS : rows);
+    dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(T, rows)));
+    if (ceil_div(T, rows) > 65535) return fail(OSM_ERR_UNSUPPORTED, "act_amax: T too large for one launch");
+    act_amax_kernel<<<grid, AMAX_THREADS, 0, st>>>(X, T, K, amax, static_cast<int>(rows));
     return check_cuda(cudaGetLastError(), "act_amax launch");
 }
 

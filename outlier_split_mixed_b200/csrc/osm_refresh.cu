@@ -137,12 +137,15 @@ __global__ void __launch_bounds__(256) refresh_stats_kernel(const float* __restr
     for (int t = threadIdx.x; t < n; t += 256) so[t] = rf_ord(score[i0 + t]);
     __syncthreads();
     if (j >= K) return;
-    const uint64_t kj = (static_cast<uint64_t>(rf_ord(score[j])) << 16) | static_cast<uint64_t>(0xFFFF - j);
+    // key i > key j  <=>  ord_i > ord_j, or ord_i == ord_j and i < j: the
+    // keys of channels below j count when >=, the others when >
+    const uint32_t oj = rf_ord(score[j]);
+    const int split = min(max(j - i0, 0), n);
     int cnt = 0;
-    for (int t = 0; t < n; ++t) {
-        const uint64_t ki = (static_cast<uint64_t>(so[t]) << 16) | static_cast<uint64_t>(0xFFFF - (i0 + t));
-        cnt += ki > kj ? 1 : 0;
-    }
+#pragma unroll 4
+    for (int t = 0; t < split; ++t) cnt += so[t] >= oj ? 1 : 0;
+#pragma unroll 4
+    for (int t = split; t < n; ++t) cnt += so[t] > oj ? 1 : 0;
     atomicAdd(rank + j, cnt);
 }
 
