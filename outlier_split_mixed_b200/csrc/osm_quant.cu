@@ -656,9 +656,11 @@ __device__ __forceinline__ void zero_padding_scale_rows(const QuantParams& p) {
 // Two CTAs per SM, except with more than six register-held pairs per
 // thread (one CTA per SM then has the registers and the shared memory for
 // a deeper ring).
-// FP: the threads' register-held pairs cover exactly the K / 2 channel pairs
-// (K / 2 == TR * NT), so no pair needs a bound check.
-template <int R, int S, int NT, int TR, int MODE, bool FP>
+// FP: 2 when the threads' register-held pairs cover exactly the K / 2
+// channel pairs (K / 2 == TR * NT: no pair needs a bound check), 1 when only
+// the last of each thread's TR pairs may lie past K / 2 (K / 2 >= (TR - 1) *
+// NT), 0 otherwise (every pair checked).
+template <int R, int S, int NT, int TR, int MODE, int FP>
 __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quantize_act_stream_kernel(QuantParams p) {
     constexpr bool HPF = MODE == QA_MX_F16;
     ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
@@ -755,14 +757,14 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
             // 32760 x 5120).
             auto route_rows = [&](auto rr) {
                 constexpr int RR = decltype(rr)::value;
-                constexpr int CH = !FP ? 1 : (TR <= 6 ? TR : (TR + 1) / 2);  // bound-checked pairs: one at a time
+                constexpr int CH = FP == 0 ? 1 : (TR <= 6 ? TR : (TR + 1) / 2);  // bound-checked pairs: one at a time
 #pragma unroll
                 for (int j0 = 0; j0 < TR; j0 += CH) {
                     uint32_t x[CH][RR];
 #pragma unroll
                     for (int jj = 0; jj < CH; ++jj) {
                         const int j = j0 + jj;
-                        if (j < TR && (FP || tid + j * NT < npairs)) {
+                        if (j < TR && (FP == 2 || (FP == 1 && j < TR - 1) || tid + j * NT < npairs)) {
 #pragma unroll
                             for (int r = 0; r < RR; ++r) x[jj][r] = ptx::ld_shared_u32(src + r * row_bytes + j * NT * 4);
                         }
@@ -770,7 +772,7 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
 #pragma unroll
                     for (int jj = 0; jj < CH; ++jj) {
                         const int j = j0 + jj;
-                        if (j < TR && (FP || tid + j * NT < npairs)) {
+                        if (j < TR && (FP == 2 || (FP == 1 && j < TR - 1) || tid + j * NT < npairs)) {
 #pragma unroll
                             for (int r = 0; r < RR; ++r) {
                                 const uint32_t h = HPF ? smooth2_mixed(x[jj][r], tsv[j], tmask[j]) : smooth2(x[jj][r], tsv[j]);
@@ -928,13 +930,16 @@ static int launch_qa(const QuantParams& p, int mode, size_t smem, cudaStream_t s
 template <int R, int S, int NT, int TR>
 static int launch_stream(const QuantParams& p, int mode, int stride, cudaStream_t st) {
     const size_t smem = stream_smem_bytes<R, S>(p.K, stride);
-    const bool fp = TR > 0 && p.K / 2 == TR * NT;
-    auto kern = fp ? (mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV, true>
-                                    : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16, true>
-                                                         : quantize_act_stream_kernel<R, S, NT, TR, QA_MX, true>))
-                   : (mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV, false>
-                                    : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16, false>
-                                                         : quantize_act_stream_kernel<R, S, NT, TR, QA_MX, false>));
+    const int np = p.K / 2;
+    const int fp = TR == 0 ? 0 : (np == TR * NT ? 2 : (np >= (TR - 1) * NT ? 1 : 0));
+    auto pick = [&](auto f) {
+        constexpr int F = decltype(f)::value;
+        return mode == QA_NV ? quantize_act_stream_kernel<R, S, NT, TR, QA_NV, F>
+                             : (mode == QA_MX_F16 ? quantize_act_stream_kernel<R, S, NT, TR, QA_MX_F16, F>
+                                                  : quantize_act_stream_kernel<R, S, NT, TR, QA_MX, F>);
+    };
+    auto kern = fp == 2 ? pick(std::integral_constant<int, 2>{})
+                        : (fp == 1 ? pick(std::integral_constant<int, 1>{}) : pick(std::integral_constant<int, 0>{}));
     int per_sm = 0, sms = 0;
     int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
     if (rc) return rc;
