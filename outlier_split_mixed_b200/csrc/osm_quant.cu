@@ -748,16 +748,15 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
         }
         const uint32_t src = raw_u32 + (i % S) * raw_bytes + tid * 4;  // this thread's first pair, row 0
         if constexpr (TR > 0) {
-            // a whole group (rows == R) routes without per-row checks, and
-            // with FP without per-pair checks; only the batch's last group
-            // can be partial
-            // The loads of a chunk of CH pairs are issued before any of its
-            // routed stores (the shared accesses keep their program order),
-            // so their latencies overlap (100.4 against 102.4 us at
-            // 32760 x 5120).
+            // A whole group (rows == R) routes without per-row checks, and
+            // pairs known to lie inside K/2 (FP) without bound checks; only
+            // the batch's last group can be partial. The loads of a chunk of
+            // CH pairs are issued before any of its routed stores (the
+            // shared accesses keep their program order), so their latencies
+            // overlap (100.4 against 102.4 us at 32760 x 5120).
             auto route_rows = [&](auto rr) {
                 constexpr int RR = decltype(rr)::value;
-                constexpr int CH = FP == 0 ? 1 : (TR <= 6 ? TR : (TR + 1) / 2);  // bound-checked pairs: one at a time
+                constexpr int CH = FP == 0 ? 1 : (TR <= 6 ? TR : (TR + 1) / 2);  // every pair checked: one at a time
 #pragma unroll
                 for (int j0 = 0; j0 < TR; j0 += CH) {
                     uint32_t x[CH][RR];
