@@ -812,6 +812,256 @@ __global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : (TR > 6 ? 1 : 2))) quanti
     }
 }
 
+// ------------------------------------------------- two-row groups, paired staging
+//
+// The streaming form for two-row groups with register-held pairs stages the
+// two rows interleaved: routed position p of the bulk (or outlier slot i)
+// is one 32-bit word, row 0's BF16 value in the low half and row 1's in the
+// high half. A routing thread then stores each channel of both rows with
+// one 32-bit store (two per channel pair instead of four 16-bit stores and
+// two row offsets), and an encoding thread takes one 32-block of both rows
+// from eight 128-bit loads: one packed abs-max chain gives both rows' block
+// maxima, and the E2M1 conversion unpacks the low or high halves exactly as
+// it would unpack a row's packed pairs. A staged block of the pair is 32
+// words plus 16 bytes of padding (144 bytes: an odd number of 16-byte units,
+// so the 16-byte reads of consecutive blocks hit distinct banks); the
+// outlier slots follow the nb blocks.
+constexpr int IP_BLOCK = 144;
+__host__ __device__ constexpr int qa_ip_bytes(int nb, int kp) { return nb * IP_BLOCK + kp * 4; }
+
+// Eight BF16 values, the low (HI = false) or high (HI = true) halves of
+// eight consecutive staged words, scaled by `inv` (a power of two, or the
+// NVFP4 element multiplier) -> eight E2M1 codes, element i in nibble i.
+template <bool HI>
+__device__ __forceinline__ uint32_t encode8_halves(const uint32_t* w, float inv) {
+    auto f = [](uint32_t x) { return __uint_as_float(HI ? (x & 0xFFFF0000u) : (x << 16)); };
+    const float2 iv = make_float2(inv, inv);
+    const float2 v0 = __fmul2_rn(make_float2(f(w[0]), f(w[1])), iv);
+    const float2 v1 = __fmul2_rn(make_float2(f(w[2]), f(w[3])), iv);
+    const float2 v2 = __fmul2_rn(make_float2(f(w[4]), f(w[5])), iv);
+    const float2 v3 = __fmul2_rn(make_float2(f(w[6]), f(w[7])), iv);
+    uint32_t out;
+    asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+        "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+        : "=r"(out)
+        : "f"(v0.x), "f"(v0.y), "f"(v1.x), "f"(v1.y), "f"(v2.x), "f"(v2.y), "f"(v3.x), "f"(v3.y));
+    return out;
+}
+
+// Encode staged block b of both rows of the pair (output rows t0, t0 + 1;
+// the second only when rows == 2). The block is read twice -- once for the
+// maxima, once, eight words at a time, for the codes -- so that the 32
+// words never need registers of their own next to the routing thread's
+// register-held pairs.
+template <int MODE>
+__device__ __forceinline__ void encode_pair_block(const QuantParams& p, uint32_t sbuf, int t0, int rows, int b) {
+    const uint32_t src = sbuf + b * IP_BLOCK;
+    using mx::bf16x2_absmax;
+    uint32_t mq[2];  // packed maxima of positions 0-15 and 16-31 (row 0 low, row 1 high)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 v0 = ptx::ld_shared_v4(src + 64 * h), v1 = ptx::ld_shared_v4(src + 64 * h + 16),
+                    v2 = ptx::ld_shared_v4(src + 64 * h + 32), v3 = ptx::ld_shared_v4(src + 64 * h + 48);
+        mq[h] = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(v0.x, v0.y), bf16x2_absmax(v0.z, v0.w)),
+                              bf16x2_absmax(bf16x2_absmax(v1.x, v1.y), bf16x2_absmax(v1.z, v1.w)));
+        mq[h] = bf16x2_absmax(mq[h], bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(v2.x, v2.y), bf16x2_absmax(v2.z, v2.w)),
+                                                   bf16x2_absmax(bf16x2_absmax(v3.x, v3.y), bf16x2_absmax(v3.z, v3.w))));
+    }
+    // element multipliers of each row for positions 0-15 and 16-31
+    float f0[2], f1[2];
+    const size_t cstride = static_cast<size_t>(p.Kbp >> 1);
+    uint8_t* codes0 = p.codes + static_cast<size_t>(t0) * cstride + b * 16;
+    if constexpr (MODE == QA_NV) {
+        const uint32_t s0 = mx::nv_block_scales(mq[0] & 0x7FFFu, mq[1] & 0x7FFFu, p.nv_k, p.nv_p2g, &f0[0], &f0[1]);
+        const uint32_t s1 = mx::nv_block_scales((mq[0] >> 16) & 0x7FFFu, (mq[1] >> 16) & 0x7FFFu, p.nv_k, p.nv_p2g,
+                                                &f1[0], &f1[1]);
+        *reinterpret_cast<uint16_t*>(p.scales + sf_offset(t0, 2 * b, p.katoms)) = static_cast<uint16_t>(s0);
+        if (rows == 2)
+            *reinterpret_cast<uint16_t*>(p.scales + sf_offset(t0 + 1, 2 * b, p.katoms)) = static_cast<uint16_t>(s1);
+    } else {
+        const uint32_t m = bf16x2_absmax(mq[0], mq[1]);
+        const bool real = b * 32 < p.Kb;
+        const int X0 = mx::bf16_block_exponent(m & 0x7FFFu, &f0[0]);
+        const int X1 = mx::bf16_block_exponent((m >> 16) & 0x7FFFu, &f1[0]);
+        f0[1] = f0[0];
+        f1[1] = f1[0];
+        p.scales[sf_offset(t0, b, p.katoms)] = static_cast<uint8_t>(real ? X0 + 127 : 0);
+        if (rows == 2) p.scales[sf_offset(t0 + 1, b, p.katoms)] = static_cast<uint8_t>(real ? X1 + 127 : 0);
+    }
+    uint32_t c0[4], c1[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 a = ptx::ld_shared_v4(src + 32 * q), d = ptx::ld_shared_v4(src + 32 * q + 16);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, d.x, d.y, d.z, d.w};
+        c0[q] = encode8_halves<false>(w, f0[q >> 1]);
+        c1[q] = encode8_halves<true>(w, f1[q >> 1]);
+    }
+    *reinterpret_cast<uint4*>(codes0) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+    if (rows == 2) *reinterpret_cast<uint4*>(codes0 + cstride) = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+}
+
+// Outlier slots 8c .. 8c + 7 of both rows (32 staged bytes) -> two 16-byte
+// stores (NVFP4: scaled by 2^-g_act).
+template <int MODE>
+__device__ __forceinline__ void copy_pair_slots(const QuantParams& p, uint32_t sbuf, int nb, int t0, int rows, int c) {
+    const uint32_t src = sbuf + nb * IP_BLOCK + c * 32;
+    const uint4 a = ptx::ld_shared_v4(src), d = ptx::ld_shared_v4(src + 16);
+    uint4 r0 = make_uint4(__byte_perm(a.x, a.y, 0x5410), __byte_perm(a.z, a.w, 0x5410), __byte_perm(d.x, d.y, 0x5410),
+                          __byte_perm(d.z, d.w, 0x5410));
+    if constexpr (MODE == QA_NV) r0 = mx::scale_bf16x8(r0, p.hp_scale);
+    *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(t0) * p.kp + c * 8) = r0;
+    if (rows == 2) {
+        uint4 r1 = make_uint4(__byte_perm(a.x, a.y, 0x7632), __byte_perm(a.z, a.w, 0x7632),
+                              __byte_perm(d.x, d.y, 0x7632), __byte_perm(d.z, d.w, 0x7632));
+        if constexpr (MODE == QA_NV) r1 = mx::scale_bf16x8(r1, p.hp_scale);
+        *reinterpret_cast<uint4*>(p.hp + static_cast<size_t>(t0 + 1) * p.kp + c * 8) = r1;
+    }
+}
+
+// The streaming kernel for two-row groups with register-held pairs (the
+// structure of quantize_act_stream_kernel: persistent CTAs, a ring of S raw
+// slots filled by one bulk copy per group, bounded waits) on the paired
+// staging. FP as for quantize_act_stream_kernel.
+template <int S, int NT, int TR, int MODE, int FP>
+__global__ void __launch_bounds__(NT, (NT <= 256 ? 3 : 2)) quantize_act_pair_kernel(QuantParams p) {
+    constexpr int R = 2;
+    constexpr bool HPF = MODE == QA_MX_F16;
+    static_assert(TR > 0, "the paired form keeps its pairs in registers");
+    ptx::grid_dep_launch();  // the dual_gemm that follows may start its prologue
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int nb = p.Kbp >> 5;
+    const int raw_bytes = R * p.K * 2;
+    uint8_t* raw = smem;
+    uint8_t* sbuf = smem + S * raw_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + ((qa_ip_bytes(nb, p.kp) + 7) & ~7));
+    __shared__ int never;  // a flag nothing sets
+    const int tid = threadIdx.x;
+    const int ngroups = (p.M + R - 1) / R;
+    const int mine = blockIdx.x < ngroups ? (ngroups - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+
+    auto issue = [&](int i) {
+        const int g = blockIdx.x + i * gridDim.x;
+        const int rows = min(R, p.M - g * R);
+        const uint32_t bar = ptx::smem_u32(&full[i % S]);
+        const uint32_t bytes = static_cast<uint32_t>(rows) * p.K * 2u;
+        ptx::mbar_arrive_expect_tx(bar, bytes + p.extra_tx);
+        ptx::bulk_load(ptx::smem_u32(raw + (i % S) * raw_bytes), p.X + static_cast<size_t>(g) * R * p.K, bytes, bar);
+    };
+    // staged word of a position given by its offset in one unpaired staged row
+    // ([blocks of 80 bytes | outlier slots], as the plan's route table)
+    auto ip_off = [&](int off) -> int {
+        if (off < nb * QA_BLOCK_BYTES) {
+            const int b = off / QA_BLOCK_BYTES;
+            return b * IP_BLOCK + ((off - b * QA_BLOCK_BYTES) >> 1) * 4;
+        }
+        return nb * IP_BLOCK + ((off - nb * QA_BLOCK_BYTES) >> 1) * 4;
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+        never = 0;
+        ptx::fence_mbar_init();
+    }
+    // the padding positions (bulk [Kb, Kbp), slots [k, kp)) of both rows are
+    // never written by the routing step: zero them once
+    {
+        const int npb = p.Kbp - p.Kb, npad = npb + (p.kp - p.k);
+        for (int c = tid; c < npad; c += NT) {
+            const int pos = p.Kb + c;
+            const int off = c < npb ? (pos >> 5) * IP_BLOCK + (pos & 31) * 4 : nb * IP_BLOCK + (p.k + c - npb) * 4;
+            *reinterpret_cast<uint32_t*>(sbuf + off) = 0u;
+        }
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int i = 0; i < S && i < mine; ++i) issue(i);
+
+    const int npairs = p.K >> 1;
+    const float2* is2 = reinterpret_cast<const float2*>(p.inv_s);
+    const int2* rt2 = reinterpret_cast<const int2*>(p.route);
+    const uint32_t raw_u32 = ptx::smem_u32(raw), sbuf_u32 = ptx::smem_u32(sbuf);
+    const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
+    // each thread keeps its pairs' inv_s and the staged addresses of their
+    // two channels in registers for all its groups
+    float2 tsv[TR];
+    uint2 tad[TR];
+    uint32_t tmask[TR];  // FP16 outlier branch: halves that are outlier slots
+#pragma unroll
+    for (int j = 0; j < TR; ++j) {
+        const int c = tid + j * NT;
+        tsv[j] = c < npairs ? __ldg(is2 + c) : make_float2(0.f, 0.f);
+        const int2 dv = c < npairs ? __ldg(rt2 + c) : make_int2(0, 0);
+        tad[j] = make_uint2(sbuf_u32 + ip_off(dv.x), sbuf_u32 + ip_off(dv.y));
+        tmask[j] = HPF ? slot_mask(dv, nb * QA_BLOCK_BYTES) : 0u;
+    }
+    const int hv = p.kp >> 3;
+    int issued = min(S, mine);
+    for (int i = 0; i < mine; ++i) {
+        const int g = blockIdx.x + i * gridDim.x;
+        const int rows = min(R, p.M - g * R);
+        const uint32_t bar = ptx::smem_u32(&full[i % S]);
+        const bool ok = ptx::mbar_wait_bounded(bar, static_cast<uint32_t>((i / S) & 1), p.wait_limit_ns, &never);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(p.status, OSM_STATUS_TIMEOUT);
+                // let every copy already issued land in this CTA's shared memory
+                for (int j = i; j < issued; ++j)
+                    if (!ptx::mbar_wait_bounded(ptx::smem_u32(&full[j % S]), static_cast<uint32_t>((j / S) & 1),
+                                                20000000ull, &never))
+                        ptx::spin_ns(1000000);
+            }
+            __syncthreads();
+            return;
+        }
+        const uint32_t src = raw_u32 + (i % S) * raw_bytes + tid * 4;  // this thread's first pair, row 0
+        // Routing: the loads of a chunk of CH pairs (both rows) are issued
+        // before any of its stores; a one-row group stages zeros as row 1.
+        auto route = [&](auto two) {
+            constexpr bool TWO = decltype(two)::value;
+            constexpr int CH = FP == 0 ? 1 : (TR <= 6 ? TR : (TR + 1) / 2);
+#pragma unroll
+            for (int j0 = 0; j0 < TR; j0 += CH) {
+                uint32_t x0[CH], x1[CH];
+#pragma unroll
+                for (int jj = 0; jj < CH; ++jj) {
+                    const int j = j0 + jj;
+                    if (j < TR && (FP == 2 || (FP == 1 && j < TR - 1) || tid + j * NT < npairs)) {
+                        x0[jj] = ptx::ld_shared_u32(src + j * NT * 4);
+                        x1[jj] = TWO ? ptx::ld_shared_u32(src + row_bytes + j * NT * 4) : 0u;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < CH; ++jj) {
+                    const int j = j0 + jj;
+                    if (j < TR && (FP == 2 || (FP == 1 && j < TR - 1) || tid + j * NT < npairs)) {
+                        const uint32_t h0 = HPF ? smooth2_mixed(x0[jj], tsv[j], tmask[j]) : smooth2(x0[jj], tsv[j]);
+                        const uint32_t h1 = HPF ? smooth2_mixed(x1[jj], tsv[j], tmask[j]) : smooth2(x1[jj], tsv[j]);
+                        ptx::st_shared_u32(tad[j].x, __byte_perm(h0, h1, 0x5410));
+                        ptx::st_shared_u32(tad[j].y, __byte_perm(h0, h1, 0x7632));
+                    }
+                }
+            }
+        };
+        if (rows == R) route(std::true_type{});
+        else route(std::false_type{});
+        __syncthreads();  // raw slot consumed, staged rows complete
+        if (tid == 0 && issued < mine) issue(issued++);
+        for (int b = tid; b < nb; b += NT) encode_pair_block<MODE>(p, sbuf_u32, g * R, rows, b);
+        for (int c = NT - 1 - tid; c < hv; c += NT) copy_pair_slots<MODE>(p, sbuf_u32, nb, g * R, rows, c);
+        if (g * R <= p.M - 1 && p.M - 1 < g * R + rows) zero_padding_scale_rows(p);
+        __syncthreads();  // staged rows free for the next group
+    }
+}
+
+template <int S>
+size_t pair_smem_bytes(int K, int nb, int kp) {
+    return static_cast<size_t>(S) * 2 * K * 2 + ((qa_ip_bytes(nb, kp) + 7) & ~7) + 8 * S;
+}
+
 template <int R, int S>
 size_t stream_smem_bytes(int K, int stride) {
     return static_cast<size_t>(S) * R * K * 2 + static_cast<size_t>(R) * stride + 8 * S;
@@ -949,6 +1199,29 @@ static int launch_stream(const QuantParams& p, int mode, int stride, cudaStream_
     return check_cuda(cudaGetLastError(), "quantize_act launch");
 }
 
+template <int S, int NT, int TR>
+static int launch_pair(const QuantParams& p, int mode, cudaStream_t st) {
+    const size_t smem = pair_smem_bytes<S>(p.K, p.Kbp >> 5, p.kp);
+    const int np = p.K / 2;
+    const int fp = np == TR * NT ? 2 : (np >= (TR - 1) * NT ? 1 : 0);
+    auto pick = [&](auto f) {
+        constexpr int F = decltype(f)::value;
+        return mode == QA_NV ? quantize_act_pair_kernel<S, NT, TR, QA_NV, F>
+                             : (mode == QA_MX_F16 ? quantize_act_pair_kernel<S, NT, TR, QA_MX_F16, F>
+                                                  : quantize_act_pair_kernel<S, NT, TR, QA_MX, F>);
+    };
+    auto kern = fp == 2 ? pick(std::integral_constant<int, 2>{})
+                        : (fp == 1 ? pick(std::integral_constant<int, 1>{}) : pick(std::integral_constant<int, 0>{}));
+    int per_sm = 0, sms = 0;
+    int rc = prepare_kernel(reinterpret_cast<const void*>(kern), NT, smem, &per_sm, &sms);
+    if (rc) return rc;
+    if (per_sm < 1) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: no CTA fits");
+    const int64_t groups = ceil_div(p.M, 2);
+    const int64_t grid = groups < static_cast<int64_t>(sms) * per_sm ? groups : static_cast<int64_t>(sms) * per_sm;
+    kern<<<static_cast<unsigned>(grid), NT, smem, st>>>(p);
+    return check_cuda(cudaGetLastError(), "quantize_act launch");
+}
+
 int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_t* codes,
                         uint8_t* scales, uint16_t* hp, cudaStream_t st) {
     if (M > 0x7FFFFFFF) return fail(OSM_ERR_UNSUPPORTED, "quantize_act: M too large");
@@ -970,9 +1243,9 @@ int launch_quantize_act(const osm_plan* pl, const uint16_t* X, int64_t M, uint8_
         // slots (23.6 against 24.6 us for 4096 x 5120), whose deeper ring
         // matters when each CTA sees only a few row groups.
         if (p.M >= 8192 && npairs <= 10 * 256 && stream_smem_bytes<2, 2>(p.K, stride) * 3 <= 220 * 1024)
-            return launch_stream<2, 2, 256, 10>(p, mode, stride, st);
-        if (npairs == 5 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 5>(p, mode, stride, st);
-        if (npairs <= 6 * STREAM_NT) return launch_stream<2, 3, STREAM_NT, 6>(p, mode, stride, st);
+            return launch_pair<2, 256, 10>(p, mode, st);
+        if (npairs == 5 * STREAM_NT) return launch_pair<3, STREAM_NT, 5>(p, mode, st);
+        if (npairs <= 6 * STREAM_NT) return launch_pair<3, STREAM_NT, 6>(p, mode, st);
         return launch_stream<2, 3, STREAM_NT, 0>(p, mode, stride, st);
     }
     if (stream_smem_bytes<1, 3>(p.K, stride) <= two_per_sm) return launch_stream<1, 3, STREAM_NT, 0>(p, mode, stride, st);
