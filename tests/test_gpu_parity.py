@@ -213,3 +213,34 @@ def test_quantize_act_large_batches_ragged_last_group(M):
     assert_bitexact("a_scales", sc[:M], scales)
     assert np.all(sc[M:] == 0), "padding rows of a_scales must be 0"
     assert_bitexact("a_hp", to_np_u16(ah).reshape(M, plan.kp), hp)
+
+
+
+@pytest.mark.parametrize("fmt", ["fp16_outliers", "nvfp4"])
+def test_quantize_act_large_batch_other_encodings(fmt):
+    # The three-CTA paired form at K = 5120 with the FP16 outlier slots and
+    # with the NVFP4 bulk encoding (E4M3 scales per 16, the per-tensor
+    # exponent), odd M: bit-exact against the oracle on every row.
+    M, K, k = 8193, 5120, 128
+    X = synth.acts_heavy_tailed(M, K, 777, frac=0.02)
+    W = synth.weights_gaussian(K, 256, 778, sigma=0.04)
+    amax, wmax = oracle.act_amax(X), oracle.weight_amax(W)
+    s, inv_s, O = oracle.calibrate(amax, wmax, 0.6, k)
+    if fmt == "nvfp4":
+        g_act, g_w = oracle.nvfp4_plan_exponents(amax, wmax, s, inv_s, O)
+        plan = osm.Plan(K, 256, k, s, O, osm.WSCALE_1x32, fmt=osm.FMT_NVFP4, g_act=g_act, g_w=g_w)
+        codes, scales, hp = oracle.quantize_act_nv(X, inv_s, O, g_act)
+    else:
+        plan = osm.Plan(K, 256, k, s, O, osm.WSCALE_1x32, hp_fp16=True)
+        codes, scales, hp = oracle.quantize_act(X, inv_s, O, hp_fp16=True)
+    Xd = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).cuda().view(torch.bfloat16)
+    ac, asc, ah = plan.alloc_packed(M)
+    osm.quantize_act(plan, Xd, ac, asc, ah)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    nb = plan.nblocks
+    assert_bitexact("a_codes", ac.cpu().numpy().reshape(M, plan.Kbp // 2), codes)
+    sc = unswizzle(asc.cpu().numpy(), M, nb)
+    assert_bitexact("a_scales", sc[:M], scales)
+    assert np.all(sc[M:] == 0), "padding rows of a_scales must be 0"
+    assert_bitexact("a_hp", to_np_u16(ah).reshape(M, plan.kp), hp)
