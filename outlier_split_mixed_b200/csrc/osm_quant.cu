@@ -308,8 +308,11 @@ __device__ __forceinline__ void load_folded_rows(const PackParams& p, int64_t n0
 // lanes); 128x1: the maximum over the strip's four blocks (four warps, via
 // shared memory). NV: the 32 positions are two NVFP4 16-blocks, each with
 // its own E4M3 scale and element multiplier.
+// Five CTAs per SM (48 registers): the tile loads of more CTAs are in
+// flight at once (the kernel waits on memory latency: 83.4-85.8 -> 72.9-74.5
+// us for the 5120 x 13824 weights against four CTAs; six CTAs spill).
 template <bool NV>
-__global__ void __launch_bounds__(PK_THREADS) pack_bulk_tiled_kernel(PackParams p) {
+__global__ void __launch_bounds__(PK_THREADS, 5) pack_bulk_tiled_kernel(PackParams p) {
     __shared__ __align__(16) uint32_t tile[128][64];
     __shared__ uint32_t red[4][64];
     __shared__ uint32_t sxs[4][64];  // scale codes per quarter and pair: MX (n | n+1 << 8), NV (n: 2 bytes | n+1: 2 bytes)
