@@ -1077,12 +1077,13 @@ size_t stream_smem_bytes(int K, int stride) {
 int launch_act_amax(const uint16_t* X, int64_t T, int64_t K, float* amax, cudaStream_t st) {
     if (T == 0) return OSM_OK;
     // rows per CTA: AMAX_ROWS, or fewer (a multiple of 64) when that would
-    // leave the GPU with less than about two waves of CTAs (small batches:
-    // 4096 x 5120 took 15.1 us with 256 rows per CTA)
+    // leave the GPU with less than about one wave of resident CTAs (small
+    // batches: 4096 x 5120 took 15.1 us with 256 rows per CTA; one wave of
+    // 128-row CTAs beat two of 64 rows by 1.3 us)
     const int64_t groups = ceil_div(K / 8, 32);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t target = 2ll * sms * 6;
+    const int64_t target = static_cast<int64_t>(sms) * 6;
     int64_t rows = ceil_div(ceil_div(T * groups, target), 64) * 64;
     rows = rows < 64 ? 64 : (rows > AMAX_ROWS ? AMAX_ROWS : rows);
     dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(T, rows)));
