@@ -171,6 +171,22 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
         return;
     }
 
+    // inputs of the table rebuild (step 4), loaded one chunk ahead; with
+    // ranks the first chunk's are loaded before anything else
+    const bool use_rank = p.rank != nullptr && p.k > 0 && p.k < p.K;
+    auto fetch = [&](int c0, int32_t& rk, uint64_t& key, float& iv) {
+        const int j = c0 + tid;
+        if (j < p.K) {
+            if (use_rank) rk = p.rank[j];
+            else key = rf_key(sk, p.score, j);
+            iv = p.s_new[p.K + j];
+        }
+    };
+    int32_t rk_n = 0;
+    uint64_t key_n = 0;
+    float iv_n = 0.0f;
+    if (use_rank) fetch(0, rk_n, key_n, iv_n);
+
     // 2. Eq. (2), computed by refresh_smooth_kernel; stage the keys
     for (int j = tid; j < p.K; j += RF_THREADS) {
         p.s[j] = p.s_new[j];
@@ -236,21 +252,25 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
         thresh = prefix_sh;  // exact: keys are unique, so the k-th largest is one key
     }
 
-    // 4. ranks, J, O, route, order, inv_s in order
+    // 4. ranks, J, O, route, order, inv_s in order. Each chunk's inputs (the
+    // channel's rank or key and its inv_s) are loaded one chunk ahead, so
+    // that their latency overlaps the previous chunk's scan and stores.
     __syncthreads();
     const int nbp = p.Kbp / 32;
+    if (!use_rank) fetch(0, rk_n, key_n, iv_n);  // the keys are staged by now
     int base_o = 0, base_j = 0;
     for (int c0 = 0; c0 < p.K; c0 += RF_THREADS) {
         const int j = c0 + tid;
         const bool valid = j < p.K;
-        const int sel = !valid ? 0
-                        : (p.rank != nullptr && p.k > 0 && p.k < p.K) ? (p.rank[j] < p.k ? 1 : 0)
-                                                                       : (rf_key(sk, p.score, j) >= thresh ? 1 : 0);
+        const int32_t rk = rk_n;
+        const uint64_t key = key_n;
+        const float iv = iv_n;
+        if (c0 + RF_THREADS < p.K) fetch(c0 + RF_THREADS, rk_n, key_n, iv_n);
+        const int sel = !valid ? 0 : use_rank ? (rk < p.k ? 1 : 0) : (key >= thresh ? 1 : 0);
         const int r_o = block_exclusive_scan(sel, warp_tot, &total) + base_o;
         const int n_sel = total;
         const int r_j = base_j + tid - (r_o - base_o);  // unselected channels before j
         if (valid) {
-            const float iv = p.inv_s[j];
             if (sel) {
                 p.O[r_o] = j;
                 p.route[j] = nbp * QA_BLOCK_BYTES + 2 * r_o;
