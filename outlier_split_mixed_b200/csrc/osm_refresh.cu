@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(RF_THREADS) plan_refresh_kernel(RefreshParams 
     float iv_n = 0.0f;
     if (use_rank) fetch(0, rk_n, key_n, iv_n);
 
-    // 2. Eq. (2), computed by refresh_smooth_kernel; stage the keys
+    // 2. Eq. (2), computed by refresh_stats_kernel; stage the keys
     for (int j = tid; j < p.K; j += RF_THREADS) {
         p.s[j] = p.s_new[j];
         p.inv_s[j] = p.s_new[p.K + j];
